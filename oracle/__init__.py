@@ -1,0 +1,58 @@
+"""CPU oracle for hash-scored top-k sparse decode attention.
+
+TEST INFRASTRUCTURE. This package is the slow, plain, obviously-correct
+reference that the CUDA library is checked against. Only the test suite,
+``__graft_entry__.smoke()`` and the ``cpu_baseline`` / ``--impl reference``
+legs of ``bench.py`` may import it. The product path (the C-ABI library and
+its Python binding) never imports, calls or links anything here, and nothing
+here imports the product path.
+
+Everything is computed in float64 with numpy, one (batch, kv-head) pair at a
+time. Where numpy supplies a primitive (a matrix product, a stable sort) it
+is used as one step; there is no blocking, fusion or reordering beyond what
+the pages' definitions state.
+
+Sources, cited by page title and section:
+
+* SOCKET technical summary -- "SOCKET - SOft Collision Kernel EsTimator for
+  sparse attention" (gist.science/ja/paper/2602.06283), section
+  "中核メカニズム：ソフト LSH" (core mechanism: soft LSH), steps 1-4, and
+  section "理論的基盤" (theoretical foundation) for the tau -> 0 limit.
+* HATA digest -- "HATA: Hash-Aware Top-k Attention" (aibr.jp/archives/117328),
+  section 3 "中核となる技術的要素" (binary hash codes compared to rank keys).
+
+Functions with no independent pin: none. Every function here is pinned by a
+``-m "not gpu"`` test in ``tests/test_oracle_*.py`` against closed forms,
+invariants, library routines or brute force.
+"""
+
+from .socket_ref import (
+    hash_key_ids,
+    value_norms_f16,
+    bucket_probabilities,
+    group_bucket_table,
+    soft_collision_scores,
+    select_topk,
+    socket_decode_pair,
+    socket_decode,
+)
+from .attention_ref import exact_attention, attend_subset, dense_decode
+from .hata_ref import binary_codes, hamming_match_scores, hata_decode_pair, hata_decode
+
+__all__ = [
+    "hash_key_ids",
+    "value_norms_f16",
+    "bucket_probabilities",
+    "group_bucket_table",
+    "soft_collision_scores",
+    "select_topk",
+    "socket_decode_pair",
+    "socket_decode",
+    "exact_attention",
+    "attend_subset",
+    "dense_decode",
+    "binary_codes",
+    "hamming_match_scores",
+    "hata_decode_pair",
+    "hata_decode",
+]

@@ -1,0 +1,217 @@
+"""Python binding of libhash_scored_top.so (argument marshalling only).
+
+Every function here checks tensor devices, dtypes and shapes, passes raw
+pointers and sizes to the C entry point of the same name, and raises
+``RuntimeError`` with the library's message on a non-zero status. All
+compute happens in the library's CUDA kernels on the current torch stream;
+torch only provides device memory (outputs and workspaces) and the stream.
+There is no CPU fallback: if the library is missing the import of
+``_lib`` fails loudly.
+"""
+
+from __future__ import annotations
+
+import ctypes
+
+import torch
+
+from . import _lib
+
+SK_F32, SK_BF16 = 0, 1
+OP_HASH_KEYS, OP_SCORE, OP_TOPK, OP_SPARSE_ATTEND, OP_DECODE, OP_HATA_HASH, OP_HATA_DECODE, OP_DENSE_DECODE = range(8)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return SK_F32
+    if t.dtype == torch.bfloat16:
+        return SK_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (float32 or bfloat16)")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        raise RuntimeError(f"{what} failed (status {rc}): {_lib.last_error()}")
+
+
+def _want(t: torch.Tensor, dtype, shape, name):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _workspace(nbytes: int, device, ws):
+    if nbytes == 0:
+        return ws
+    if ws is None or ws.numel() * ws.element_size() < nbytes:
+        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    return ws
+
+
+def _ws_bytes(ws):
+    return 0 if ws is None else ws.numel() * ws.element_size()
+
+
+# ---------------------------------------------------------------- cache allocation / layout
+def empty_ids(B: int, Hkv: int, Ncap: int, L: int, device="cuda") -> torch.Tensor:
+    """Bucket-ID cache in the library's key-block interleaved layout [B, Hkv, Ncap/32, L, 32] uint8."""
+    return torch.zeros(B, Hkv, Ncap // 32, L, 32, dtype=torch.uint8, device=device)
+
+
+def empty_norms(B: int, Hkv: int, Ncap: int, device="cuda") -> torch.Tensor:
+    return torch.zeros(B, Hkv, Ncap, dtype=torch.float16, device=device)
+
+
+def empty_codes(B: int, Hkv: int, Ncap: int, device="cuda") -> torch.Tensor:
+    """Hard-hash code cache [B, Hkv, Ncap/32, 16, 32] uint8 (byte m of key n at [.., n//32, m, n%32])."""
+    return torch.zeros(B, Hkv, Ncap // 32, 16, 32, dtype=torch.uint8, device=device)
+
+
+def ids_to_natural(ids: torch.Tensor) -> torch.Tensor:
+    """[B, Hkv, Ncap/32, L, 32] -> [B, Hkv, Ncap, L] (a permutation of bytes, no arithmetic)."""
+    B, H, nb, L, _ = ids.shape
+    return ids.permute(0, 1, 2, 4, 3).reshape(B, H, nb * 32, L)
+
+
+def natural_to_ids(nat: torch.Tensor) -> torch.Tensor:
+    """[B, Hkv, Ncap, L] -> [B, Hkv, Ncap/32, L, 32] (inverse of ids_to_natural)."""
+    B, H, n, L = nat.shape
+    return nat.reshape(B, H, n // 32, 32, L).permute(0, 1, 2, 4, 3).contiguous()
+
+
+# ---------------------------------------------------------------- entry points
+def workspace_bytes(op: int, B, Hq, Hkv, Ncap, N, d, L=0, P=0, k=0) -> int:
+    n = _lib.lib.sk_workspace_bytes(op, B, Hq, Hkv, Ncap, N, d, L, P, k)
+    if n == ctypes.c_size_t(-1).value:
+        raise ValueError("invalid shapes for workspace query")
+    return n
+
+
+def socket_hash_keys(K, V, R, L: int, P: int, ids, norms, n_begin: int = 0, n_count: int | None = None):
+    """SOCKET step 1 for keys [n_begin, n_begin + n_count) of every pair (see the C header)."""
+    B, Hkv, Ncap, d = K.shape
+    n_count = Ncap - n_begin if n_count is None else n_count
+    _want(V, K.dtype, K.shape, "V")
+    _want(R, torch.bfloat16, (L * P, d), "R")
+    _want(ids, torch.uint8, (B, Hkv, Ncap // 32, L, 32), "ids")
+    _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
+    rc = _lib.lib.socket_hash_keys(_ptr(K), _ptr(V), _dtype_code(K), _ptr(R), B, Hkv, Ncap, n_begin, n_count, d, L, P,
+                                   _ptr(ids), _ptr(norms), _stream())
+    _check(rc, "socket_hash_keys")
+
+
+def socket_score(Q, R, ids, norms, N: int, L: int, P: int, tau: float, scores, ws=None):
+    """SOCKET steps 2-3: scores [B, Hkv, Ncap] f32 for keys < N."""
+    B, Hq, d = Q.shape
+    _, Hkv, nb, L_, _ = ids.shape
+    Ncap = nb * 32
+    _want(scores, torch.float32, (B, Hkv, Ncap), "scores")
+    _want(R, torch.bfloat16, (L * P, d), "R")
+    ws = _workspace(workspace_bytes(OP_SCORE, B, Hq, Hkv, Ncap, N, d, L, P, 0), Q.device, ws)
+    rc = _lib.lib.socket_score(_ptr(Q), _dtype_code(Q), _ptr(R), _ptr(ids), _ptr(norms), B, Hq, Hkv, Ncap, N, d, L, P,
+                               ctypes.c_float(tau), _ptr(scores), _ptr(ws), _ws_bytes(ws), _stream())
+    _check(rc, "socket_score")
+
+
+def socket_topk(scores, N: int, k: int, idx):
+    """SOCKET step 4 (selection): idx [B, Hkv, k] int32 ascending."""
+    B, Hkv, Ncap = scores.shape
+    _want(scores, torch.float32, scores.shape, "scores")
+    _want(idx, torch.int32, (B, Hkv, k), "idx")
+    rc = _lib.lib.socket_topk(_ptr(scores), B, Hkv, Ncap, N, k, _ptr(idx), None, 0, _stream())
+    _check(rc, "socket_topk")
+
+
+def socket_sparse_attend(Q, K, V, idx, scale: float, O, ws=None):
+    """SOCKET step 4 (attention over idx): O [B, Hq, d] f32."""
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = K.shape
+    k = idx.shape[-1]
+    _want(K, Q.dtype, K.shape, "K")
+    _want(V, Q.dtype, K.shape, "V")
+    _want(idx, torch.int32, (B, Hkv, k), "idx")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    ws = _workspace(workspace_bytes(OP_SPARSE_ATTEND, B, Hq, Hkv, Ncap, k, d, 0, 0, k), Q.device, ws)
+    rc = _lib.lib.socket_sparse_attend(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(idx), B, Hq, Hkv, Ncap, d, k,
+                                       ctypes.c_float(scale), _ptr(O), _ptr(ws), _ws_bytes(ws), _stream())
+    _check(rc, "socket_sparse_attend")
+
+
+def socket_decode(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k: int, scale: float, O, idx_out=None,
+                  ws=None):
+    """The fused decode step (SOCKET steps 2-4)."""
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = K.shape
+    _want(K, Q.dtype, K.shape, "K")
+    _want(V, Q.dtype, K.shape, "V")
+    _want(R, torch.bfloat16, (L * P, d), "R")
+    _want(ids, torch.uint8, (B, Hkv, Ncap // 32, L, 32), "ids")
+    _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    if idx_out is not None:
+        _want(idx_out, torch.int32, (B, Hkv, k), "idx_out")
+    ws = _workspace(workspace_bytes(OP_DECODE, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    rc = _lib.lib.socket_decode(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R), _ptr(ids), _ptr(norms), B, Hq, Hkv,
+                                Ncap, N, d, L, P, ctypes.c_float(tau), k, ctypes.c_float(scale), _ptr(O),
+                                _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
+    _check(rc, "socket_decode")
+
+
+def hata_hash_keys(K, R128, codes, n_begin: int = 0, n_count: int | None = None):
+    """128-bit sign codes of keys [n_begin, n_begin + n_count) of every pair."""
+    B, Hkv, Ncap, d = K.shape
+    n_count = Ncap - n_begin if n_count is None else n_count
+    _want(R128, torch.bfloat16, (128, d), "R128")
+    _want(codes, torch.uint8, (B, Hkv, Ncap // 32, 16, 32), "codes")
+    rc = _lib.lib.hata_hash_keys(_ptr(K), _dtype_code(K), _ptr(R128), B, Hkv, Ncap, n_begin, n_count, d, _ptr(codes),
+                                 _stream())
+    _check(rc, "hata_hash_keys")
+
+
+def hata_decode(Q, K, V, R128, codes, N: int, k: int, scale: float, O, idx_out=None, ws=None):
+    """Hard-hash decode step: Hamming scores, exact top-k, attention over the selection."""
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = K.shape
+    _want(K, Q.dtype, K.shape, "K")
+    _want(V, Q.dtype, K.shape, "V")
+    _want(R128, torch.bfloat16, (128, d), "R128")
+    _want(codes, torch.uint8, (B, Hkv, Ncap // 32, 16, 32), "codes")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    if idx_out is not None:
+        _want(idx_out, torch.int32, (B, Hkv, k), "idx_out")
+    rc = _lib.lib.hata_decode(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R128), _ptr(codes), B, Hq, Hkv, Ncap, N,
+                              d, k, ctypes.c_float(scale), _ptr(O), _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
+    _check(rc, "hata_decode")
+
+
+def dense_decode(Q, K, V, N: int, scale: float, O, ws=None):
+    """Dense decode attention over the first N cached keys."""
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = K.shape
+    _want(K, Q.dtype, K.shape, "K")
+    _want(V, Q.dtype, K.shape, "V")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    ws = _workspace(workspace_bytes(OP_DENSE_DECODE, B, Hq, Hkv, Ncap, N, d), Q.device, ws)
+    rc = _lib.lib.dense_decode(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), B, Hq, Hkv, Ncap, N, d, ctypes.c_float(scale),
+                               _ptr(O), _ptr(ws), _ws_bytes(ws), _stream())
+    _check(rc, "dense_decode")
+
+
+def check_status():
+    """Synchronises the current stream and raises if a kernel flagged an error."""
+    _check(_lib.lib.sk_check_status(_stream()), "sk_check_status")

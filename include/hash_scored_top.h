@@ -1,0 +1,194 @@
+/*
+ * hash_scored_top.h -- C ABI of libhash_scored_top.so: hash-scored top-k sparse
+ * decode attention on NVIDIA B200 (sm_100a).
+ *
+ * The method is SOCKET (technical summary "SOCKET - SOft Collision Kernel
+ * EsTimator for sparse attention", gist.science/ja/paper/2602.06283, section
+ * 中核メカニズム：ソフト LSH, steps 1-4), plus a hard-hash (Hamming) variant
+ * after the HATA digest ("HATA: Hash-Aware Top-k Attention",
+ * aibr.jp/archives/117328, section 3). Each entry point below names the step
+ * it implements.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - All tensor arguments are DEVICE pointers to contiguous memory owned by
+ *   the caller. The library allocates nothing and frees nothing; scratch
+ *   memory is passed in as `ws` / `ws_bytes` (query the size with
+ *   sk_workspace_bytes). `stream` is a cudaStream_t (NULL = legacy default).
+ * - Calls are asynchronous on `stream`. Arguments are validated on the host
+ *   before anything is launched; on failure nothing is launched, a non-zero
+ *   sk_status is returned and sk_last_error() describes it. A failed launch
+ *   returns SK_ERR_CUDA with the CUDA error text in sk_last_error().
+ * - Results are deterministic: repeated calls on the same inputs give
+ *   bit-identical outputs (no floating-point atomics touch result values).
+ * - Shapes: B batch, Hq query heads, Hkv KV heads (Hq % Hkv == 0, group size
+ *   G = Hq / Hkv, query head h reads KV head h / G), d head dim (64 or 128),
+ *   Ncap cache capacity in keys (multiple of 32), N <= Ncap keys in use,
+ *   L hash tables of P hyperplanes each (2^P buckets per table), k keys kept.
+ *   A "pair" is one (batch, KV head); pair p = b * Hkv + kvh.
+ *
+ * Memory layouts
+ * --------------
+ *   Q      [B][Hq][d]          dtype `kv` (f32 or bf16)
+ *   K, V   [B][Hkv][Ncap][d]   dtype `kv`
+ *   O      [B][Hq][d]          f32
+ *   R      [L*P][d]            bf16; row l*P + j is hyperplane j of table l
+ *   R128   [128][d]            bf16; hyperplanes of the 128-bit hard-hash codes
+ *   norms  [B][Hkv][Ncap]      f16; cached |v| of each key
+ *   ids    per pair, key-block interleaved: the bucket ID of key n in table l
+ *          of pair p is byte  p*Ncap*L + (n/32)*32*L + l*32 + (n%32)  (uint8;
+ *          P <= 8, so a table has at most 256 buckets).
+ *   codes  per pair, key-block interleaved like ids with 16 "tables": byte m
+ *          of the 128-bit code of key n of pair p is at
+ *          p*Ncap*16 + (n/32)*512 + m*32 + (n%32); code bit c is bit c%8 of
+ *          byte c/8.
+ *   scores [B][Hkv][Ncap]      f32 (only the first N per pair are written)
+ *   idx    [B][Hkv][k]         int32, ascending key indices
+ */
+#ifndef HASH_SCORED_TOP_H
+#define HASH_SCORED_TOP_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { SK_F32 = 0, SK_BF16 = 1 } sk_dtype;
+
+typedef enum {
+  SK_OK = 0,
+  SK_ERR_INVALID_ARG = 1,  /* bad shape, null pointer, out-of-range parameter */
+  SK_ERR_UNSUPPORTED = 2,  /* valid but not implemented (e.g. d not 64/128)  */
+  SK_ERR_CUDA = 3,         /* a CUDA call or launch failed                    */
+  SK_ERR_TIMEOUT = 4,      /* a device-side bounded wait gave up              */
+  SK_ERR_WORKSPACE = 5     /* ws is NULL or smaller than required             */
+} sk_status;
+
+/* Operation codes for sk_workspace_bytes. */
+typedef enum {
+  SK_OP_HASH_KEYS = 0,
+  SK_OP_SCORE = 1,
+  SK_OP_TOPK = 2,
+  SK_OP_SPARSE_ATTEND = 3,
+  SK_OP_DECODE = 4,
+  SK_OP_HATA_HASH = 5,
+  SK_OP_HATA_DECODE = 6,
+  SK_OP_DENSE_DECODE = 7
+} sk_op;
+
+/*
+ * Prefill hashing, SOCKET step 1: for keys n in [n_begin, n_begin + n_count)
+ * of every pair, writes the L bucket IDs (bit j of table l's ID is
+ * [k_n . r_{l*P+j} > 0], least significant bit first) and the value norm
+ * |v_n| rounded to the nearest f16 (ties to even).
+ * K, V: [B][Hkv][Ncap][d] (dtype kv); R: [L*P][d] bf16.
+ * ids, norms: outputs in the layouts above. Keys outside the range are not
+ * touched, so appending one decoded token is n_begin = N, n_count = 1.
+ * The projections accumulate in f32; the norm in f64.
+ * Requires 1 <= P <= 8, 1 <= L <= 64, L*P <= 512, 0 <= n_begin,
+ * n_begin + n_count <= Ncap (n_count == 0 is a no-op).
+ */
+int socket_hash_keys(const void* K, const void* V, sk_dtype kv, const void* R, int B, int Hkv,
+                     int Ncap, int n_begin, int n_count, int d, int L, int P, void* ids,
+                     void* norms, void* stream);
+
+/*
+ * Soft collision scores, SOCKET steps 2-3: for every pair, the soft bucket
+ * assignment p_{h,l}(b) = softmax_b(sum_j s_bj * (q_hat_h . r_{l*P+j}) / tau)
+ * (s_bj = +1 if bit j of b is set, else -1; q_hat = q / |q|), summed over the
+ * G query heads of the pair, and then score_n = norm_n * sum_l T_l(id_l(n))
+ * for n < N. Q: [B][Hq][d] in dtype q. scores: [B][Hkv][Ncap] f32 output.
+ * The bucket tables go through ws: sk_workspace_bytes(SK_OP_SCORE, ...) bytes.
+ * Requires 1 <= P <= 8, 1 <= L <= 64, tau > 0.
+ */
+int socket_score(const void* Q, sk_dtype q, const void* R, const void* ids, const void* norms,
+                 int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau,
+                 float* scores, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Deterministic top-k, SOCKET step 4: per pair, the k largest of the first N
+ * scores (non-negative f32), ties going to the lower key index; writes the
+ * chosen indices in ascending order to idx [B][Hkv][k]. Requires 1 <= k <= N.
+ * ws: sk_workspace_bytes(SK_OP_TOPK, ...) bytes (may be 0 -> ws may be NULL).
+ */
+int socket_topk(const float* scores, int B, int Hkv, int Ncap, int N, int k, int* idx, void* ws,
+                size_t ws_bytes, void* stream);
+
+/*
+ * Exact attention over the selected subset, SOCKET step 4: for every query
+ * head h of pair p, O_h = softmax_i(q_h . k_i * scale) v_i over i in idx[p]
+ * (renormalised over the subset), with f32 accumulation. Entries of idx must
+ * lie in [0, Ncap). ws: sk_workspace_bytes(SK_OP_SPARSE_ATTEND, ...) bytes.
+ * Requires 1 <= G <= 8 for bf16 K/V.
+ */
+int socket_sparse_attend(const void* Q, const void* K, const void* V, sk_dtype kv, const int* idx,
+                         int B, int Hq, int Hkv, int Ncap, int d, int k, float scale, float* O,
+                         void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The fused decode step, SOCKET steps 2-4 in one launch: bucket table,
+ * scores, exact top-k and attention over the selection, one thread-block
+ * cluster per pair with the scores kept on chip. The result equals
+ * socket_score -> socket_topk -> socket_sparse_attend. idx_out (nullable)
+ * receives the selected indices [B][Hkv][k] ascending. Shapes the fused
+ * kernel cannot hold on chip run that unfused chain instead (same results).
+ * Requires 1 <= P <= 8, 1 <= L <= 64, 1 <= k <= N, tau > 0.
+ * ws: sk_workspace_bytes(SK_OP_DECODE, ...) bytes.
+ */
+int socket_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R,
+                  const void* ids, const void* norms, int B, int Hq, int Hkv, int Ncap, int N,
+                  int d, int L, int P, float tau, int k, float scale, float* O, int* idx_out,
+                  void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Hard-hash codes (HATA digest, section 3, with seeded random hyperplanes
+ * standing in for the learned hash): for keys n in [n_begin, n_begin+n_count)
+ * of every pair, code bit c = [k_n . r_c > 0] for the 128 rows of R128,
+ * written to `codes` in the layout above.
+ */
+int hata_hash_keys(const void* K, sk_dtype kv, const void* R128, int B, int Hkv, int Ncap,
+                   int n_begin, int n_count, int d, void* codes, void* stream);
+
+/*
+ * Hard-hash decode step: query codes from R128, score_n = sum over the G
+ * query heads of (128 - popcount(code_q ^ code_n)), exact top-k (ties to the
+ * lower index) and exact attention over the selection, as socket_decode.
+ * ws: sk_workspace_bytes(SK_OP_HATA_DECODE, ...) bytes.
+ */
+int hata_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R128,
+                const void* codes, int B, int Hq, int Hkv, int Ncap, int N, int d, int k,
+                float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Dense decode attention over all N cached keys (the FlashAttention-style
+ * baseline the SOCKET page compares against, section 実験結果):
+ * O_h = softmax(q_h . K^T * scale) V, split over keys with an exact merge.
+ * ws: sk_workspace_bytes(SK_OP_DENSE_DECODE, ...) bytes.
+ */
+int dense_decode(const void* Q, const void* K, const void* V, sk_dtype kv, int B, int Hq, int Hkv,
+                 int Ncap, int N, int d, float scale, float* O, void* ws, size_t ws_bytes,
+                 void* stream);
+
+/* Scratch bytes needed by `op` for these shapes (0 if none). Arguments an
+ * op does not use are ignored. Returns (size_t)-1 for invalid shapes. */
+size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P,
+                          int k);
+
+/* Synchronises `stream`, then reports and clears the library's device error
+ * word: SK_ERR_TIMEOUT if a device-side bounded wait of an earlier kernel gave
+ * up, SK_ERR_UNSUPPORTED if a kernel found its shared-memory plan did not fit
+ * (it then wrote nothing); SK_ERR_CUDA on a pending CUDA error; else SK_OK. */
+int sk_check_status(void* stream);
+
+/* Thread-local description of the last non-OK return (never NULL). */
+const char* sk_last_error(void);
+
+/* Library version string. */
+const char* sk_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HASH_SCORED_TOP_H */

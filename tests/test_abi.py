@@ -1,0 +1,110 @@
+"""The C-ABI library loads, exports every entry point its header declares, and
+validates arguments on the host (no GPU needed: these paths launch nothing)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from tests.conftest import ROOT
+
+HEADER = os.path.join(ROOT, "include", "hash_scored_top.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s*([a-z_][a-z0-9_]*)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from hash_scored_top_b200 import build
+    build.build()
+    from hash_scored_top_b200 import _lib
+    return _lib
+
+
+def test_header_lists_the_path_entry_points():
+    names = _declared_functions()
+    for want in ("socket_hash_keys", "socket_score", "socket_topk", "socket_sparse_attend", "socket_decode",
+                 "hata_hash_keys", "hata_decode", "dense_decode", "sk_workspace_bytes", "sk_check_status",
+                 "sk_last_error", "sk_version"):
+        assert want in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    for name in _declared_functions():
+        assert hasattr(lib.lib, name), f"{name} declared in the header but not exported"
+        assert name in lib.SIGNATURES, f"{name} has no ctypes signature in the binding"
+    assert "sm_100a" in lib.version()
+
+
+def test_workspace_sizes(lib):
+    from hash_scored_top_b200 import api
+    # fused decode at the 100K-token Llama-8B-like shape needs no workspace
+    assert api.workspace_bytes(api.OP_DECODE, 4, 32, 8, 102400, 102400, 128, 32, 8, 3103) == 0
+    assert api.workspace_bytes(api.OP_SCORE, 4, 32, 8, 102400, 102400, 128, 32, 8, 0) == 32 * 65536
+    n = api.workspace_bytes(api.OP_SPARSE_ATTEND, 4, 32, 8, 102400, 102400, 128, 0, 0, 3103)
+    assert n == 32 * 13 * 4 * 130 * 4       # 13 splits of <= 256 keys, (m, l, o[128]) per head
+    assert api.workspace_bytes(api.OP_DENSE_DECODE, 1, 8, 8, 4096, 4096, 64) > 0
+    with pytest.raises(ValueError):
+        api.workspace_bytes(api.OP_DECODE, 1, 3, 2, 64, 64, 128, 8, 4, 8)     # Hq % Hkv != 0
+
+
+def _rc_and_msg(lib, fn, *args):
+    rc = fn(*args)
+    return rc, lib.last_error()
+
+
+def test_host_validation_rejects_without_launching(lib):
+    L = lib.lib
+    p = ctypes.c_void_p(16)          # never dereferenced: validation fails first
+    null = None
+    # socket_decode: NULL query
+    rc, msg = _rc_and_msg(lib, L.socket_decode, null, p, p, 1, p, p, p, 1, 4, 1, 64, 64, 128, 8, 4, 0.5, 8, 0.1, p,
+                          null, null, 0, null)
+    assert rc == 1 and "Q is NULL" in msg
+    # Hq not a multiple of Hkv
+    rc, msg = _rc_and_msg(lib, L.socket_decode, p, p, p, 1, p, p, p, 1, 3, 2, 64, 64, 128, 8, 4, 0.5, 8, 0.1, p,
+                          null, null, 0, null)
+    assert rc == 1 and "multiple" in msg
+    # unsupported head dim
+    rc, msg = _rc_and_msg(lib, L.socket_decode, p, p, p, 1, p, p, p, 1, 4, 1, 64, 64, 96, 8, 4, 0.5, 8, 0.1, p,
+                          null, null, 0, null)
+    assert rc == 2
+    # k > N
+    rc, msg = _rc_and_msg(lib, L.socket_decode, p, p, p, 1, p, p, p, 1, 4, 1, 64, 32, 128, 8, 4, 0.5, 33, 0.1, p,
+                          null, null, 0, null)
+    assert rc == 1 and "k=33" in msg
+    # P too large for byte IDs
+    rc, msg = _rc_and_msg(lib, L.socket_decode, p, p, p, 1, p, p, p, 1, 4, 1, 64, 64, 128, 8, 9, 0.5, 8, 0.1, p,
+                          null, null, 0, null)
+    assert rc == 2 and "P=9" in msg
+    # tau must be positive
+    rc, msg = _rc_and_msg(lib, L.socket_decode, p, p, p, 1, p, p, p, 1, 4, 1, 64, 64, 128, 8, 4, 0.0, 8, 0.1, p,
+                          null, null, 0, null)
+    assert rc == 1 and "tau" in msg
+    # Ncap not a multiple of 32
+    rc, msg = _rc_and_msg(lib, L.socket_hash_keys, p, p, 1, p, 1, 1, 40, 0, 40, 128, 8, 4, p, p, null)
+    assert rc == 1 and "Ncap" in msg
+    # key range outside the cache
+    rc, msg = _rc_and_msg(lib, L.socket_hash_keys, p, p, 1, p, 1, 1, 64, 60, 8, 128, 8, 4, p, p, null)
+    assert rc == 1 and "range" in msg
+    # score without a workspace
+    rc, msg = _rc_and_msg(lib, L.socket_score, p, 1, p, p, p, 1, 4, 1, 64, 64, 128, 8, 4, 0.5, p, null, 0, null)
+    assert rc == 5 and "workspace" in msg
+    # sparse attention with too small a workspace
+    rc, msg = _rc_and_msg(lib, L.socket_sparse_attend, p, p, p, 1, p, 1, 4, 1, 64, 128, 8, 0.1, p, p, 16, null)
+    assert rc == 5
+    # top-k with k = 0
+    rc, msg = _rc_and_msg(lib, L.socket_topk, p, 1, 1, 64, 64, 0, p, null, 0, null)
+    assert rc == 1
+    # hard-hash decode with a group of 16 heads
+    rc, msg = _rc_and_msg(lib, L.hata_decode, p, p, p, 1, p, p, 1, 16, 1, 64, 64, 128, 8, 0.1, p, null, null, 0, null)
+    assert rc == 2 and "G=16" in msg
+    # unknown dtype
+    rc, msg = _rc_and_msg(lib, L.dense_decode, p, p, p, 7, 1, 4, 1, 64, 64, 128, 0.1, p, p, 1 << 20, null)
+    assert rc == 1 and "dtype" in msg

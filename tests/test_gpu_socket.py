@@ -1,0 +1,272 @@
+"""GPU parity of the SOCKET path against the oracle, through the C ABI.
+
+Sizes here finish in seconds on the oracle and still span several tiles,
+several CTAs of a cluster and ragged tails. Full-size workloads are covered
+by test_gpu_fullsize.py on sampled pairs.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import attention_ref as ao
+from oracle import socket_ref as so
+from hash_scored_top_b200 import workloads as wl
+from tests import parity as pa
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module")
+def api():
+    from hash_scored_top_b200 import build
+    build.build()
+    from hash_scored_top_b200 import api as _api
+    return _api
+
+
+def _w(name):
+    return {
+        "tiny_f32": wl.TINY_F32,
+        "llama1b_ragged": wl.shrink(wl.LLAMA_1B, B=1, Hkv=2, Hq=8, N=9001, k=9001 // 33),
+        "llama8b_needles": wl.shrink(wl.LLAMA_8B, B=2, Hkv=2, Hq=8, N=12000, k=12000 // 33),
+        "qwen_l48_g8": wl.shrink(wl.QWEN3_30B, B=1, Hkv=2, Hq=16, N=10000, k=10000 // 50),
+        "d64_g1": wl.shrink(wl.LLAMA_1B, B=2, Hkv=1, Hq=1, N=3000, k=100, L=20, P=6, tau=0.4),
+        "g2_small_n": wl.shrink(wl.LLAMA_8B, B=1, Hkv=3, Hq=6, N=70, k=9, needles=0, L=5, P=3, tau=0.7),
+    }[name]
+
+
+def _cache(api, w, inp, pairs=None):
+    ids_nat, norms, proj = pa.oracle_socket_cache(inp, w, pairs)
+    ids, nrm = pa.to_device_cache(ids_nat, norms, DEV)
+    return ids, nrm, ids_nat, norms, proj
+
+
+# ---------------------------------------------------------------- step 1: hashing
+
+@pytest.mark.parametrize("name", ["tiny_f32", "llama1b_ragged", "qwen_l48_g8", "d64_g1"])
+def test_hash_keys_match_oracle(api, name):
+    w = _w(name)
+    inp = wl.make_inputs(w, DEV)
+    Ncap = inp["K"].shape[2]
+    ids = api.empty_ids(w.B, w.Hkv, Ncap, w.L, DEV)
+    norms = api.empty_norms(w.B, w.Hkv, Ncap, DEV)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, norms)
+    torch.cuda.synchronize()
+    gpu_nat = api.ids_to_natural(ids).cpu().numpy()
+    ref_nat, ref_norms, proj = pa.oracle_socket_cache(inp, w)
+    R = inp["R"].double().cpu().numpy()
+    total_robust = 0
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            K = inp["K"][b, h, : w.N].double().cpu().numpy()
+            robust = pa.sign_band(K, R, proj[(b, h)]).reshape(w.N, w.L, w.P).all(axis=2)
+            total_robust += int(robust.sum())
+            assert pa.check_ids(gpu_nat[b, h, : w.N], ref_nat[b, h, : w.N], robust) == 0
+            assert np.array_equal(norms[b, h, : w.N].cpu().numpy(), ref_norms[b, h, : w.N])
+    assert total_robust >= 0.99 * w.B * w.Hkv * w.N * w.L
+
+
+def test_hash_keys_append_touches_only_the_range(api):
+    w = _w("llama1b_ragged")
+    inp = wl.make_inputs(w, DEV)
+    Ncap = inp["K"].shape[2]
+    ids = api.empty_ids(w.B, w.Hkv, Ncap, w.L, DEV)
+    norms = api.empty_norms(w.B, w.Hkv, Ncap, DEV)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, norms, 0, w.N - 1)
+    before_ids, before_norms = ids.clone(), norms.clone()
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, norms, w.N - 1, 1)   # append one token
+    full_ids = api.empty_ids(w.B, w.Hkv, Ncap, w.L, DEV)
+    full_norms = api.empty_norms(w.B, w.Hkv, Ncap, DEV)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, full_ids, full_norms, 0, w.N)
+    torch.cuda.synchronize()
+    assert torch.equal(ids, full_ids) and torch.equal(norms, full_norms)
+    nat_b, nat_a = api.ids_to_natural(before_ids), api.ids_to_natural(ids)
+    assert torch.equal(nat_b[:, :, : w.N - 1], nat_a[:, :, : w.N - 1])
+    assert torch.equal(nat_a[:, :, w.N:], torch.zeros_like(nat_a[:, :, w.N:]))
+
+
+# ---------------------------------------------------------------- steps 2-3: scores
+
+@pytest.mark.parametrize("name", ["tiny_f32", "llama1b_ragged", "qwen_l48_g8", "d64_g1", "g2_small_n"])
+def test_scores_match_oracle(api, name):
+    w = _w(name)
+    inp = wl.make_inputs(w, DEV)
+    Ncap = inp["K"].shape[2]
+    ids, nrm, ids_nat, norms, _ = _cache(api, w, inp)
+    scores = torch.full((w.B, w.Hkv, Ncap), -7.0, device=DEV)
+    api.socket_score(inp["Q"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, scores)
+    torch.cuda.synchronize()
+    R = inp["R"].double().cpu().numpy()
+    worst = 0.0
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            Qg, _, _ = pa.pair_arrays(inp, w, b, h)
+            T = so.group_bucket_table(Qg, R, w.L, w.P, w.tau)
+            ref = so.soft_collision_scores(T, ids_nat[b, h, : w.N], norms[b, h, : w.N])
+            got = scores[b, h, : w.N].double().cpu().numpy()
+            worst = max(worst, float(np.max(np.abs(got - ref) / np.maximum(ref, 1e-30))))
+            assert np.all(scores[b, h, w.N:].cpu().numpy() == -7.0)      # tail untouched
+    assert worst <= pa.SCORE_REL_TOL, worst
+
+
+# ---------------------------------------------------------------- step 4: selection
+
+@pytest.mark.parametrize("N,ks,kind", [
+    (70, [1, 9, 69, 70], "ties"),
+    (5000, [1, 7, 165, 4999], "ties"),
+    (33001, [1, 1000, 33001], "random"),
+    (102400, [3103], "random"),
+    (4096, [1, 128, 4096], "equal"),
+])
+def test_topk_matches_oracle_exactly(api, N, ks, kind):
+    g = torch.Generator(device="cpu").manual_seed(N)
+    B, Hkv = 2, 2
+    Ncap = (N + 31) // 32 * 32
+    if kind == "ties":
+        s = torch.randint(0, 20, (B, Hkv, Ncap), generator=g).float() * 0.25
+    elif kind == "equal":
+        s = torch.full((B, Hkv, Ncap), 1.5)
+    else:
+        s = torch.rand(B, Hkv, Ncap, generator=g) * 10
+    scores = s.to(DEV)
+    for k in ks:
+        idx = torch.empty(B, Hkv, k, dtype=torch.int32, device=DEV)
+        api.socket_topk(scores, N, k, idx)
+        torch.cuda.synchronize()
+        for b in range(B):
+            for h in range(Hkv):
+                want = so.select_topk(s[b, h, :N].double().numpy(), k)
+                assert np.array_equal(idx[b, h].cpu().numpy(), want), (N, k, kind, b, h)
+
+
+# ---------------------------------------------------------------- step 4: attention over the subset
+
+@pytest.mark.parametrize("dtype,d,G,k", [
+    ("bf16", 128, 4, 1), ("bf16", 128, 4, 17), ("bf16", 128, 4, 1000), ("bf16", 128, 8, 300),
+    ("bf16", 64, 4, 129), ("bf16", 128, 1, 33), ("bf16", 64, 2, 250), ("f32", 128, 1, 128), ("f32", 64, 3, 77),
+])
+def test_sparse_attend_matches_oracle(api, dtype, d, G, k):
+    torch.manual_seed(k * 7 + d + G)
+    B, Hkv, N = 2, 2, 4096
+    dt = torch.bfloat16 if dtype == "bf16" else torch.float32
+    Q = torch.randn(B, Hkv * G, d).to(dt)
+    K = torch.randn(B, Hkv, N, d).to(dt)
+    V = torch.randn(B, Hkv, N, d).to(dt)
+    idx = torch.stack([torch.stack([torch.randperm(N)[:k].sort().values for _ in range(Hkv)]) for _ in range(B)])
+    O = torch.empty(B, Hkv * G, d, device=DEV)
+    api.socket_sparse_attend(Q.to(DEV), K.to(DEV), V.to(DEV), idx.int().to(DEV), d ** -0.5, O)
+    torch.cuda.synchronize()
+    tol = pa.BF16_TOL if dtype == "bf16" else pa.F32_TOL
+    for b in range(B):
+        for h in range(Hkv):
+            ref = ao.attend_subset(Q[b, h * G:(h + 1) * G].double().numpy(), K[b, h].double().numpy(),
+                                   V[b, h].double().numpy(), idx[b, h].numpy(), d ** -0.5)
+            err = pa.row_rel_err(O[b, h * G:(h + 1) * G].cpu().numpy(), ref)
+            assert err < tol, (err, b, h)
+
+
+# ---------------------------------------------------------------- fused decode
+
+def _decode_and_compare(api, w, inp, ids, nrm, ids_nat, norms, tol, use_chain=False):
+    Ncap = inp["K"].shape[2]
+    O = torch.empty(w.B, w.Hq, w.d, device=DEV)
+    idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=DEV)
+    if use_chain:
+        scores = torch.empty(w.B, w.Hkv, Ncap, device=DEV)
+        api.socket_score(inp["Q"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, scores)
+        api.socket_topk(scores, w.N, w.k, idx)
+        api.socket_sparse_attend(inp["Q"], inp["K"], inp["V"], idx, w.scale, O)
+    else:
+        api.socket_decode(inp["Q"], inp["K"], inp["V"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, w.k, w.scale, O, idx)
+    api.check_status()
+    R = inp["R"].double().cpu().numpy()
+    compared = 0
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            Qg, K, V = pa.pair_arrays(inp, w, b, h)
+            o_ref, idx_ref, s_ref = so.socket_decode_pair(Qg, K, V, R, ids_nat[b, h, : w.N], norms[b, h, : w.N],
+                                                          w.L, w.P, w.tau, w.k, w.scale)
+            got = idx[b, h].cpu().numpy()
+            assert pa.check_selection(s_ref, got, w.k) == [], (b, h)
+            if np.array_equal(got, idx_ref):
+                compared += 1
+                err = pa.row_rel_err(O[b, h * w.G:(h + 1) * w.G].cpu().numpy(), o_ref)
+                assert err < tol, (err, b, h)
+    assert compared >= max(1, (w.B * w.Hkv * 3) // 4)
+    return O, idx
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "llama1b_ragged", "llama8b_needles", "qwen_l48_g8", "d64_g1",
+                                  "g2_small_n"])
+def test_fused_decode_matches_oracle(api, name):
+    w = _w(name)
+    inp = wl.make_inputs(w, DEV)
+    ids, nrm, ids_nat, norms, _ = _cache(api, w, inp)
+    O, idx = _decode_and_compare(api, w, inp, ids, nrm, ids_nat, norms, pa.out_tol(w))
+    if w.needles:
+        for b in range(w.B):
+            for h in range(w.Hkv):
+                assert set(inp["needle_pos"][b, h].tolist()) <= set(idx[b, h].cpu().tolist())
+    # the unfused chain selects exactly the same keys
+    O2, idx2 = _decode_and_compare(api, w, inp, ids, nrm, ids_nat, norms, pa.out_tol(w), use_chain=True)
+    assert torch.equal(idx, idx2)
+
+
+def test_fused_decode_is_deterministic(api):
+    w = _w("llama8b_needles")
+    inp = wl.make_inputs(w, DEV)
+    ids, nrm, *_ = _cache(api, w, inp)
+    outs = []
+    for _ in range(3):
+        O = torch.empty(w.B, w.Hq, w.d, device=DEV)
+        idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=DEV)
+        api.socket_decode(inp["Q"], inp["K"], inp["V"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, w.k, w.scale, O, idx)
+        outs.append((O, idx))
+    torch.cuda.synchronize()
+    for O, idx in outs[1:]:
+        assert torch.equal(O, outs[0][0]) and torch.equal(idx, outs[0][1])
+
+
+@pytest.mark.parametrize("name", ["tiny_f32", "llama1b_ragged"])
+def test_decode_with_k_equal_n_is_dense_attention(api, name):
+    w = _w(name)
+    w = wl.shrink(w, k=w.N)
+    inp = wl.make_inputs(w, DEV)
+    ids, nrm, *_ = _cache(api, w, inp)
+    O = torch.empty(w.B, w.Hq, w.d, device=DEV)
+    idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=DEV)
+    api.socket_decode(inp["Q"], inp["K"], inp["V"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, w.k, w.scale, O, idx)
+    api.check_status()
+    assert torch.equal(idx.cpu(), torch.arange(w.N, dtype=torch.int32).expand(w.B, w.Hkv, w.N))
+    ref = ao.dense_decode(inp["Q"].double().cpu().numpy(), inp["K"].double().cpu().numpy(),
+                          inp["V"].double().cpu().numpy(), w.scale, N=w.N)
+    assert pa.row_rel_err(O.cpu().numpy(), ref) < pa.out_tol(w)
+
+
+def test_decode_k_one_picks_the_top_key(api):
+    w = wl.shrink(_w("llama8b_needles"), k=1)
+    inp = wl.make_inputs(w, DEV)
+    ids, nrm, ids_nat, norms, _ = _cache(api, w, inp)
+    O, idx = _decode_and_compare(api, w, inp, ids, nrm, ids_nat, norms, pa.BF16_TOL)
+    # a single selected key: the output is that key's value row
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            v = inp["V"][b, h, idx[b, h, 0].item()].float()
+            assert torch.allclose(O[b, h * w.G:(h + 1) * w.G], v.expand(w.G, -1), rtol=0, atol=1e-6)
+
+
+# ---------------------------------------------------------------- dense decode
+
+@pytest.mark.parametrize("name", ["tiny_f32", "llama1b_ragged", "qwen_l48_g8"])
+def test_dense_decode_matches_oracle(api, name):
+    w = _w(name)
+    inp = wl.make_inputs(w, DEV)
+    O = torch.empty(w.B, w.Hq, w.d, device=DEV)
+    api.dense_decode(inp["Q"], inp["K"], inp["V"], w.N, w.scale, O)
+    torch.cuda.synchronize()
+    ref = ao.dense_decode(inp["Q"].double().cpu().numpy(), inp["K"].double().cpu().numpy(),
+                          inp["V"].double().cpu().numpy(), w.scale, N=w.N)
+    assert pa.row_rel_err(O.cpu().numpy(), ref) < pa.out_tol(w)

@@ -35,6 +35,7 @@ SIGNATURES = {
     "dense_decode": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _z, _p]),
     "sk_workspace_bytes": (_z, [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "sk_check_status": (_i, [_p]),
+    "sk_profile_phases": (_i, [_p]),
     "sk_last_error": (ctypes.c_char_p, []),
     "sk_version": (ctypes.c_char_p, []),
 }

@@ -68,9 +68,29 @@ def _ws_bytes(ws):
 
 
 # ---------------------------------------------------------------- cache allocation / layout
+def ids_bytes_per_key(L: int) -> int:
+    """Bytes per key of the bucket-ID cache (see the C header)."""
+    return 16 if L <= 16 else 32 if L <= 32 else 48 if L <= 48 else 64
+
+
+def _chunk_size(L: int, chunk: int) -> int:
+    if chunk == 0:
+        return 16 if L <= 16 else 32
+    return 16 if L <= 48 else 32
+
+
+def _byte_positions(L: int, n: int, device) -> torch.Tensor:
+    """pos[i, l]: byte of key i (i < n) that holds table l's ID (the rotated layout)."""
+    r = torch.arange(n, device=device)[:, None] % 32
+    ll = torch.arange(L, device=device)[None, :]
+    c = (ll >= 32).long()
+    S = torch.where(c == 1, _chunk_size(L, 1), _chunk_size(L, 0))
+    return 32 * c + torch.remainder(ll - 32 * c - r, S)
+
+
 def empty_ids(B: int, Hkv: int, Ncap: int, L: int, device="cuda") -> torch.Tensor:
-    """Bucket-ID cache in the library's key-block interleaved layout [B, Hkv, Ncap/32, L, 32] uint8."""
-    return torch.zeros(B, Hkv, Ncap // 32, L, 32, dtype=torch.uint8, device=device)
+    """Bucket-ID cache [B, Hkv, Ncap, ids_bytes_per_key(L)] uint8 (rotated key-major layout)."""
+    return torch.zeros(B, Hkv, Ncap, ids_bytes_per_key(L), dtype=torch.uint8, device=device)
 
 
 def empty_norms(B: int, Hkv: int, Ncap: int, device="cuda") -> torch.Tensor:
@@ -78,20 +98,23 @@ def empty_norms(B: int, Hkv: int, Ncap: int, device="cuda") -> torch.Tensor:
 
 
 def empty_codes(B: int, Hkv: int, Ncap: int, device="cuda") -> torch.Tensor:
-    """Hard-hash code cache [B, Hkv, Ncap/32, 16, 32] uint8 (byte m of key n at [.., n//32, m, n%32])."""
-    return torch.zeros(B, Hkv, Ncap // 32, 16, 32, dtype=torch.uint8, device=device)
+    """Hard-hash code cache [B, Hkv, Ncap, 16] uint8: byte j of key n holds code byte (j + n) mod 16."""
+    return torch.zeros(B, Hkv, Ncap, 16, dtype=torch.uint8, device=device)
 
 
-def ids_to_natural(ids: torch.Tensor) -> torch.Tensor:
-    """[B, Hkv, Ncap/32, L, 32] -> [B, Hkv, Ncap, L] (a permutation of bytes, no arithmetic)."""
-    B, H, nb, L, _ = ids.shape
-    return ids.permute(0, 1, 2, 4, 3).reshape(B, H, nb * 32, L)
+def ids_to_natural(ids: torch.Tensor, L: int) -> torch.Tensor:
+    """Cache layout -> [B, Hkv, Ncap, L] with [.., n, l] the ID of table l (a byte gather, no arithmetic)."""
+    B, H, n, _ = ids.shape
+    pos = _byte_positions(L, n, ids.device).expand(B, H, n, L)
+    return torch.gather(ids, -1, pos)
 
 
 def natural_to_ids(nat: torch.Tensor) -> torch.Tensor:
-    """[B, Hkv, Ncap, L] -> [B, Hkv, Ncap/32, L, 32] (inverse of ids_to_natural)."""
+    """[B, Hkv, Ncap, L] -> cache layout (inverse of ids_to_natural; padding bytes are 0)."""
     B, H, n, L = nat.shape
-    return nat.reshape(B, H, n // 32, 32, L).permute(0, 1, 2, 4, 3).contiguous()
+    out = torch.zeros(B, H, n, ids_bytes_per_key(L), dtype=nat.dtype, device=nat.device)
+    pos = _byte_positions(L, n, nat.device).expand(B, H, n, L)
+    return out.scatter_(-1, pos, nat)
 
 
 # ---------------------------------------------------------------- entry points
@@ -108,7 +131,7 @@ def socket_hash_keys(K, V, R, L: int, P: int, ids, norms, n_begin: int = 0, n_co
     n_count = Ncap - n_begin if n_count is None else n_count
     _want(V, K.dtype, K.shape, "V")
     _want(R, torch.bfloat16, (L * P, d), "R")
-    _want(ids, torch.uint8, (B, Hkv, Ncap // 32, L, 32), "ids")
+    _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
     _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
     rc = _lib.lib.socket_hash_keys(_ptr(K), _ptr(V), _dtype_code(K), _ptr(R), B, Hkv, Ncap, n_begin, n_count, d, L, P,
                                    _ptr(ids), _ptr(norms), _stream())
@@ -118,8 +141,8 @@ def socket_hash_keys(K, V, R, L: int, P: int, ids, norms, n_begin: int = 0, n_co
 def socket_score(Q, R, ids, norms, N: int, L: int, P: int, tau: float, scores, ws=None):
     """SOCKET steps 2-3: scores [B, Hkv, Ncap] f32 for keys < N."""
     B, Hq, d = Q.shape
-    _, Hkv, nb, L_, _ = ids.shape
-    Ncap = nb * 32
+    _, Hkv, Ncap, _ = ids.shape
+    _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
     _want(scores, torch.float32, (B, Hkv, Ncap), "scores")
     _want(R, torch.bfloat16, (L * P, d), "R")
     ws = _workspace(workspace_bytes(OP_SCORE, B, Hq, Hkv, Ncap, N, d, L, P, 0), Q.device, ws)
@@ -160,7 +183,7 @@ def socket_decode(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k:
     _want(K, Q.dtype, K.shape, "K")
     _want(V, Q.dtype, K.shape, "V")
     _want(R, torch.bfloat16, (L * P, d), "R")
-    _want(ids, torch.uint8, (B, Hkv, Ncap // 32, L, 32), "ids")
+    _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
     _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
     _want(O, torch.float32, (B, Hq, d), "O")
     if idx_out is not None:
@@ -177,7 +200,7 @@ def hata_hash_keys(K, R128, codes, n_begin: int = 0, n_count: int | None = None)
     B, Hkv, Ncap, d = K.shape
     n_count = Ncap - n_begin if n_count is None else n_count
     _want(R128, torch.bfloat16, (128, d), "R128")
-    _want(codes, torch.uint8, (B, Hkv, Ncap // 32, 16, 32), "codes")
+    _want(codes, torch.uint8, (B, Hkv, Ncap, 16), "codes")
     rc = _lib.lib.hata_hash_keys(_ptr(K), _dtype_code(K), _ptr(R128), B, Hkv, Ncap, n_begin, n_count, d, _ptr(codes),
                                  _stream())
     _check(rc, "hata_hash_keys")
@@ -190,10 +213,11 @@ def hata_decode(Q, K, V, R128, codes, N: int, k: int, scale: float, O, idx_out=N
     _want(K, Q.dtype, K.shape, "K")
     _want(V, Q.dtype, K.shape, "V")
     _want(R128, torch.bfloat16, (128, d), "R128")
-    _want(codes, torch.uint8, (B, Hkv, Ncap // 32, 16, 32), "codes")
+    _want(codes, torch.uint8, (B, Hkv, Ncap, 16), "codes")
     _want(O, torch.float32, (B, Hq, d), "O")
     if idx_out is not None:
         _want(idx_out, torch.int32, (B, Hkv, k), "idx_out")
+    ws = _workspace(workspace_bytes(OP_HATA_DECODE, B, Hq, Hkv, Ncap, N, d, 16, 8, k), Q.device, ws)
     rc = _lib.lib.hata_decode(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R128), _ptr(codes), B, Hq, Hkv, Ncap, N,
                               d, k, ctypes.c_float(scale), _ptr(O), _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
     _check(rc, "hata_decode")

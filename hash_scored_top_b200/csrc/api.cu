@@ -4,7 +4,9 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "../../include/hash_scored_top.h"
 #include "socket_kernels.cuh"
@@ -14,6 +16,7 @@ using namespace hst;
 namespace {
 
 thread_local std::string g_last_error = "no error";
+unsigned long long* g_phase_ts = nullptr;     // profiling hook, see sk_profile_phases
 
 int fail(int code, const char* fmt, ...) {
   char buf[512];
@@ -32,6 +35,40 @@ int check_launch(const char* what) {
 }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+// Raises a kernel's dynamic shared-memory limit (and allows 16-CTA clusters)
+// once per kernel; later calls with the same or a smaller size skip the
+// driver call. Kernels are told apart by address.
+struct KernelAttr {
+  const void* fn;
+  size_t smem;
+  bool big_cluster;
+};
+
+template <typename Kern>
+cudaError_t set_kernel_smem(Kern kern, size_t smem, bool big_cluster = false) {
+  static std::mutex mu;
+  static std::vector<KernelAttr> done;
+  const void* fn = reinterpret_cast<const void*>(kern);
+  std::lock_guard<std::mutex> lock(mu);
+  KernelAttr* rec = nullptr;
+  for (auto& r : done)
+    if (r.fn == fn) rec = &r;
+  if (rec == nullptr) {
+    done.push_back(KernelAttr{fn, 0, false});
+    rec = &done.back();
+  }
+  cudaError_t e = cudaSuccess;
+  if (smem > rec->smem) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e == cudaSuccess) rec->smem = smem;
+  }
+  if (e == cudaSuccess && big_cluster && !rec->big_cluster) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e == cudaSuccess) rec->big_cluster = true;
+  }
+  return e;
+}
 
 constexpr int kMaxL = 64;
 constexpr int kNumSMs = 148;
@@ -74,24 +111,25 @@ int check_dtype(sk_dtype t) {
   } while (0)
 
 // ---------------------------------------------------------------- plans
-constexpr int kAttendKeysPerSplit = 256;
-
+// Splits over keys of the attention kernel: one wave of ~2 CTAs per SM
+// (sparse) or several waves (dense), at least 16 keys each.
 int attend_splits(int n, int pairs, bool dense) {
-  if (!dense) return (n + kAttendKeysPerSplit - 1) / kAttendKeysPerSplit;
-  // dense: aim at ~4 CTAs per SM, at least 512 keys per split
-  int splits = (4 * kNumSMs + pairs - 1) / pairs;
-  const int max_splits = (n + 511) / 512;
+  const int target = (dense ? 4 : 2) * kNumSMs;
+  int splits = dense ? (target + pairs - 1) / pairs : target / pairs;
+  int max_splits = (n + 15) / 16;
+  if (max_splits > ATTEND_MAX_SPLITS) max_splits = ATTEND_MAX_SPLITS;
   if (splits > max_splits) splits = max_splits;
   return splits < 1 ? 1 : splits;
 }
 
-size_t attend_part_bytes(int pairs, int splits, int G, int d) {
-  return (size_t)pairs * splits * G * (d + 2) * sizeof(float);
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Workspace of the attention kernel: partials, then one counter per pair.
+size_t attend_ws_bytes(int pairs, int splits, int G, int d) {
+  return align256((size_t)pairs * splits * G * (d + 2) * sizeof(float)) + align256((size_t)pairs * 4);
 }
 
-size_t attend_smem_bytes(int G, int d) {
-  return (size_t)(2 * FUSED_WARPS * G + FUSED_WARPS * G * d + 2 * G + G * d) * sizeof(float);
-}
+int table_chunks_of(int L) { return ids_bytes_per_key(L) > 32 ? 2 : 1; }
 
 // Fused-kernel plan: cluster size C and slice sizes, or C = 0 if the shape
 // cannot run fused.
@@ -102,34 +140,31 @@ struct FusedPlan {
 // Capacities of the fused kernel's shared-memory plan, with the dynamic
 // window starting at byte SMEM_BASE_EXPECTED (the kernel re-checks).
 constexpr uint32_t kTableAddr = 65536;
-constexpr uint32_t kSegBBytes = SMEM_BASE_EXPECTED + SMEM_DYN_MAX - kTableAddr - TABLE_BYTES;
-uint32_t fused_key_capacity() {
-  const uint32_t fixed = ((sizeof(SelShared) + 15u) & ~15u) + (4u << HIST1_BITS) + (4u << HIST2_BITS) +
-                         (4u << HIST3_BITS);
-  const uint32_t segA = kTableAddr - SMEM_BASE_EXPECTED;
-  return (segA - fixed) / 4u + kSegBBytes / 4u;
-}
+constexpr uint32_t kFixedBytes = ((sizeof(SelShared) + 15u) & ~15u) + 4u * (hist_words(0) + hist_words(1) +
+                                                                             hist_words(2));
+constexpr uint32_t kSegAFree = kTableAddr - SMEM_BASE_EXPECTED - kFixedBytes;
+uint32_t seg_b_bytes(int nch) { return SMEM_BASE_EXPECTED + SMEM_DYN_MAX - kTableAddr - nch * TABLE_BYTES; }
+uint32_t fused_key_capacity(int nch) { return kSegAFree / 4u + seg_b_bytes(nch) / 4u; }
 
-FusedPlan plan_fused(int pairs, int N, int k, int G, int d, int L, int P, bool hata, int max_c) {
+FusedPlan plan_select(int pairs, int N, int k, int G, int d, int L, int P, bool hata, int max_c) {
   FusedPlan fp;
-  if (G > 8) return fp;
+  const int nch = table_chunks_of(L);
   const int nblk = (N + 31) / 32;
   int c = 1;
   while (c * 2 <= max_c && pairs * c * 2 <= kNumSMs) c *= 2;
   for (; c <= max_c; c *= 2) {
     const int bpc = (nblk + c - 1) / c;
-    const int chunk = (k + c - 1) / c;
-    const int nl = (L + c - 1) / c;
-    const size_t scratch = hata ? (size_t)G * 16 * 4 : (size_t)table_scratch_doubles(G, d, nl, P) * 8;
-    const size_t attend = attend_smem_bytes(G, d);
-    if ((uint32_t)bpc * 32u <= fused_key_capacity() && chunk * 4 <= TABLE_BYTES && scratch <= kSegBBytes &&
-        attend <= kSegBBytes) {
+    const int per = ((L + c - 1) / c + 3) & ~3;
+    const int nl = per < L ? per : L;
+    const size_t scratch = hata ? hamming_scratch_bytes(G, d, nl) : table_scratch_bytes(G, d, nl, P);
+    if ((uint32_t)bpc * 32u <= fused_key_capacity(nch) && scratch <= kSegAFree) {
       fp.C = c;
       fp.blocks_per_cta = bpc;
-      fp.chunk = chunk;
+      fp.chunk = (k + c - 1) / c;
       return fp;
     }
   }
+  (void)k;
   return fp;
 }
 
@@ -148,7 +183,7 @@ int max_cluster_size() {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  auto kern = socket_decode_fused_kernel<128, 1, __nv_bfloat16, false>;
+  auto kern = socket_select_kernel<128, 32, __nv_bfloat16, false>;
   int n = 0;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) == cudaSuccess &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SMEM_DYN_MAX) == cudaSuccess &&
@@ -161,12 +196,9 @@ int max_cluster_size() {
   return cached;
 }
 
-template <typename Kern>
-int launch_cluster(Kern kern, int grid, int C, size_t smem, cudaStream_t s, const FusedParams& p) {
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return check_launch("cudaFuncSetAttribute(smem)");
-  if (C > 8 && cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess)
-    return check_launch("cudaFuncSetAttribute(cluster)");
+template <typename Kern, typename Params>
+int launch_cluster(Kern kern, int grid, int C, size_t smem, cudaStream_t s, const Params& p) {
+  if (set_kernel_smem(kern, smem, C > 8) != cudaSuccess) return check_launch("cudaFuncSetAttribute");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(FUSED_THREADS, 1, 1);
@@ -184,26 +216,52 @@ int launch_cluster(Kern kern, int grid, int C, size_t smem, cudaStream_t s, cons
   return check_launch("fused kernel");
 }
 
-template <int D, typename KVT, bool HATA>
-int launch_fused_t(const FusedParams& p, int pairs, cudaStream_t s) {
-  if (p.L <= 32) return launch_cluster(socket_decode_fused_kernel<D, 1, KVT, HATA>, pairs * p.C, p.C, SMEM_DYN_MAX, s, p);
-  return launch_cluster(socket_decode_fused_kernel<D, 2, KVT, HATA>, pairs * p.C, p.C, SMEM_DYN_MAX, s, p);
+template <int D, typename QT, bool HATA>
+int launch_select_t(const FusedParams& p, int pairs, cudaStream_t s) {
+  const int grid = pairs * p.C;
+  switch (ids_bytes_per_key(p.L)) {
+    case 16: return launch_cluster(socket_select_kernel<D, 16, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p);
+    case 32: return launch_cluster(socket_select_kernel<D, 32, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p);
+    case 48: return launch_cluster(socket_select_kernel<D, 48, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p);
+    default: return launch_cluster(socket_select_kernel<D, 64, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p);
+  }
 }
 
-int launch_fused(const FusedParams& p, int pairs, int d, sk_dtype kv, bool hata, cudaStream_t s) {
+int launch_select(const FusedParams& p, int pairs, int d, sk_dtype q, bool hata, cudaStream_t s) {
   if (hata) {
-    if (d == 128) return kv == SK_BF16 ? launch_fused_t<128, __nv_bfloat16, true>(p, pairs, s)
-                                       : launch_fused_t<128, float, true>(p, pairs, s);
-    return kv == SK_BF16 ? launch_fused_t<64, __nv_bfloat16, true>(p, pairs, s)
-                         : launch_fused_t<64, float, true>(p, pairs, s);
+    if (d == 128) return q == SK_BF16 ? launch_select_t<128, __nv_bfloat16, true>(p, pairs, s)
+                                      : launch_select_t<128, float, true>(p, pairs, s);
+    return q == SK_BF16 ? launch_select_t<64, __nv_bfloat16, true>(p, pairs, s)
+                        : launch_select_t<64, float, true>(p, pairs, s);
   }
-  if (d == 128) return kv == SK_BF16 ? launch_fused_t<128, __nv_bfloat16, false>(p, pairs, s)
-                                     : launch_fused_t<128, float, false>(p, pairs, s);
-  return kv == SK_BF16 ? launch_fused_t<64, __nv_bfloat16, false>(p, pairs, s)
-                       : launch_fused_t<64, float, false>(p, pairs, s);
+  if (d == 128) return q == SK_BF16 ? launch_select_t<128, __nv_bfloat16, false>(p, pairs, s)
+                                    : launch_select_t<128, float, false>(p, pairs, s);
+  return q == SK_BF16 ? launch_select_t<64, __nv_bfloat16, false>(p, pairs, s)
+                      : launch_select_t<64, float, false>(p, pairs, s);
 }
 
 // ---------------------------------------------------------------- unfused pieces
+template <int D, int LP, typename QT>
+int launch_tables_t(const TableParams& tp, int pairs, int G, cudaStream_t s) {
+  const int ny = tp.L < 16 ? tp.L : 16;
+  const size_t smem = table_scratch_bytes(G, D, (tp.L + ny - 1) / ny, tp.P);
+  if (smem > (size_t)SMEM_DYN_MAX) return fail(SK_ERR_UNSUPPORTED, "bucket table scratch too large (G=%d)", G);
+  auto kern = bucket_table_kernel<D, LP, QT>;
+  set_kernel_smem(kern, smem);
+  kern<<<dim3(pairs, ny), 256, smem, s>>>(tp);
+  return check_launch("bucket_table_kernel");
+}
+
+template <int D, typename QT>
+int launch_tables_d(const TableParams& tp, int pairs, int G, cudaStream_t s) {
+  switch (ids_bytes_per_key(tp.L)) {
+    case 16: return launch_tables_t<D, 16, QT>(tp, pairs, G, s);
+    case 32: return launch_tables_t<D, 32, QT>(tp, pairs, G, s);
+    case 48: return launch_tables_t<D, 48, QT>(tp, pairs, G, s);
+    default: return launch_tables_t<D, 64, QT>(tp, pairs, G, s);
+  }
+}
+
 int launch_tables(const void* Q, sk_dtype q, const void* R, int B, int Hq, int Hkv, int d, int L, int P, float tau,
                   float* T, cudaStream_t s) {
   TableParams tp;
@@ -212,26 +270,25 @@ int launch_tables(const void* Q, sk_dtype q, const void* R, int B, int Hq, int H
   tp.T = T;
   tp.Hq = Hq;
   tp.Hkv = Hkv;
-  tp.d = d;
   tp.L = L;
   tp.P = P;
   tp.tau = tau;
-  const int G = Hq / Hkv;
-  const int ny = L < 16 ? L : 16;
-  const size_t smem = (size_t)table_scratch_doubles(G, d, (L + ny - 1) / ny, P) * 8;
-  if (smem > (size_t)SMEM_DYN_MAX) return fail(SK_ERR_UNSUPPORTED, "bucket table scratch too large (G=%d)", G);
-  dim3 grid(B * Hkv, ny);
-  if (q == SK_BF16) {
-    cudaFuncSetAttribute(bucket_table_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    bucket_table_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(tp);
-  } else {
-    cudaFuncSetAttribute(bucket_table_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    bucket_table_kernel<float><<<grid, 256, smem, s>>>(tp);
-  }
-  return check_launch("bucket_table_kernel");
+  const int G = Hq / Hkv, pairs = B * Hkv;
+  if (d == 128) return q == SK_BF16 ? launch_tables_d<128, __nv_bfloat16>(tp, pairs, G, s)
+                                    : launch_tables_d<128, float>(tp, pairs, G, s);
+  return q == SK_BF16 ? launch_tables_d<64, __nv_bfloat16>(tp, pairs, G, s)
+                      : launch_tables_d<64, float>(tp, pairs, G, s);
 }
 
 constexpr int kScoreBlocksPerCta = 256;
+
+template <int LP>
+int launch_score_t(const ScoreParams& sp, dim3 grid, cudaStream_t s) {
+  const int smem = (int)(kTableAddr + table_chunks(LP) * TABLE_BYTES - SMEM_BASE_EXPECTED);
+  set_kernel_smem(socket_score_kernel<LP>, smem);
+  socket_score_kernel<LP><<<grid, FUSED_THREADS, smem, s>>>(sp);
+  return check_launch("socket_score_kernel");
+}
 
 int launch_score(const float* T, const void* ids, const void* norms, int pairs, int Ncap, int N, int L, float* scores,
                  cudaStream_t s) {
@@ -242,23 +299,20 @@ int launch_score(const float* T, const void* ids, const void* norms, int pairs, 
   sp.scores = scores;
   sp.Ncap = Ncap;
   sp.N = N;
-  sp.L = L;
   sp.blocks_per_cta = kScoreBlocksPerCta;
   const int nblk = (N + 31) / 32;
-  dim3 grid(pairs, (nblk + kScoreBlocksPerCta - 1) / kScoreBlocksPerCta);
-  const int smem = (int)(kTableAddr + TABLE_BYTES - SMEM_BASE_EXPECTED);
-  if (L <= 32) {
-    cudaFuncSetAttribute(socket_score_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    socket_score_kernel<1><<<grid, 256, smem, s>>>(sp);
-  } else {
-    cudaFuncSetAttribute(socket_score_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    socket_score_kernel<2><<<grid, 256, smem, s>>>(sp);
+  const dim3 grid(pairs, (nblk + kScoreBlocksPerCta - 1) / kScoreBlocksPerCta);
+  switch (ids_bytes_per_key(L)) {
+    case 16: return launch_score_t<16>(sp, grid, s);
+    case 32: return launch_score_t<32>(sp, grid, s);
+    case 48: return launch_score_t<48>(sp, grid, s);
+    default: return launch_score_t<64>(sp, grid, s);
   }
-  return check_launch("socket_score_kernel");
 }
 
-constexpr int kTopkFixed = (int)(((sizeof(SelShared) + 15) & ~15) + (4 << HIST1_BITS) + (4 << HIST2_BITS) +
-                                 (4 << HIST3_BITS));
+size_t table_image_bytes(int pairs, int L) { return (size_t)pairs * table_chunks_of(L) * TABLE_BYTES; }
+
+constexpr int kTopkFixed = (int)kFixedBytes;
 
 int topk_cluster_size(int N, int max_c) {
   const int cap = (SMEM_DYN_MAX - kTopkFixed) / 4;
@@ -280,9 +334,7 @@ int launch_topk(const float* scores, int pairs, int Ncap, int N, int k, int* idx
   tp.keys_per_cta = (N + C - 1) / C;
   const size_t smem = kTopkFixed + (size_t)tp.keys_per_cta * 4;
   auto kern = socket_topk_kernel;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
-    return check_launch("cudaFuncSetAttribute(topk smem)");
-  if (C > 8) cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+  if (set_kernel_smem(kern, smem, C > 8) != cudaSuccess) return check_launch("cudaFuncSetAttribute(topk smem)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pairs * C, 1, 1);
   cfg.blockDim = dim3(FUSED_THREADS, 1, 1);
@@ -301,16 +353,31 @@ int launch_topk(const float* scores, int pairs, int Ncap, int N, int k, int* idx
 }
 
 template <int D, typename KVT>
-int launch_attend_t(const AttendParams& ap, int pairs, int G, cudaStream_t s) {
-  const size_t smem = attend_smem_bytes(G, D);
-  cudaFuncSetAttribute(attend_split_kernel<D, KVT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  attend_split_kernel<D, KVT><<<dim3(pairs, ap.splits), FUSED_THREADS, smem, s>>>(ap);
-  return check_launch("attend_split_kernel");
+int launch_attend_t(const AttendParams& ap, int pairs, int G, bool pdl, cudaStream_t s) {
+  const size_t smem = attend_smem_bytes<D>(G, ap.idx ? ap.keys_per_split : 0);
+  auto kern = socket_attend_kernel<D, KVT>;
+  if (set_kernel_smem(kern, smem) != cudaSuccess) return check_launch("cudaFuncSetAttribute(attend smem)");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pairs, ap.splits, 1);
+  cfg.blockDim = dim3(ATTEND_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ap);
+  if (e != cudaSuccess) return fail(SK_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
+  return check_launch("socket_attend_kernel");
 }
 
-// Attention over idx (sparse, n = k) or all keys (dense, idx = NULL, n = N).
+// Attention over idx (sparse, n = k) or all keys (dense, idx = NULL, n = N)
+// through workspace ws (partials + counters). zero_counters: clear the
+// counters first (standalone calls); otherwise the selection kernel did.
 int launch_attend(const void* Q, const void* K, const void* V, sk_dtype kv, const int* idx, int B, int Hq, int Hkv,
-                  int Ncap, int n, int d, float scale, float* O, void* ws, size_t ws_bytes, cudaStream_t s) {
+                  int Ncap, int n, int d, float scale, float* O, void* ws, size_t ws_bytes, bool pdl,
+                  bool zero_counters, cudaStream_t s) {
   const int pairs = B * Hkv, G = Hq / Hkv;
   if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
   AttendParams ap;
@@ -318,6 +385,7 @@ int launch_attend(const void* Q, const void* K, const void* V, sk_dtype kv, cons
   ap.K = K;
   ap.V = V;
   ap.idx = idx;
+  ap.O = O;
   ap.Hq = Hq;
   ap.Hkv = Hkv;
   ap.Ncap = Ncap;
@@ -325,28 +393,36 @@ int launch_attend(const void* Q, const void* K, const void* V, sk_dtype kv, cons
   ap.splits = attend_splits(n, pairs, idx == nullptr);
   ap.keys_per_split = (n + ap.splits - 1) / ap.splits;
   ap.scale = scale;
-  const size_t need = attend_part_bytes(pairs, ap.splits, G, d);
+  const size_t need = attend_ws_bytes(pairs, ap.splits, G, d);
   if (ws == nullptr || ws_bytes < need)
     return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
   ap.part = reinterpret_cast<float*>(ws);
-  int rc;
-  if (d == 128) rc = kv == SK_BF16 ? launch_attend_t<128, __nv_bfloat16>(ap, pairs, G, s)
-                                   : launch_attend_t<128, float>(ap, pairs, G, s);
-  else rc = kv == SK_BF16 ? launch_attend_t<64, __nv_bfloat16>(ap, pairs, G, s)
-                          : launch_attend_t<64, float>(ap, pairs, G, s);
-  if (rc != SK_OK) return rc;
-  merge_splits_kernel<<<pairs * G, d, 0, s>>>(ap.part, O, Hq, Hkv, d, ap.splits);
-  return check_launch("merge_splits_kernel");
+  ap.counters = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(ws) +
+                                                align256((size_t)pairs * ap.splits * G * (d + 2) * sizeof(float)));
+  if (zero_counters) {
+    const cudaError_t e = cudaMemsetAsync(ap.counters, 0, (size_t)pairs * 4, s);
+    if (e != cudaSuccess) return fail(SK_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
+  }
+  if (d == 128) return kv == SK_BF16 ? launch_attend_t<128, __nv_bfloat16>(ap, pairs, G, pdl, s)
+                                     : launch_attend_t<128, float>(ap, pairs, G, pdl, s);
+  return kv == SK_BF16 ? launch_attend_t<64, __nv_bfloat16>(ap, pairs, G, pdl, s)
+                       : launch_attend_t<64, float>(ap, pairs, G, pdl, s);
 }
 
-size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
-
-// Workspace of the unfused decode chain: tables, scores, indices, attention partials.
-size_t chain_ws_bytes(int B, int Hq, int Hkv, int Ncap, int d, int k) {
+// Workspace of a decode step: the index list (when idx_out is NULL) then the
+// attention workspace.
+size_t decode_ws_bytes(int B, int Hq, int Hkv, int k, int d) {
   const int pairs = B * Hkv, G = Hq / Hkv;
-  return align256((size_t)pairs * TABLE_BYTES) + align256((size_t)pairs * Ncap * 4) +
-         align256((size_t)pairs * k * 4) + align256(attend_part_bytes(pairs, attend_splits(k, pairs, false), G, d));
+  return align256((size_t)pairs * k * 4) + attend_ws_bytes(pairs, attend_splits(k, pairs, false), G, d);
 }
+
+// Workspace of the unfused decode chain: tables, scores, then a decode workspace.
+size_t chain_ws_bytes(int B, int Hq, int Hkv, int Ncap, int d, int L, int k) {
+  const int pairs = B * Hkv;
+  return align256(table_image_bytes(pairs, L)) + align256((size_t)pairs * Ncap * 4) + decode_ws_bytes(B, Hq, Hkv, k, d);
+}
+
+constexpr int kAppendMaxKeys = 16;
 
 int hash_launch(const void* K, const void* V, sk_dtype kv, const void* R, int B, int Hkv, int Ncap, int n_begin,
                 int n_count, int d, int L, int P, void* ids, void* norms, cudaStream_t s) {
@@ -365,14 +441,21 @@ int hash_launch(const void* K, const void* V, sk_dtype kv, const void* R, int B,
   hp.P = P;
   hp.pairs = B * Hkv;
   const int LP = L * P;
+  if (n_count <= kAppendMaxKeys) {      // decode-time append: a few keys per pair
+    const dim3 grid(hp.pairs, n_count);
+    const int threads = (LP + 31) / 32 * 32;
+    if (kv == SK_BF16) hash_keys_append_kernel<__nv_bfloat16><<<grid, threads, 0, s>>>(hp);
+    else hash_keys_append_kernel<float><<<grid, threads, 0, s>>>(hp);
+    return check_launch("hash_keys_append_kernel");
+  }
   const size_t smem = (((size_t)d * LP * 2 + 15) & ~(size_t)15) + (size_t)32 * d * 4 + (size_t)LP * 4;
   const long units = (long)hp.pairs * ((n_begin + n_count - 1) / 32 - n_begin / 32 + 1);
   const int grid = (int)(units < 8L * kNumSMs ? units : 8L * kNumSMs);
   if (kv == SK_BF16) {
-    cudaFuncSetAttribute(hash_keys_simt_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    set_kernel_smem(hash_keys_simt_kernel<__nv_bfloat16>, smem);
     hash_keys_simt_kernel<__nv_bfloat16><<<grid, HASH_THREADS, smem, s>>>(hp);
   } else {
-    cudaFuncSetAttribute(hash_keys_simt_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    set_kernel_smem(hash_keys_simt_kernel<float>, smem);
     hash_keys_simt_kernel<float><<<grid, HASH_THREADS, smem, s>>>(hp);
   }
   return check_launch("hash_keys_simt_kernel");
@@ -417,7 +500,7 @@ int socket_score(const void* Q, sk_dtype q, const void* R, const void* ids, cons
   SK_TRY(check_heads(B, Hq, Hkv, d));
   SK_TRY(check_cache(Ncap, N));
   SK_TRY(check_tables(L, P, tau));
-  const size_t need = (size_t)B * Hkv * TABLE_BYTES;
+  const size_t need = table_image_bytes(B * Hkv, L);
   if (ws == nullptr || ws_bytes < need)
     return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
   cudaStream_t s = as_stream(stream);
@@ -450,8 +533,73 @@ int socket_sparse_attend(const void* Q, const void* K, const void* V, sk_dtype k
   SK_TRY(check_heads(B, Hq, Hkv, d));
   if (Ncap < 32 || Ncap % 32) return fail(SK_ERR_INVALID_ARG, "Ncap=%d must be a positive multiple of 32", Ncap);
   if (k < 1) return fail(SK_ERR_INVALID_ARG, "k=%d must be >= 1", k);
-  return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, ws, ws_bytes, as_stream(stream));
+  return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, ws, ws_bytes, false, true,
+                       as_stream(stream));
 }
+
+namespace {
+
+// The decode step: selection kernel (tables, scores, exact top-k -> index list)
+// then the attention kernel (programmatic dependent launch), or the unfused
+// chain when the selection cannot keep a pair's keys on chip.
+int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, const void* ids,
+                const void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k,
+                float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, bool hata, cudaStream_t s) {
+  const int pairs = B * Hkv, G = Hq / Hkv;
+  if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
+  const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, hata, max_cluster_size());
+  if (fp.C == 0 && hata) return fail(SK_ERR_UNSUPPORTED, "hard-hash decode: N=%d too large for one cluster", N);
+  const size_t need = fp.C > 0 ? decode_ws_bytes(B, Hq, Hkv, k, d) : chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
+  char* w = reinterpret_cast<char*>(ws);
+  if (fp.C == 0) {        // unfused chain through the workspace
+    float* T = reinterpret_cast<float*>(w);
+    w += align256(table_image_bytes(pairs, L));
+    float* scores = reinterpret_cast<float*>(w);
+    w += align256((size_t)pairs * Ncap * 4);
+    int* idx = idx_out ? idx_out : reinterpret_cast<int*>(w);
+    w += align256((size_t)pairs * k * 4);
+    SK_TRY(launch_tables(Q, kv, R, B, Hq, Hkv, d, L, P, tau, T, s));
+    SK_TRY(launch_score(T, ids, norms, pairs, Ncap, N, L, scores, s));
+    SK_TRY(launch_topk(scores, pairs, Ncap, N, k, idx, s));
+    return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, w,
+                         attend_ws_bytes(pairs, attend_splits(k, pairs, false), G, d), false, true, s);
+  }
+  int* idx = idx_out ? idx_out : reinterpret_cast<int*>(w);
+  w += align256((size_t)pairs * k * 4);
+  const int splits = attend_splits(k, pairs, false);
+  unsigned int* counters = reinterpret_cast<unsigned int*>(
+      w + align256((size_t)pairs * splits * G * (d + 2) * sizeof(float)));
+  FusedParams p;
+  p.Q = Q;
+  p.K = K;
+  p.V = V;
+  p.R = reinterpret_cast<const __nv_bfloat16*>(R);
+  p.ids = reinterpret_cast<const uint8_t*>(ids);
+  p.norms = reinterpret_cast<const __half*>(norms);
+  p.O = O;
+  p.idx_out = idx;
+  p.counters = counters;
+  p.phase_ts = g_phase_ts;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.Ncap = Ncap;
+  p.N = N;
+  p.L = L;
+  p.P = P;
+  p.k = k;
+  p.C = fp.C;
+  p.blocks_per_cta = fp.blocks_per_cta;
+  p.chunk = fp.chunk;
+  p.tau = tau;
+  p.scale = scale;
+  SK_TRY(launch_select(p, pairs, d, kv, hata, s));
+  return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, w, attend_ws_bytes(pairs, splits, G, d),
+                       true, false, s);
+}
+
+}  // namespace
 
 int socket_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, const void* ids,
                   const void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k,
@@ -468,50 +616,8 @@ int socket_decode(const void* Q, const void* K, const void* V, sk_dtype kv, cons
   SK_TRY(check_cache(Ncap, N));
   SK_TRY(check_tables(L, P, tau));
   if (k < 1 || k > N) return fail(SK_ERR_INVALID_ARG, "k=%d must be in [1, N=%d]", k, N);
-  const int pairs = B * Hkv, G = Hq / Hkv;
-  if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
-  cudaStream_t s = as_stream(stream);
-  const FusedPlan fp = plan_fused(pairs, N, k, G, d, L, P, false, max_cluster_size());
-  if (fp.C > 0) {
-    FusedParams p;
-    p.Q = Q;
-    p.K = K;
-    p.V = V;
-    p.R = reinterpret_cast<const __nv_bfloat16*>(R);
-    p.ids = reinterpret_cast<const uint8_t*>(ids);
-    p.norms = reinterpret_cast<const __half*>(norms);
-    p.O = O;
-    p.idx_out = idx_out;
-    p.Hq = Hq;
-    p.Hkv = Hkv;
-    p.Ncap = Ncap;
-    p.N = N;
-    p.L = L;
-    p.P = P;
-    p.k = k;
-    p.C = fp.C;
-    p.blocks_per_cta = fp.blocks_per_cta;
-    p.chunk = fp.chunk;
-    p.tau = tau;
-    p.scale = scale;
-    return launch_fused(p, pairs, d, kv, false, s);
-  }
-  // unfused chain through the workspace
-  const size_t need = chain_ws_bytes(B, Hq, Hkv, Ncap, d, k);
-  if (ws == nullptr || ws_bytes < need)
-    return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
-  char* w = reinterpret_cast<char*>(ws);
-  float* T = reinterpret_cast<float*>(w);
-  w += align256((size_t)pairs * TABLE_BYTES);
-  float* scores = reinterpret_cast<float*>(w);
-  w += align256((size_t)pairs * Ncap * 4);
-  int* idx = idx_out ? idx_out : reinterpret_cast<int*>(w);
-  w += align256((size_t)pairs * k * 4);
-  const size_t part_bytes = align256(attend_part_bytes(pairs, attend_splits(k, pairs, false), G, d));
-  SK_TRY(launch_tables(Q, kv, R, B, Hq, Hkv, d, L, P, tau, T, s));
-  SK_TRY(launch_score(T, ids, norms, pairs, Ncap, N, L, scores, s));
-  SK_TRY(launch_topk(scores, pairs, Ncap, N, k, idx, s));
-  return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, w, part_bytes, s);
+  return decode_impl(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, scale, O, idx_out, ws, ws_bytes,
+                     false, as_stream(stream));
 }
 
 int hata_hash_keys(const void* K, sk_dtype kv, const void* R128, int B, int Hkv, int Ncap, int n_begin, int n_count,
@@ -533,8 +639,6 @@ int hata_hash_keys(const void* K, sk_dtype kv, const void* R128, int B, int Hkv,
 int hata_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R128, const void* codes, int B,
                 int Hq, int Hkv, int Ncap, int N, int d, int k, float scale, float* O, int* idx_out, void* ws,
                 size_t ws_bytes, void* stream) {
-  (void)ws;
-  (void)ws_bytes;
   SK_NONNULL(Q);
   SK_NONNULL(K);
   SK_NONNULL(V);
@@ -545,32 +649,10 @@ int hata_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const 
   SK_TRY(check_heads(B, Hq, Hkv, d));
   SK_TRY(check_cache(Ncap, N));
   if (k < 1 || k > N) return fail(SK_ERR_INVALID_ARG, "k=%d must be in [1, N=%d]", k, N);
-  const int pairs = B * Hkv, G = Hq / Hkv;
-  if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
-  const FusedPlan fp = plan_fused(pairs, N, k, G, d, 16, 8, true, max_cluster_size());
-  if (fp.C == 0) return fail(SK_ERR_UNSUPPORTED, "hard-hash decode: N=%d / k=%d too large for one cluster", N, k);
-  FusedParams p;
-  p.Q = Q;
-  p.K = K;
-  p.V = V;
-  p.R = reinterpret_cast<const __nv_bfloat16*>(R128);
-  p.ids = reinterpret_cast<const uint8_t*>(codes);
-  p.norms = nullptr;
-  p.O = O;
-  p.idx_out = idx_out;
-  p.Hq = Hq;
-  p.Hkv = Hkv;
-  p.Ncap = Ncap;
-  p.N = N;
-  p.L = 16;
-  p.P = 8;
-  p.k = k;
-  p.C = fp.C;
-  p.blocks_per_cta = fp.blocks_per_cta;
-  p.chunk = fp.chunk;
-  p.tau = 1.f;
-  p.scale = scale;
-  return launch_fused(p, pairs, d, kv, true, as_stream(stream));
+  if (Hq / Hkv > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", Hq / Hkv);
+  // 128 code bits = 16 byte-tables of 8 hyperplanes; no norms
+  return decode_impl(Q, K, V, kv, R128, codes, codes, B, Hq, Hkv, Ncap, N, d, 16, 8, 1.f, k, scale, O, idx_out, ws,
+                     ws_bytes, true, as_stream(stream));
 }
 
 int dense_decode(const void* Q, const void* K, const void* V, sk_dtype kv, int B, int Hq, int Hkv, int Ncap, int N,
@@ -582,7 +664,8 @@ int dense_decode(const void* Q, const void* K, const void* V, sk_dtype kv, int B
   SK_TRY(check_dtype(kv));
   SK_TRY(check_heads(B, Hq, Hkv, d));
   SK_TRY(check_cache(Ncap, N));
-  return launch_attend(Q, K, V, kv, nullptr, B, Hq, Hkv, Ncap, N, d, scale, O, ws, ws_bytes, as_stream(stream));
+  return launch_attend(Q, K, V, kv, nullptr, B, Hq, Hkv, Ncap, N, d, scale, O, ws, ws_bytes, false, true,
+                       as_stream(stream));
 }
 
 size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, int k) {
@@ -593,25 +676,38 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
     case SK_OP_HASH_KEYS:
     case SK_OP_HATA_HASH:
     case SK_OP_TOPK:
-    case SK_OP_HATA_DECODE:
       return 0;
     case SK_OP_SCORE:
-      return (size_t)pairs * TABLE_BYTES;
+      if (L < 1 || L > kMaxL) return bad;
+      return table_image_bytes(pairs, L);
     case SK_OP_SPARSE_ATTEND:
       if (k < 1) return bad;
-      return attend_part_bytes(pairs, attend_splits(k, pairs, false), G, d);
+      return attend_ws_bytes(pairs, attend_splits(k, pairs, false), G, d);
     case SK_OP_DENSE_DECODE:
       if (N < 1) return bad;
-      return attend_part_bytes(pairs, attend_splits(N, pairs, true), G, d);
-    case SK_OP_DECODE: {
+      return attend_ws_bytes(pairs, attend_splits(N, pairs, true), G, d);
+    case SK_OP_DECODE:
+    case SK_OP_HATA_DECODE: {
       if (k < 1 || N < 1 || G > 8) return bad;
-      const FusedPlan fp = plan_fused(pairs, N, k, G, d, L, P, false, 8);
-      if (fp.C > 0) return 0;
-      return chain_ws_bytes(B, Hq, Hkv, Ncap, d, k);
+      if (op == SK_OP_HATA_DECODE) {
+        L = 16;
+        P = 8;
+      }
+      if (L < 1 || L > kMaxL || P < 1 || P > 8) return bad;
+      // the unfused chain runs when the selection cannot hold a pair's keys on
+      // chip; 8-CTA clusters are always available, 16-CTA ones may not be
+      const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, op == SK_OP_HATA_DECODE, 8);
+      if (fp.C > 0 || op == SK_OP_HATA_DECODE) return decode_ws_bytes(B, Hq, Hkv, k, d);
+      return chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
     }
     default:
       return bad;
   }
+}
+
+int sk_profile_phases(unsigned long long* device_buffer) {
+  g_phase_ts = device_buffer;
+  return SK_OK;
 }
 
 int sk_check_status(void* stream) {

@@ -2,25 +2,23 @@
 // technical summary, section 中核メカニズム：ソフト LSH, step 4: exact
 // attention on the selected subset), for the G query heads of one KV head.
 //
-// bf16 K/V: one warp processes 16 keys per step on the tensor cores
-// (mma.sync m16n8k16, bf16 in, f32 accumulate), with the keys on the M side:
-//   S^T[16 keys x 8 head slots] = K_tile[16 x d] . Q^T[d x 8]
-//   O^T[d x 8 slots]           += V_tile^T[d x 16] . P^T[16 x 8]
-// Each lane loads its operands straight from global memory with 16-byte
-// loads: the contraction index of each product (head dim for QK, key for
-// PV) is permuted consistently on both operands, so every fragment register
-// is a contiguous 4-byte piece of a loaded 16-byte chunk (no shared memory,
-// no ldmatrix). P^T is moved from the accumulator layout to the B-operand
-// layout with movmatrix.trans. The probabilities are split P = P_hi + P_lo
-// (both bf16) so the PV product carries ~16 mantissa bits of P: for G <= 4
-// the lo parts ride in the unused head slots 4..7 of the same MMA; for
-// 5 <= G <= 8 a second MMA adds them.
+// bf16 K/V, one warp per 16-key tile:
+//   * the warp's lanes issue one 1-D bulk copy (TMA engine) per selected K or
+//     V row into the warp's shared-memory slot (rows padded to 2D + 16 bytes,
+//     which makes the ldmatrix reads below conflict-free) and wait on the
+//     slot's mbarrier (bounded wait);
+//   * tensor cores (mma.sync m16n8k16, bf16 in, f32 accumulate) with the keys
+//     on the M side:  S^T[16 keys x 8 head slots] = K_tile . Q^T and
+//     O^T[d x 8 slots] += V_tile^T . P^T; K and Q^T fragments come from
+//     ldmatrix, V^T fragments from ldmatrix.trans, and P^T moves from the
+//     accumulator layout to the operand layout with movmatrix.trans;
+//   * P is split as P_hi + P_lo (both bf16) so the PV product carries ~16
+//     mantissa bits of P: for G <= 4 the lo parts ride in head slots 4..7 of
+//     the same MMA, for 5 <= G <= 8 a second MMA adds them.
+// Softmax: per head a running max m and sum l in the log2 domain (logits are
+// pre-multiplied by scale * log2(e)).
 //
-// f32 K/V: a plain SIMT path (lanes over the head dim), used for small
-// fp32 caches.
-//
-// Softmax: per head, running max m and sum l in the log2 domain (logits are
-// pre-multiplied by scale * log2(e)); exp2 of non-positive arguments only.
+// f32 K/V: a SIMT path, one head per warp (lanes over the head dim).
 #pragma once
 
 #include "common.cuh"
@@ -44,16 +42,46 @@ __device__ __forceinline__ uint32_t movmatrix_trans(uint32_t x) {
   return y;
 }
 
-__device__ __forceinline__ uint32_t u4get(const uint4& v, int e) {
-  return e == 0 ? v.x : e == 1 ? v.y : e == 2 ? v.z : v.w;
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3) : "r"(addr));
 }
 
-// Per-warp partial result of attention over a subset: for head slot i of this
-// lane, running max m (log2 domain), lane-partial sum l, and the unnormalised
-// output fragment acc.
+__device__ __forceinline__ void ldsm_x4_trans(uint32_t addr, uint32_t& a0, uint32_t& a1, uint32_t& a2, uint32_t& a3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(a0), "=r"(a1), "=r"(a2), "=r"(a3) : "r"(addr));
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t addr, uint32_t& b0, uint32_t& b1) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(addr));
+}
+
+// Padded row stride of K/V/Q rows in shared memory (bytes).
+template <int D>
+__host__ __device__ constexpr int kv_row_bytes() { return 2 * D + 16; }
+// One warp slot: 16 K rows then 16 V rows.
+template <int D>
+__host__ __device__ constexpr int kv_slot_bytes() { return 32 * kv_row_bytes<D>(); }
+// Q^T staging: 8 head rows.
+template <int D>
+__host__ __device__ constexpr int q_stage_bytes() { return 8 * kv_row_bytes<D>(); }
+
+// Copies the group's bf16 query rows into padded rows at `qs` (rows >= G zero).
+// All threads of the block; the caller synchronises afterwards.
+template <int D>
+__device__ __forceinline__ void stage_q(const __nv_bfloat16* __restrict__ Qg, int G, unsigned char* qs) {
+  constexpr int RS = kv_row_bytes<D>();
+  for (int e = threadIdx.x; e < 8 * (D / 8); e += blockDim.x) {
+    const int h = e / (D / 8), c8 = e % (D / 8);
+    const uint4 v = h < G ? *reinterpret_cast<const uint4*>(Qg + (size_t)h * D + 8 * c8) : make_uint4(0, 0, 0, 0);
+    *reinterpret_cast<uint4*>(qs + h * RS + 16 * c8) = v;
+  }
+}
+
+// Per-warp running state for the G head slots of this lane (2 per lane).
 template <int D>
 struct MmaAttendState {
-  float acc[D / 16][4];
+  float acc[D / 16][4];   // O^T fragments: rows dv = 16j + r (+8), columns = head slots 2c, 2c+1
   float m[2];
   float l[2];
   __device__ __forceinline__ void init() {
@@ -64,89 +92,63 @@ struct MmaAttendState {
   }
 };
 
-// Q^T fragments of a lane: qb[q][e] packs Q[head r][32q + 8c + 2e .. +1], zero
-// for head slots >= G. Q is bf16 [G][D] (row stride D).
-template <int D>
-__device__ __forceinline__ void load_q_frag(uint32_t (&qb)[D / 32][4], const __nv_bfloat16* __restrict__ Qg,
-                                            int G, int lane) {
-  const int r = lane >> 2, c = lane & 3;
-#pragma unroll
-  for (int q = 0; q < D / 32; ++q) {
-    if (r < G) {
-      const uint4 v = *reinterpret_cast<const uint4*>(Qg + (size_t)r * D + 32 * q + 8 * c);
-      qb[q][0] = v.x; qb[q][1] = v.y; qb[q][2] = v.z; qb[q][3] = v.w;
-    } else {
-      qb[q][0] = qb[q][1] = qb[q][2] = qb[q][3] = 0u;
-    }
-  }
-}
-
-// Row loads of one 16-key tile for this lane.
-template <int D>
-struct KVTile {
-  uint4 k[2][D / 32];     // key rows r and r+8: chunk q covers dims 32q + 8c .. +8
-  uint4 v[4][D / 64];     // value rows 2c, 2c+1, 2c+8, 2c+9: half covers dims 64*half + 8r .. +8
-  bool kvalid[2];
-  bool vvalid[4];
-};
-
-// keys(i) gives the cache row of tile key i (0..15); nvalid of them are real,
-// the rest are padding (loaded from row keys(0), then masked). Rows are
-// clamped into [0, nrows) so a bad index can never read outside the cache.
+// Issues the bulk copies of one tile's K and V rows into a warp slot.
+// keys(i) is the cache row of tile key i < nvalid; rows are clamped into
+// [0, nrows). The tile's transaction bytes are armed on `mbar` first.
 template <int D, typename KeyFn>
-__device__ __forceinline__ void load_kv_tile(KVTile<D>& t, const __nv_bfloat16* __restrict__ Kp,
-                                             const __nv_bfloat16* __restrict__ Vp, KeyFn keys, int nvalid,
-                                             int nrows, int lane) {
-  const int r = lane >> 2, c = lane & 3;
-  auto clamp_row = [&](int x) { return min(max(x, 0), nrows - 1); };
-  const int row0 = clamp_row(keys(0));
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    const int i = r + 8 * s;
-    t.kvalid[s] = i < nvalid;
-    const int row = t.kvalid[s] ? clamp_row(keys(i)) : row0;
-    const __nv_bfloat16* base = Kp + (size_t)row * D + 8 * c;
-#pragma unroll
-    for (int q = 0; q < D / 32; ++q) t.k[s][q] = ldg_stream(base + 32 * q);
-  }
-#pragma unroll
-  for (int s = 0; s < 4; ++s) {
-    const int i = 2 * c + (s & 1) + 8 * (s >> 1);
-    t.vvalid[s] = i < nvalid;
-    const int row = t.vvalid[s] ? clamp_row(keys(i)) : row0;
-    const __nv_bfloat16* base = Vp + (size_t)row * D + 8 * r;
-#pragma unroll
-    for (int h = 0; h < D / 64; ++h) t.v[s][h] = ldg_stream(base + 64 * h);
+__device__ __forceinline__ void issue_tile_copies(uint32_t slot, uint32_t mbar, const __nv_bfloat16* __restrict__ Kp,
+                                                  const __nv_bfloat16* __restrict__ Vp, KeyFn keys, int nvalid,
+                                                  int nrows, int lane) {
+  constexpr int RS = kv_row_bytes<D>();
+  fence_proxy_async_shared();
+  if (lane == 0) mbar_arrive_expect_tx(mbar, (uint32_t)nvalid * 2u * D * 2u);
+  __syncwarp();
+  const int i = lane & 15;
+  if (i < nvalid) {
+    const int row = min(max(keys(i), 0), nrows - 1);
+    const __nv_bfloat16* src = (lane < 16 ? Kp : Vp) + (size_t)row * D;
+    bulk_copy_g2s(slot + (lane < 16 ? 0u : 16u * RS) + (uint32_t)i * RS, src, 2u * D, mbar);
   }
 }
 
-// One 16-key step of attention for a warp. `packed` selects the G <= 4 mode.
+// One 16-key step of attention for a warp, reading the tile from its slot.
 template <int D>
-__device__ __forceinline__ void mma_attend_tile(MmaAttendState<D>& st, KVTile<D>& t,
-                                                const uint32_t (&qb)[D / 32][4], float scale_log2,
-                                                bool packed, int lane) {
-  const int c = lane & 3;
+__device__ __forceinline__ void mma_attend_slot(MmaAttendState<D>& st, uint32_t slot, uint32_t qs, int nvalid,
+                                                float scale_log2, bool packed, int lane) {
+  constexpr int RS = kv_row_bytes<D>();
+  const int r = lane >> 2, c = lane & 3, mtx = lane >> 3, mrow = lane & 7;
+  const uint32_t kslot = slot, vslot = slot + 16u * RS;
+  // padding V rows hold stale data: zero them (their P is 0; keep 0 * v finite)
+  if (nvalid < 16) {
+    const int i = lane & 15;
+    if (i >= nvalid && lane < 16) {
+#pragma unroll
+      for (int c8 = 0; c8 < D / 8; ++c8)
+        asm volatile("st.shared.v4.u32 [%0], {%1,%1,%1,%1};" ::"r"(vslot + (uint32_t)i * RS + 16u * c8), "r"(0u)
+                     : "memory");
+    }
+    __syncwarp();
+  }
   // ---- S^T = K . Q^T
   float s[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-  for (int q = 0; q < D / 32; ++q) {
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      mma_bf16_16816(s, u4get(t.k[0][q], 2 * h), u4get(t.k[1][q], 2 * h), u4get(t.k[0][q], 2 * h + 1),
-                     u4get(t.k[1][q], 2 * h + 1), qb[q][2 * h], qb[q][2 * h + 1]);
-    }
+  for (int q = 0; q < D / 16; ++q) {
+    uint32_t a0, a1, a2, a3, b0, b1;
+    ldsm_x4(kslot + (uint32_t)((mtx & 1) * 8 + mrow) * RS + (uint32_t)(16 * q + (mtx >> 1) * 8) * 2u, a0, a1, a2, a3);
+    ldsm_x2(qs + (uint32_t)mrow * RS + (uint32_t)(16 * q + (mtx & 1) * 8) * 2u, b0, b1);
+    mma_bf16_16816(s, a0, a1, a2, a3, b0, b1);
   }
 #pragma unroll
   for (int i = 0; i < 4; ++i) s[i] *= scale_log2;
-  if (packed) {                      // slots 4..7 mirror heads 0..3
+  if (packed) {                      // head slots 4..7 mirror heads 0..3
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const float o = __shfl_xor_sync(FULL, s[i], 2);
       if (c >= 2) s[i] = o;
     }
   }
-  if (!t.kvalid[0]) { s[0] = -INFINITY; s[1] = -INFINITY; }
-  if (!t.kvalid[1]) { s[2] = -INFINITY; s[3] = -INFINITY; }
+  if (r >= nvalid) { s[0] = -INFINITY; s[1] = -INFINITY; }
+  if (r + 8 >= nvalid) { s[2] = -INFINITY; s[3] = -INFINITY; }
 
   // ---- online softmax per head slot (2 per lane)
   float p[4];
@@ -191,21 +193,12 @@ __device__ __forceinline__ void mma_attend_tile(MmaAttendState<D>& st, KVTile<D>
     }
   }
 
-  // ---- O^T += V^T . P^T  (padding value rows are zeroed)
-#pragma unroll
-  for (int s2 = 0; s2 < 4; ++s2) {
-    if (!t.vvalid[s2]) {
-#pragma unroll
-      for (int h = 0; h < D / 64; ++h) t.v[s2][h] = make_uint4(0, 0, 0, 0);
-    }
-  }
+  // ---- O^T += V^T . P^T
 #pragma unroll
   for (int j = 0; j < D / 16; ++j) {
-    const int h = j >> 2, e = j & 3;
-    const uint32_t x0 = u4get(t.v[0][h], e), x1 = u4get(t.v[1][h], e);
-    const uint32_t x2 = u4get(t.v[2][h], e), x3 = u4get(t.v[3][h], e);
-    const uint32_t a0 = __byte_perm(x0, x1, 0x5410), a1 = __byte_perm(x0, x1, 0x7632);
-    const uint32_t a2 = __byte_perm(x2, x3, 0x5410), a3 = __byte_perm(x2, x3, 0x7632);
+    uint32_t a0, a1, a2, a3;
+    ldsm_x4_trans(vslot + (uint32_t)((mtx >> 1) * 8 + mrow) * RS + (uint32_t)(16 * j + (mtx & 1) * 8) * 2u, a0, a1, a2,
+                  a3);
     mma_bf16_16816(st.acc[j], a0, a1, a2, a3, bh0, bh1);
     if (!packed) mma_bf16_16816(st.acc[j], a0, a1, a2, a3, bl0, bl1);
   }
@@ -221,12 +214,29 @@ struct PartialView {
   int D;
 };
 
+__host__ __device__ inline size_t partial_bytes(int nslots, int G, int D) {
+  return (size_t)(2 * nslots * G + nslots * G * D + 2 * G + G * D) * sizeof(float);
+}
+
+__device__ __forceinline__ PartialView partial_view(float* base, int nslots, int G, int D, float*& cM, float*& cL,
+                                                    float*& cO) {
+  PartialView pv;
+  pv.G = G;
+  pv.D = D;
+  pv.pm = base;
+  pv.pl = pv.pm + nslots * G;
+  pv.po = pv.pl + nslots * G;
+  cM = pv.po + (size_t)nslots * G * D;
+  cL = cM + G;
+  cO = cL + G;
+  return pv;
+}
+
 // Writes a warp's MMA state into partial slot w (heads < G only).
 template <int D>
-__device__ __forceinline__ void store_mma_partial(MmaAttendState<D>& st, const PartialView& pv, int w,
-                                                  bool packed, int lane) {
+__device__ __forceinline__ void store_mma_partial(MmaAttendState<D>& st, const PartialView& pv, int w, bool packed,
+                                                  int lane) {
   const int r = lane >> 2, c = lane & 3;
-  // total l over the 8 key lanes
   float l[2];
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
@@ -236,7 +246,7 @@ __device__ __forceinline__ void store_mma_partial(MmaAttendState<D>& st, const P
     v += __shfl_xor_sync(FULL, v, 16);
     l[i] = v;
   }
-  // packed: O(head) = hi column (lane c<2) + lo column (lane c^2)
+  // packed: O(head) = hi column (lane c < 2) + lo column (lane c ^ 2)
 #pragma unroll
   for (int j = 0; j < D / 16; ++j) {
 #pragma unroll
@@ -259,83 +269,109 @@ __device__ __forceinline__ void store_mma_partial(MmaAttendState<D>& st, const P
         float* po = pv.po + ((size_t)w * pv.G + h) * D;
 #pragma unroll
         for (int j = 0; j < D / 16; ++j) {
-          const int dv = 64 * (j >> 2) + 8 * r + 2 * (j & 3);
-          po[dv] = st.acc[j][i];
-          po[dv + 1] = st.acc[j][2 + i];
+          po[16 * j + r] = st.acc[j][i];
+          po[16 * j + r + 8] = st.acc[j][2 + i];
         }
       }
     }
   }
 }
 
-// ---------------------------------------------------------------- f32 SIMT path
-template <int D>
-struct SimtAttendState {
-  float acc[8][D / 32];   // head slot, dims lane + 32*i
-  float m[8];
-  float l[8];
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      m[h] = -INFINITY;
-      l[h] = 0.f;
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i) acc[h][i] = 0.f;
-    }
-  }
-};
-
-// One key for all G (<= 8) heads; q[h][i] holds Q[h][lane + 32 i] * scale_log2.
-template <int D>
-__device__ __forceinline__ void simt_attend_key(SimtAttendState<D>& st, const float* __restrict__ krow,
-                                                const float* __restrict__ vrow, const float (&q)[8][D / 32], int G,
-                                                int lane) {
-  float kv[D / 32], vv[D / 32];
-#pragma unroll
-  for (int i = 0; i < D / 32; ++i) {
-    kv[i] = krow[lane + 32 * i];
-    vv[i] = vrow[lane + 32 * i];
-  }
-#pragma unroll
-  for (int h = 0; h < 8; ++h) {
-    if (h < G) {
-      float s = 0.f;
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i) s = fmaf(q[h][i], kv[i], s);
-      s = warp_sum(s);
-      const float m_new = fmaxf(st.m[h], s);
-      const float alpha = exp2f(st.m[h] - m_new);
-      const float p = exp2f(s - m_new);
-      st.l[h] = st.l[h] * alpha + p;
-      st.m[h] = m_new;
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i) st.acc[h][i] = st.acc[h][i] * alpha + p * vv[i];
-    }
+// Marks partial slot w as empty (no keys) for every head.
+__device__ __forceinline__ void store_empty_partial(const PartialView& pv, int w, int lane) {
+  for (int h = lane; h < pv.G; h += 32) {
+    pv.pm[w * pv.G + h] = -INFINITY;
+    pv.pl[w * pv.G + h] = 0.f;
   }
 }
 
-template <int D>
-__device__ __forceinline__ void store_simt_partial(const SimtAttendState<D>& st, const PartialView& pv, int w,
-                                                   int lane) {
+// bf16 attention of `cnt` listed keys by warps 0..ncw-1 (warp w owns slot
+// `slot0 + w * slot_stride` and mbarrier `mbar0 + 8 w`, phase bits in
+// phases[w]); results go to partial slots 0..ncw-1. Other warps do nothing.
+template <int D, typename KeyFn>
+__device__ void attend_tiles_bf16(const __nv_bfloat16* __restrict__ Kp, const __nv_bfloat16* __restrict__ Vp,
+                                  KeyFn keys, int cnt, int nrows, int G, float scale, uint32_t qs, uint32_t slot0,
+                                  uint32_t slot_stride, uint32_t mbar0, uint32_t* phases, int ncw,
+                                  const PartialView& pv) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp >= ncw) return;
+  const bool packed = G <= 4;
+  const float scale_log2 = scale * LOG2E;
+  MmaAttendState<D> st;
+  st.init();
+  const uint32_t slot = slot0 + (uint32_t)warp * slot_stride;
+  const uint32_t mbar = mbar0 + 8u * warp;
+  uint32_t phase = phases[warp];
+  const int ntiles = (cnt + 15) / 16;
+  bool ok = true;
+  for (int t = warp; t < ntiles && ok; t += ncw) {
+    const int nvalid = min(16, cnt - 16 * t);
+    issue_tile_copies<D>(slot, mbar, Kp, Vp, [&](int i) { return keys(16 * t + i); }, nvalid, nrows, lane);
+    ok = mbar_wait_bounded(mbar, phase);
+    phase ^= 1u;
+    if (ok) mma_attend_slot<D>(st, slot, qs, nvalid, scale_log2, packed, lane);
+    __syncwarp();
+  }
+  if (!ok) {           // a copy never completed: wait once more (bounded) so none is left in flight
+    mbar_wait_bounded(mbar, phase ^ 1u);
+  }
+  if (lane == 0) phases[warp] = phase;
+  store_mma_partial<D>(st, pv, warp, packed, lane);
+}
+
+// f32 attention: warp w handles head w % G for the keys j = w / G, w / G + nwg, ...
+// (nwg = ncw / G warps per head). Direct loads, lanes over the head dim.
+template <int D, typename KeyFn>
+__device__ void attend_keys_f32(const float* __restrict__ Qg, const float* __restrict__ Kp,
+                                const float* __restrict__ Vp, KeyFn keys, int cnt, int nrows, int G, float scale,
+                                int ncw, const PartialView& pv) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (warp >= ncw) return;
+  const int nwg = max(1, ncw / G);
+  if (warp >= nwg * G) {
+    store_empty_partial(pv, warp, lane);
+    return;
+  }
+  const int h = warp % G;
+  const float scale_log2 = scale * LOG2E;
+  float q[D / 32], acc[D / 32];
 #pragma unroll
-  for (int h = 0; h < 8; ++h) {
-    if (h < pv.G) {
-      if (lane == 0) {
-        pv.pm[w * pv.G + h] = st.m[h];
-        pv.pl[w * pv.G + h] = st.l[h];
-      }
-      float* po = pv.po + ((size_t)w * pv.G + h) * D;
+  for (int i = 0; i < D / 32; ++i) {
+    q[i] = Qg[h * D + lane + 32 * i] * scale_log2;
+    acc[i] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  for (int j = warp / G; j < cnt; j += nwg) {
+    const int row = min(max(keys(j), 0), nrows - 1);
+    const float* kr = Kp + (size_t)row * D;
+    const float* vr = Vp + (size_t)row * D;
+    float s = 0.f;
 #pragma unroll
-      for (int i = 0; i < D / 32; ++i) po[lane + 32 * i] = st.acc[h][i];
+    for (int i = 0; i < D / 32; ++i) s = fmaf(q[i], kr[lane + 32 * i], s);
+    s = warp_sum(s);
+    const float m_new = fmaxf(m, s);
+    const float alpha = exp2f(m - m_new);
+    const float pr = exp2f(s - m_new);
+    l = l * alpha + pr;
+    m = m_new;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) acc[i] = acc[i] * alpha + pr * vr[lane + 32 * i];
+  }
+  for (int hh = 0; hh < G; ++hh) {
+    if (lane == 0) {
+      pv.pm[warp * G + hh] = hh == h ? m : -INFINITY;
+      pv.pl[warp * G + hh] = hh == h ? l : 0.f;
     }
   }
+  float* po = pv.po + ((size_t)warp * G + h) * D;
+#pragma unroll
+  for (int i = 0; i < D / 32; ++i) po[lane + 32 * i] = acc[i];
 }
 
 // Merges nslots partial slots into (M[h], Lsum[h], O[h][D]) with a fixed
-// slot order; all threads of the block participate. Slot results with no
-// keys have m = -inf and contribute nothing.
-__device__ __forceinline__ void merge_partials(const PartialView& pv, int nslots, float* M, float* Lsum,
-                                               float* O) {
+// slot order; all threads of the block participate. Slots with m = -inf
+// contribute nothing.
+__device__ __forceinline__ void merge_partials(const PartialView& pv, int nslots, float* M, float* Lsum, float* O) {
   const int G = pv.G, D = pv.D;
   for (int h = threadIdx.x; h < G; h += blockDim.x) {
     float mm = -INFINITY;

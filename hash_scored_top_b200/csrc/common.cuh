@@ -18,6 +18,32 @@ __device__ unsigned int g_error_word = 0u;
 constexpr unsigned ERR_TIMEOUT = 1u;   // a bounded wait gave up
 constexpr unsigned ERR_LAYOUT = 2u;    // a launch's shared-memory plan did not fit
 
+// ---------------------------------------------------------------- bucket-ID cache layout
+// Each key stores its L bucket IDs in LP bytes, split in chunks of S_0, S_1
+// tables: L <= 16 -> [16]; L <= 32 -> [32]; L <= 48 -> [32, 16]; L <= 64 ->
+// [32, 32]. Inside chunk c (tables 32c ..), byte j of key n holds the ID of
+// table 32c + (j + n) mod S_c, zero where that table is >= L. A warp scoring
+// 32 consecutive keys then reads, at step j, 32 different tables -- one per
+// lane -- which is what makes its shared-memory lookups conflict-free.
+__host__ __device__ constexpr int ids_bytes_per_key(int L) {
+  return L <= 16 ? 16 : L <= 32 ? 32 : L <= 48 ? 48 : 64;
+}
+__host__ __device__ constexpr int id_chunk_size(int L, int chunk) {
+  return chunk == 0 ? (L <= 16 ? 16 : 32) : (L <= 48 ? 16 : 32);
+}
+// Byte position of table l's ID inside the bytes of key n.
+__host__ __device__ inline int id_byte_pos(int L, int l, int n) {
+  const int c = l >= 32 ? 1 : 0;
+  const int S = id_chunk_size(L, c);
+  return 32 * c + (((l - 32 * c - n) % S) + S) % S;
+}
+// Table whose ID sits at byte b of key n (>= L: padding).
+__host__ __device__ inline int id_byte_table(int L, int b, int n) {
+  const int c = b >= 32 ? 1 : 0;
+  const int S = id_chunk_size(L, c);
+  return 32 * c + ((b - 32 * c) + n) % S;
+}
+
 // ---------------------------------------------------------------- loads
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 r;
@@ -101,6 +127,59 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
   return v;
+}
+
+// ---------------------------------------------------------------- mbarriers and bulk copies
+__device__ __forceinline__ void mbar_init(uint32_t addr, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(addr), "r"(count) : "memory");
+}
+
+// Makes mbarrier initialisations visible to the async (bulk copy) proxy.
+__device__ __forceinline__ void fence_mbar_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+// Orders this thread's earlier shared-memory accesses (generic proxy) before
+// later bulk copies into the same memory (async proxy).
+__device__ __forceinline__ void fence_proxy_async_shared() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t addr, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(addr), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete, for at most about
+// one second of SM clock; on giving up sets ERR_TIMEOUT and returns false.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity) {
+  if (mbar_try_wait(addr, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(addr, parity)) {
+    if (clock64() - t0 > 2000000000LL) {
+      atomicOr(&g_error_word, ERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// 1-D bulk copy (TMA engine) global -> this CTA's shared memory, completing
+// `bytes` of transaction count on the mbarrier. Both addresses 16-byte
+// aligned, bytes a multiple of 16. No multicast.
+__device__ __forceinline__ void bulk_copy_g2s(uint32_t dst, const void* src, uint32_t bytes, uint32_t mbar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(mbar)
+               : "memory");
 }
 
 // ---------------------------------------------------------------- bf16 pairs

@@ -1,25 +1,24 @@
 // Soft collision scoring, SOCKET step 3 (SOCKET technical summary, section
 // 中核メカニズム：ソフト LSH, step 3): score_n = |v_n| * sum_l T_l(id_l(n)).
 //
-// Work unit: one warp scores one block of 32 consecutive keys. The bucket
-// IDs are stored key-block interleaved (per 32-key block, table l's 32 IDs
-// are 32 contiguous bytes), so lane t loads the 32 IDs of table t of the block
-// with two 16-byte loads -- a warp reads the block's L*32 bytes fully
-// coalesced. Lane t then looks up T_t(id) for each of the 32 keys; all lanes
-// read a different table column at every step, so the 32 lookups of a warp
-// instruction fall in 32 different banks (conflict-free by construction).
+// Work unit: one lane scores one key; a warp scores 32 consecutive keys.
+// Lane t loads its key's LP ID bytes (the rotated key-major layout of
+// common.cuh) with 16-byte loads; a warp reads 32 * LP contiguous bytes.
+// At step j the byte the lane reads belongs to table 32c + (j + t) mod S_c
+// (t = key index mod 32), so the 32 lanes look up 32 different tables.
 //
-// Shared-memory table layout: row b (bucket) at byte b*256, column l at l*4,
-// 256 rows x 64 columns of f32 (64 KB), placed at a 64 KB-aligned shared
-// address. The address of entry (id, column) is then the column's address
-// with byte 1 replaced by the ID -- a single byte-permute per lookup.
-// Rows >= 2^P and columns >= L hold zero, so any stored byte is a valid row.
+// Shared-memory tables: one per ID chunk, 64 KB each at a 64 KB-aligned
+// shared address; row b (bucket) at byte b*256, column x at 4x, and column x
+// holds table 32c + (x mod S_c) -- every table appears 64 / S_c times. Lane t
+// at step j reads column t + j (< 64), whose bank is (t + j) mod 32: the 32
+// lookups of a warp hit 32 banks. The address is the lane's column-0 address
+// with byte 1 replaced by the ID (one byte-permute) plus the compile-time
+// offset 4j in the load instruction. Rows >= 2^P and tables >= L hold zero.
 //
-// The 32 per-table values of a key live in 32 different lanes; a butterfly
-// reduce-scatter (5 exchange rounds) leaves lane t with key t's sum. The sum
-// is a fixed binary tree of depth 5 (6 with two table chunks), which bounds
-// the f32 relative error of a score by 8 * 2^-24 (entry rounding, tree,
-// product with the norm) -- below the 1e-6 near-tie window of the selection.
+// The LP values of a key go to 8 (16 for LP > 32) partial sums of at most 4
+// terms that are added in a fixed tree, so an f32 score carries at most 9
+// roundings of 2^-24 (entry, sums, norm product) -- below the 1e-6 relative
+// near-tie window of the selection.
 #pragma once
 
 #include "common.cuh"
@@ -29,72 +28,74 @@ namespace hst {
 constexpr int TABLE_BYTES = 65536;     // 256 buckets x 64 columns x 4 bytes
 constexpr int TABLE_COLS = 64;
 
-// Ids of one 32-key block for this lane: chunk c covers table 32c + lane.
-template <int NCHUNK>
-struct IdBlock {
-  uint4 w[NCHUNK][2];
+template <int LP>
+struct KeyIds {
+  uint4 w[LP / 16];
   uint16_t norm;
 };
 
-template <int NCHUNK, bool NORM = true>
-__device__ __forceinline__ void load_id_block(IdBlock<NCHUNK>& blk, const uint8_t* __restrict__ ids_blk,
-                                              const __half* __restrict__ norms_blk, int L, int lane) {
+template <int LP, bool NORM>
+__device__ __forceinline__ void load_key_ids(KeyIds<LP>& k, const uint8_t* __restrict__ ids_key,
+                                             const __half* __restrict__ norm_key) {
 #pragma unroll
-  for (int c = 0; c < NCHUNK; ++c) {
-    const int l = 32 * c + lane;
-    if (l < L) {
-      const uint8_t* p = ids_blk + (size_t)l * 32;
-      blk.w[c][0] = ldg_stream(p);
-      blk.w[c][1] = ldg_stream(p + 16);
-    } else {
-      blk.w[c][0] = make_uint4(0, 0, 0, 0);
-      blk.w[c][1] = make_uint4(0, 0, 0, 0);
-    }
-  }
-  if (NORM) blk.norm = ldg_u16(norms_blk + lane);
+  for (int i = 0; i < LP / 16; ++i) k.w[i] = ldg_stream(ids_key + 16 * i);
+  if (NORM) k.norm = ldg_u16(norm_key);
 }
 
-__device__ __forceinline__ uint32_t word_of(const uint4 (&w)[2], int n) {
-  const uint4& q = w[n >> 4];
-  const int e = (n >> 2) & 3;
-  return e == 0 ? q.x : e == 1 ? q.y : e == 2 ? q.z : q.w;
+template <int J>
+__device__ __forceinline__ float lds_imm(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared.f32 %0, [%1+%2];" : "=f"(v) : "r"(addr), "n"(4 * J));
+  return v;
 }
 
-// Sum over lanes of v[n] lands in lane n (v[0] on return).
-__device__ __forceinline__ float butterfly_reduce_scatter(float (&v)[32], int lane) {
-#pragma unroll
-  for (int s = 16; s >= 1; s >>= 1) {
-    const bool upper = (lane & s) != 0;
-#pragma unroll
-    for (int i = 0; i < s; ++i) {
-      const float send = upper ? v[i] : v[i + s];
-      const float keep = upper ? v[i + s] : v[i];
-      v[i] = keep + __shfl_xor_sync(FULL, send, s);
-    }
-  }
-  return v[0];
-}
+// Number of partial sums: every partial gets at most 4 terms.
+template <int LP>
+struct ScoreAcc {
+  static constexpr int N = LP > 32 ? 16 : 8;
+};
 
-// Score (f32, >= 0) of key (block start + lane). col_addr[c] is the shared
-// address of table column 32c + lane in bucket row 0.
-template <int NCHUNK, bool NORM = true>
-__device__ __forceinline__ float score_id_block(const IdBlock<NCHUNK>& blk, const uint32_t (&col_addr)[NCHUNK],
-                                                int lane) {
-  float v[32];
-#pragma unroll
-  for (int c = 0; c < NCHUNK; ++c) {
-#pragma unroll
-    for (int n = 0; n < 32; ++n) {
-      const uint32_t w = word_of(blk.w[c], n);
-      const uint32_t addr = __byte_perm(col_addr[c], w, 0x3240u | ((uint32_t)(n & 3) << 4));
-      const float t = lds_f32(addr);
-      v[n] = (c == 0) ? t : v[n] + t;
-    }
+template <int LP, int J>
+struct ScoreStep {
+  // Looks up byte J of the key (unrolled over J by recursion).
+  static __device__ __forceinline__ void run(const KeyIds<LP>& k, uint32_t col0, uint32_t col1,
+                                             float (&acc)[ScoreAcc<LP>::N]) {
+    constexpr int NA = ScoreAcc<LP>::N;
+    constexpr int C = J >= 32 ? 1 : 0;
+    constexpr int JL = J - 32 * C;
+    const uint4& q = k.w[J / 16];
+    constexpr int E = (J / 4) % 4;
+    const uint32_t w = E == 0 ? q.x : E == 1 ? q.y : E == 2 ? q.z : q.w;
+    const uint32_t a = __byte_perm(C ? col1 : col0, w, 0x3240u | ((uint32_t)(J & 3) << 4));
+    const float v = lds_imm<JL>(a);
+    if (J < NA) acc[J % NA] = v;
+    else acc[J % NA] += v;
+    ScoreStep<LP, J + 1>::run(k, col0, col1, acc);
   }
-  const float mass = butterfly_reduce_scatter(v, lane);
+};
+template <int LP>
+struct ScoreStep<LP, LP> {
+  static __device__ __forceinline__ void run(const KeyIds<LP>&, uint32_t, uint32_t, float (&)[ScoreAcc<LP>::N]) {}
+};
+
+// Score (f32, >= 0) of this lane's key. colX = shared address of column
+// `lane` (row 0) of the table of chunk X.
+template <int LP, bool NORM>
+__device__ __forceinline__ float score_key(const KeyIds<LP>& k, uint32_t col0, uint32_t col1) {
+  constexpr int NA = ScoreAcc<LP>::N;
+  float acc[NA];
+  ScoreStep<LP, 0>::run(k, col0, col1, acc);
+#pragma unroll
+  for (int w = NA / 2; w >= 1; w /= 2)
+#pragma unroll
+    for (int i = 0; i < w; ++i) acc[i] = acc[2 * i] + acc[2 * i + 1];
+  const float mass = acc[0];
   if (!NORM) return mass;    // hard-hash scores: exact small integers
-  const float s = __half2float(__ushort_as_half(blk.norm)) * mass;
+  const float s = __half2float(__ushort_as_half(k.norm)) * mass;
   return fmaxf(s, 0.0f);     // scores are >= 0; NaN (0 * inf) maps to 0
 }
+
+// Column x of chunk c's table holds table 32c + (x mod S_c).
+__host__ __device__ inline int column_table(int L, int c, int x) { return 32 * c + x % id_chunk_size(L, c); }
 
 }  // namespace hst

@@ -3,43 +3,46 @@
 // the top-k keys are chosen deterministically).
 //
 // The keys of one (batch, KV-head) pair are split over the C CTAs of a
-// cluster; CTA c holds the 32-bit sort keys of its slice in shared memory.
-// Sort keys are the bit patterns of non-negative f32 scores (monotone as
-// unsigned integers) or small non-negative integers (hard-hash scores).
-// Selection is a most-significant-digit radix select over up to three digit
-// levels: every CTA histograms the digit of its keys that match the prefix
-// found so far, the histograms are summed across the cluster through
-// distributed shared memory, and the bin holding the k-th largest key is
-// found by a descending scan. A level stops early when the whole bin is
-// taken. The final level resolves exact ties: among keys equal to the
-// threshold, the ones with the lowest key index are taken (CTAs hold
-// ascending index ranges, so CTA order then lane order is index order).
-// The chosen indices are written in ascending order.
+// cluster; CTA c holds the 32-bit sort keys of an ascending index range in
+// shared memory. Sort keys are the bit patterns of non-negative f32 scores,
+// which order like the scores as unsigned integers.
+//
+// Selection is a most-significant-digit radix select over three digit levels
+// (bits 30..20, 19..9, 8..0): every CTA histograms the digit of its keys that
+// match the prefix found so far, each CTA sums the cluster's histograms
+// through distributed shared memory, and a descending scan finds the bin that
+// holds the k-th largest key. A level ends the search early when the whole
+// bin is taken. After the last level the threshold t is exact and the tie
+// rule applies: among keys equal to t, the lowest indices are taken.
+//
+// Output order: every CTA counts its selected keys, publishes (greater,
+// equal) counts to the whole cluster, and writes its keys in ascending index
+// order at the offset of the CTAs before it, so the result is ascending.
 #pragma once
+
+#include <cooperative_groups.h>
 
 #include "common.cuh"
 
 namespace hst {
 
+namespace cg = cooperative_groups;
+
 constexpr int SEL_MAX_C = 16;
+constexpr int SEL_LEVELS = 3;
+__host__ __device__ constexpr int sel_bits(int level) { return level == 2 ? 9 : 11; }
+__host__ __device__ constexpr int sel_shift(int level) { return level == 0 ? 20 : level == 1 ? 9 : 0; }
 
-// One digit level: key bits [shift, shift + bits).
-struct DigitLevel {
-  int shift;
-  int bits;
-};
-
-// Broadcast results of the selection, in shared memory.
+// Broadcast results and scratch of the selection, in shared memory.
 struct SelShared {
-  uint32_t bin;                 // bin of the k-th largest key at the current level
-  uint32_t above;               // cluster-wide count in bins above it
-  uint32_t total_in_bin;        // cluster-wide count in the bin
-  uint32_t warp_tmp[32];        // block-scan scratch
-  uint32_t red[32][SEL_MAX_C];  // per-warp, per-CTA partial sums
-  uint32_t above_c[SEL_MAX_C];  // per-CTA count above the bin (this level)
-  uint32_t eq_c[SEL_MAX_C];     // per-CTA count in the bin (this level)
-  uint32_t cnt_w[32][2];        // compaction: per-warp (greater, equal) counts
-  uint32_t off_w[32][2];        // compaction: per-warp (selected, equal) offsets
+  uint32_t bin;                  // bin of the k-th largest key at the current level
+  uint32_t above;                // cluster-wide count in bins above it
+  uint32_t total_in_bin;         // cluster-wide count in the bin
+  uint32_t pad;
+  uint32_t warp_tmp[32];         // block-scan scratch
+  uint32_t cnt_w[32][2];         // compaction: per-warp (greater, equal) counts
+  uint32_t off_w[32][2];         // compaction: per-warp (selected, equal) offsets
+  uint32_t counts[SEL_MAX_C][2]; // (greater, equal) published by every CTA of the cluster
 };
 
 // Block-wide exclusive scan of one value per thread (thread order).
@@ -68,164 +71,150 @@ __device__ __forceinline__ uint32_t block_exclusive_scan(uint32_t v, SelShared* 
   return before + x - v;
 }
 
-// Cluster-wide resolution of one histogram level. hist_addr is the shared
-// address of this CTA's histogram (nbins u32; the same offset in every CTA).
-// need >= 1 keys are still to be taken among keys matching the prefix.
-// Writes sh->bin / above / total_in_bin and, for every CTA c < C,
-// sh->above_c[c] and sh->eq_c[c].
-__device__ void resolve_level(uint32_t hist_addr, int nbins, uint32_t need, int C, SelShared* sh) {
-  const int tid = threadIdx.x, nthr = blockDim.x;
-  const int lane = tid & 31, warp = tid >> 5, nw = nthr >> 5;
-  const int bpt = (nbins + nthr - 1) / nthr;          // bins per thread (descending order)
+// Cluster-wide resolution of one histogram level of nbins bins; thread t
+// handles bins [nbins - (t + 1) * BPT, nbins - t * BPT) (none once that is
+// negative). `hist` is this CTA's histogram (same shared offset in every CTA).
+// need >= 1 keys are still to be taken among the keys that match the prefix.
+// Writes sh->bin, sh->above, sh->total_in_bin.
+template <int BPT>
+__device__ void resolve_level(const uint32_t* hist, int nbins, uint32_t need, int C, SelShared* sh) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int tid = threadIdx.x;
+  const int base = nbins - (tid + 1) * BPT;            // this thread: bins [base, base + BPT)
+  const bool mine = base >= 0;
   if (tid == 0) {            // defaults, overwritten by the thread that holds the k-th key
     sh->bin = 0;
     sh->above = 0;
     sh->total_in_bin = 0;
   }
-  uint32_t local = 0;
-  for (int j = 0; j < bpt; ++j) {
-    const int bin = nbins - 1 - (tid * bpt + j);
-    if (bin >= 0) {
-      for (int c = 0; c < C; ++c) local += ld_cluster_u32(mapa(hist_addr + 4u * bin, c));
-    }
-  }
-  const uint32_t before = block_exclusive_scan(local, sh);
-  if (before < need && need <= before + local) {
-    uint32_t run = before;
-    for (int j = 0; j < bpt; ++j) {
-      const int bin = nbins - 1 - (tid * bpt + j);
-      if (bin < 0) break;
-      uint32_t tot = 0;
-      for (int c = 0; c < C; ++c) tot += ld_cluster_u32(mapa(hist_addr + 4u * bin, c));
-      if (run + tot >= need) {
-        sh->bin = (uint32_t)bin;
-        sh->above = run;
-        sh->total_in_bin = tot;
-        break;
+  uint32_t tot[BPT];
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) tot[j] = 0;
+  if (mine) {
+    for (int c = 0; c < C; ++c) {
+      const uint32_t* h = cluster.map_shared_rank(hist, c) + base;
+      if constexpr (BPT % 4 == 0) {
+#pragma unroll
+        for (int j = 0; j < BPT; j += 4) {
+          const uint4 v = *reinterpret_cast<const uint4*>(h + j);
+          tot[j] += v.x; tot[j + 1] += v.y; tot[j + 2] += v.z; tot[j + 3] += v.w;
+        }
+      } else if constexpr (BPT % 2 == 0) {
+#pragma unroll
+        for (int j = 0; j < BPT; j += 2) {
+          const uint2 v = *reinterpret_cast<const uint2*>(h + j);
+          tot[j] += v.x; tot[j + 1] += v.y;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) tot[j] += h[j];
       }
-      run += tot;
     }
   }
-  __syncthreads();
-  const int bin_sel = min((int)sh->bin, nbins - 1);
-  // per-CTA counts above the bin
-  for (int c = 0; c < C; ++c) {
-    uint32_t part = 0;
-    for (int j = 0; j < bpt; ++j) {
-      const int bin = nbins - 1 - (tid * bpt + j);
-      if (bin > bin_sel) part += ld_cluster_u32(mapa(hist_addr + 4u * bin, c));
+  uint32_t local = 0;
+#pragma unroll
+  for (int j = 0; j < BPT; ++j) local += tot[j];
+  const uint32_t before = block_exclusive_scan(local, sh);   // keys in bins above this thread's
+  if (mine && before < need && need <= before + local) {
+    uint32_t run = before;
+#pragma unroll
+    for (int j = BPT - 1; j >= 0; --j) {                      // descending bins
+      if (run < need && need <= run + tot[j]) {
+        sh->bin = (uint32_t)(base + j);
+        sh->above = run;
+        sh->total_in_bin = tot[j];
+      }
+      run += tot[j];
     }
-    part = warp_sum(part);
-    if (lane == 0) sh->red[warp][c] = part;
-  }
-  __syncthreads();
-  if (tid < C) {
-    uint32_t s = 0;
-    for (int w = 0; w < nw; ++w) s += sh->red[w][tid];
-    sh->above_c[tid] = s;
-    sh->eq_c[tid] = ld_cluster_u32(mapa(hist_addr + 4u * bin_sel, tid));
   }
   __syncthreads();
 }
 
-// Histogram pass over this CTA's keys: keys whose bits above `lv.shift + lv.bits`
-// ... i.e. (key >> pshift) == prefix are counted in bin (key >> lv.shift) & mask.
-// pshift == 32 means "no prefix" (all keys).
+// Counts keys matching the prefix in bin (key >> shift) & mask of `hist`.
+// pshift >= 32 means "no prefix" (all keys).
 template <typename KeyAt>
-__device__ __forceinline__ void histogram_pass(KeyAt key_at, int n, DigitLevel lv, int pshift, uint32_t prefix,
-                                               uint32_t* hist) {
-  const uint32_t mask = (1u << lv.bits) - 1u;
+__device__ __forceinline__ void histogram_pass(KeyAt key_at, int n, int shift, int bits, int pshift,
+                                               uint32_t prefix, uint32_t* hist) {
+  const uint32_t mask = (1u << bits) - 1u;
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
     const uint32_t k = key_at(i);
     const bool match = pshift >= 32 ? true : ((k >> pshift) == prefix);
-    if (match) atomicAdd(&hist[(k >> lv.shift) & mask], 1u);
+    if (match) atomicAdd(&hist[(k >> shift) & mask], 1u);
   }
 }
 
-// Result of the cluster selection for this CTA.
-struct SelPlan {
-  uint32_t t;          // threshold key: select keys > t, and ties == t by rank
-  uint32_t take_eq;    // ties == t this CTA takes (UINT_MAX: all)
-  uint32_t out_off;    // position of this CTA's first selected key in the output
-  uint32_t n_sel;      // keys this CTA selects
+__device__ __forceinline__ void sel_stamp(unsigned long long* ts, int phase) {
+  if (ts != nullptr && threadIdx.x == 0) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    ts[blockIdx.x * 24 + phase] = t;
+  }
+}
+
+// Threshold of the pair, identical in every CTA of the cluster.
+struct SelThreshold {
+  uint32_t t;        // keys > t are selected
+  uint32_t take_eq;  // keys == t: the first take_eq of them in index order (UINT_MAX: all)
 };
 
-// Full selection over up to 3 levels. `hist[l]` are this CTA's zeroed
-// histograms (u32, 1 << levels[l].bits bins); level 0 is filled by the caller
-// before the cluster barrier that precedes this call (sync_before_first).
-// k: keys to select for the pair (1 <= k <= total keys). rank: this CTA.
-template <typename KeyAt>
-__device__ SelPlan cluster_select(KeyAt key_at, int n_local, const DigitLevel* levels, int nlevels,
-                                  uint32_t* const* hist, uint32_t k, int C, int rank, SelShared* sh) {
+// The three-level search (NT threads per CTA). hist[0] holds this CTA's
+// level-0 histogram and the cluster has synchronised since it was filled;
+// hist[1], hist[2] are zeroed.
+template <int NT, typename KeyAt>
+__device__ SelThreshold cluster_threshold(KeyAt key_at, int n_local, uint32_t* const* hist, uint32_t k, int C,
+                                          SelShared* sh, unsigned long long* ts = nullptr) {
   uint32_t need = k;
-  uint32_t prefix = 0;        // digits found so far (at the current level's granularity)
+  uint32_t prefix = 0;
   int pshift = 32;
-  uint32_t acc_above[SEL_MAX_C];
+  SelThreshold th;
 #pragma unroll
-  for (int c = 0; c < SEL_MAX_C; ++c) acc_above[c] = 0;
-  SelPlan plan;
-  for (int lvl = 0; lvl < nlevels; ++lvl) {
-    const DigitLevel lv = levels[lvl];
+  for (int lvl = 0; lvl < SEL_LEVELS; ++lvl) {
     if (lvl > 0) {
-      histogram_pass(key_at, n_local, lv, pshift, prefix, hist[lvl]);
+      histogram_pass(key_at, n_local, sel_shift(lvl), sel_bits(lvl), pshift, prefix, hist[lvl]);
       __syncthreads();
+      sel_stamp(ts, 14 + 2 * lvl);
       cluster_sync();
+      sel_stamp(ts, 15 + 2 * lvl);
     }
-    resolve_level(smem_u32(hist[lvl]), 1 << lv.bits, need, C, sh);
-    const uint32_t bin = sh->bin;
-    for (int c = 0; c < C; ++c) acc_above[c] += sh->above_c[c];
+    constexpr int B01 = (1 << 11) / NT > 0 ? (1 << 11) / NT : 1;
+    constexpr int B2 = (1 << 9) / NT > 0 ? (1 << 9) / NT : 1;
+    if (lvl < 2) resolve_level<B01>(hist[lvl], 1 << 11, need, C, sh);
+    else resolve_level<B2>(hist[lvl], 1 << 9, need, C, sh);
     need -= sh->above;
-    prefix = (prefix << lv.bits) | bin;
-    pshift = lv.shift;
-    const bool whole = (need == sh->total_in_bin);
-    if (whole || lvl == nlevels - 1) {
-      // threshold = smallest key in the bin (whole) or the exact key (last level, shift 0)
-      plan.t = prefix << lv.shift;
-      uint32_t eq_before = 0, sel_before = 0;
-      for (int c = 0; c < C; ++c) {
-        uint32_t take;
-        if (whole) {
-          take = sh->eq_c[c];
-        } else {
-          const uint32_t left = need > eq_before ? need - eq_before : 0u;
-          take = left < sh->eq_c[c] ? left : sh->eq_c[c];
-        }
-        const uint32_t sel_c = acc_above[c] + take;
-        if (c == rank) {
-          plan.out_off = sel_before;
-          plan.n_sel = sel_c;
-          plan.take_eq = whole ? 0xffffffffu : take;
-        }
-        sel_before += sel_c;
-        eq_before += sh->eq_c[c];
-      }
+    prefix = (prefix << sel_bits(lvl)) | sh->bin;
+    pshift = sel_shift(lvl);
+    const bool whole = need == sh->total_in_bin;
+    if (whole || lvl == SEL_LEVELS - 1) {
+      th.t = prefix << sel_shift(lvl);          // smallest key of the bin (exact key at the last level)
+      th.take_eq = whole ? 0xffffffffu : need;  // whole bin: every key >= t
       break;
     }
   }
-  return plan;
+  return th;
 }
 
-// Ordered compaction of this CTA's selected keys. Keys i in [0, n) with
-// key > t, or key >= t when take_eq == UINT_MAX, or key == t among the first
-// take_eq such keys in index order, are emitted in ascending i at output
-// positions plan.out_off, plan.out_off + 1, ... via emit(pos, i).
+// Ordered compaction of this CTA's selected keys (ascending index i in [0, n)):
+// pass 1 counts, the counts are exchanged across the cluster, pass 2 calls
+// emit(pos, i) with the key's position in the pair's ascending output.
+// rank: this CTA's rank; keys of CTA c precede those of CTA c + 1.
 template <typename KeyAt, typename Emit>
-__device__ void ordered_compact(KeyAt key_at, int n, const SelPlan& plan, SelShared* sh, Emit emit) {
+__device__ void ordered_compact(KeyAt key_at, int n, const SelThreshold& th, int C, int rank, SelShared* sh,
+                                Emit emit, unsigned long long* ts = nullptr) {
+  cg::cluster_group cluster = cg::this_cluster();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const bool all_eq = plan.take_eq == 0xffffffffu;
+  const bool all_eq = th.take_eq == 0xffffffffu;
   const int nchunks = (n + 31) / 32;
   const int per_warp = (nchunks + nw - 1) / nw;
   const int c0 = warp * per_warp;
   const int c1 = min(nchunks, c0 + per_warp);
-  // pass 1: per-warp counts of (key > t) and (key == t)
+  // pass 1: per-warp counts of (key > t) and (key == t); "> t" means ">= t" when all ties are taken
   uint32_t n_gt = 0, n_eq = 0;
   for (int ch = c0; ch < c1; ++ch) {
     const int i = ch * 32 + lane;
-    uint32_t k = 0;
-    bool valid = i < n;
-    if (valid) k = key_at(i);
-    const bool gt = valid && (all_eq ? k >= plan.t : k > plan.t);
-    const bool eq = valid && !all_eq && k == plan.t;
+    const bool valid = i < n;
+    const uint32_t k = valid ? key_at(i) : 0u;
+    const bool gt = valid && (all_eq ? k >= th.t : k > th.t);
+    const bool eq = valid && !all_eq && k == th.t;
     n_gt += __popc(__ballot_sync(FULL, gt));
     n_eq += __popc(__ballot_sync(FULL, eq));
   }
@@ -234,33 +223,63 @@ __device__ void ordered_compact(KeyAt key_at, int n, const SelPlan& plan, SelSha
     sh->cnt_w[warp][1] = n_eq;
   }
   __syncthreads();
+  // CTA totals, published to every CTA of the cluster
+  if (threadIdx.x < C) {
+    uint32_t g = 0, e = 0;
+    for (int w = 0; w < nw; ++w) {
+      g += sh->cnt_w[w][0];
+      e += sh->cnt_w[w][1];
+    }
+    uint32_t* dst = cluster.map_shared_rank(&sh->counts[rank][0], (unsigned)threadIdx.x);
+    dst[0] = g;
+    dst[1] = e;
+  }
+  sel_stamp(ts, 19);
+  cluster_sync();
+  sel_stamp(ts, 20);
+  // this CTA's tie quota and output offset, from the published counts
   if (threadIdx.x == 0) {
-    uint32_t sel = 0, eq = 0;
+    uint32_t eq_before = 0, sel_before = 0, my_take = 0, my_off = 0;
+    for (int c = 0; c < C; ++c) {
+      const uint32_t e = sh->counts[c][1];
+      const uint32_t left = th.take_eq > eq_before ? th.take_eq - eq_before : 0u;
+      const uint32_t take = all_eq ? 0u : (left < e ? left : e);
+      if (c == rank) {
+        my_take = take;
+        my_off = sel_before;
+      }
+      sel_before += sh->counts[c][0] + take;
+      eq_before += e;
+    }
+    // per-warp offsets inside this CTA
+    uint32_t sel = my_off, eqr = 0;
     for (int w = 0; w < nw; ++w) {
       sh->off_w[w][0] = sel;
-      sh->off_w[w][1] = eq;
-      const uint32_t left = all_eq ? 0u : (plan.take_eq > eq ? plan.take_eq - eq : 0u);
+      sh->off_w[w][1] = eqr;
+      const uint32_t left = my_take > eqr ? my_take - eqr : 0u;
       const uint32_t e = sh->cnt_w[w][1];
       sel += sh->cnt_w[w][0] + (left < e ? left : e);
-      eq += e;
+      eqr += e;
     }
+    sh->pad = my_take;
   }
   __syncthreads();
-  // pass 2: emit in order
+  sel_stamp(ts, 21);
+  const uint32_t my_take = sh->pad;
+  // pass 2: emit in index order
   uint32_t sel_run = sh->off_w[warp][0];
   uint32_t eq_run = sh->off_w[warp][1];
   const uint32_t ltmask = lanemask_lt();
   for (int ch = c0; ch < c1; ++ch) {
     const int i = ch * 32 + lane;
-    uint32_t k = 0;
     const bool valid = i < n;
-    if (valid) k = key_at(i);
-    const bool gt = valid && (all_eq ? k >= plan.t : k > plan.t);
-    const bool eq = valid && !all_eq && k == plan.t;
+    const uint32_t k = valid ? key_at(i) : 0u;
+    const bool gt = valid && (all_eq ? k >= th.t : k > th.t);
+    const bool eq = valid && !all_eq && k == th.t;
     const uint32_t meq = __ballot_sync(FULL, eq);
-    const bool take = gt || (eq && (eq_run + __popc(meq & ltmask)) < plan.take_eq);
+    const bool take = gt || (eq && (eq_run + __popc(meq & ltmask)) < my_take);
     const uint32_t msel = __ballot_sync(FULL, take);
-    if (take) emit(plan.out_off + sel_run + __popc(msel & ltmask), i);
+    if (take) emit(sel_run + __popc(msel & ltmask), i);
     sel_run += __popc(msel);
     eq_run += __popc(meq);
   }

@@ -4,6 +4,8 @@
 // attend.cuh for the steps.
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "attend.cuh"
 #include "common.cuh"
 #include "hash_kernels.cuh"
@@ -13,22 +15,22 @@
 
 namespace hst {
 
+namespace cg = cooperative_groups;
+
 // ---------------------------------------------------------------- shared constants
 constexpr int SMEM_BASE_EXPECTED = 1024;         // dynamic shared window start on sm_100
 constexpr int SMEM_DYN_MAX = 232448;             // 227 KB opt-in per block
-constexpr int HIST1_BITS = 11, HIST2_BITS = 11, HIST3_BITS = 9;
-constexpr int FUSED_THREADS = 256;
+__host__ __device__ constexpr int hist_words(int level) { return 1 << sel_bits(level); }
+constexpr int FUSED_THREADS = 1024;              // 32 warps: enough loads in flight to stream HBM
 constexpr int FUSED_WARPS = FUSED_THREADS / 32;
-constexpr int SCORE_PF = 4;                      // 32-key blocks in flight per warp
+constexpr int SCORE_PF = 2;                      // 32-key blocks in flight per warp
+constexpr int ATTEND_THREADS = 256;              // the attention kernel
+constexpr int ATTEND_WARPS = ATTEND_THREADS / 32;
+constexpr int ATTEND_MAX_SPLITS = 128;           // one head's partials fit in the warp slots
 
 __device__ __forceinline__ uint32_t key_of(float s) { return __float_as_uint(s); }
 
-// Digit levels for f32 score keys (bit 31 is always 0 for s >= 0).
-__device__ __forceinline__ void f32_levels(DigitLevel (&lv)[3]) {
-  lv[0] = {20, HIST1_BITS};
-  lv[1] = {9, HIST2_BITS};
-  lv[2] = {0, HIST3_BITS};
-}
+__host__ __device__ constexpr int table_chunks(int LP) { return LP > 32 ? 2 : 1; }
 
 struct FusedParams {
   const void* Q;
@@ -38,39 +40,56 @@ struct FusedParams {
   const uint8_t* ids;
   const __half* norms;
   float* O;
-  int* idx_out;
+  int* idx_out;                   // [pairs][k] ascending (always written)
+  unsigned int* counters;         // [pairs] zeroed here for the attention kernel's merge (may be null)
+  unsigned long long* phase_ts;   // optional: [grid][PHASES] globaltimer stamps (profiling)
   int Hq, Hkv, Ncap, N, L, P, k, C, blocks_per_cta, chunk;
   float tau, scale;
 };
 
-// Shared-memory plan of the fused kernel (all addresses are shared-window
-// addresses). The 64 KB table sits at a 64 KB-aligned address; sort keys
-// fill segment A (after the fixed items) and then segment B (after the table).
+constexpr int PHASES = 24;
+
+__device__ __forceinline__ void stamp(unsigned long long* ts, int phase) {
+  if (ts != nullptr && threadIdx.x == 0) {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    ts[blockIdx.x * PHASES + phase] = t;
+    if (phase == 0 || phase == 7) ts[blockIdx.x * PHASES + 22 + (phase == 7)] = (unsigned long long)clock64();
+  }
+}
+
+// Where the sort keys of a CTA live: the first nA in segment A, the rest in B.
+struct FusedKeys {
+  uint32_t keysA, nA, keysB;
+  __device__ __forceinline__ uint32_t addr(uint32_t i) const { return i < nA ? keysA + 4u * i : keysB + 4u * (i - nA); }
+};
+
+// Shared-memory plan of the selection kernel (addresses are shared-window
+// addresses). The nch tables (64 KB each) start at the first 64 KB-aligned
+// address; segment A lies before them, segment B after. The selection state
+// and histograms open segment A; sort keys fill the rest of A, then B.
 struct FusedSmem {
-  uint32_t base, tbl, segA, segA_end, segB, segB_end;
-  uint32_t sel, hist1, hist2, hist3;
-  uint32_t keysA, nA;        // first nA keys in segment A
-  uint32_t keysB;            // the rest in segment B
-  __device__ void plan(uint32_t dyn_base, uint32_t dyn_size) {
+  uint32_t base, tbl0, tbl1, segA_end, segB, segB_end;
+  uint32_t sel, hist0, hist1, hist2;
+  uint32_t keysA, nA, keysB;
+  __device__ void plan(uint32_t dyn_base, uint32_t dyn_size, int nch) {
     base = dyn_base;
-    tbl = (dyn_base + 65535u) & ~65535u;
-    segA = dyn_base;
-    segA_end = tbl;
-    segB = tbl + TABLE_BYTES;
+    tbl0 = (dyn_base + 65535u) & ~65535u;
+    tbl1 = tbl0 + TABLE_BYTES;
+    segA_end = tbl0;
+    segB = tbl0 + (uint32_t)nch * TABLE_BYTES;
     segB_end = dyn_base + dyn_size;
-    uint32_t a = segA;
+    uint32_t a = dyn_base;
     sel = a;   a += (sizeof(SelShared) + 15u) & ~15u;
-    hist1 = a; a += 4u << HIST1_BITS;
-    hist2 = a; a += 4u << HIST2_BITS;
-    hist3 = a; a += 4u << HIST3_BITS;
+    hist0 = a; a += 4u * hist_words(0);
+    hist1 = a; a += 4u * hist_words(1);
+    hist2 = a; a += 4u * hist_words(2);
     keysA = a;
     nA = (segA_end > a) ? (segA_end - a) / 4u : 0u;
     keysB = segB;
   }
-  __device__ uint32_t key_capacity() const { return nA + (segB_end - segB) / 4u; }
-  __device__ __forceinline__ uint32_t key_addr(uint32_t i) const {
-    return i < nA ? keysA + 4u * i : keysB + 4u * (i - nA);
-  }
+  __device__ uint32_t key_capacity() const { return nA + (segB_end > segB ? (segB_end - segB) / 4u : 0u); }
+  __device__ __forceinline__ FusedKeys keys() const { return FusedKeys{keysA, nA, keysB}; }
 };
 
 template <typename T>
@@ -78,262 +97,282 @@ __device__ __forceinline__ T* sptr(unsigned char* dyn, uint32_t base, uint32_t a
   return reinterpret_cast<T*>(dyn + (addr - base));
 }
 
-// Zero rows >= 2^P and columns >= L of a table at shared address tbl.
-__device__ __forceinline__ void zero_table_padding(unsigned char* dyn, uint32_t base, uint32_t tbl, int L, int P) {
-  float* t = sptr<float>(dyn, base, tbl);
+// Zeroes, in the first copy of every chunk table (columns x < S_c), the cells
+// of rows >= 2^P and of tables >= L.
+template <int LP>
+__device__ __forceinline__ void zero_table_padding(float* t0, float* t1, int L, int P) {
   const int nb = 1 << P;
-  for (int e = threadIdx.x; e < 256 * TABLE_COLS; e += blockDim.x) {
-    const int b = e / TABLE_COLS, l = e % TABLE_COLS;
-    if (b >= nb || l >= L) t[e] = 0.f;
+#pragma unroll
+  for (int c = 0; c < table_chunks(LP); ++c) {
+    float* t = c ? t1 : t0;
+    const int S = id_chunk_size(L, c);
+    for (int e = threadIdx.x; e < 256 * S; e += blockDim.x) {
+      const int b = e / S, x = e % S;
+      if (b >= nb || 32 * c + x >= L) t[b * TABLE_COLS + x] = 0.f;
+    }
   }
 }
 
-// Scores this CTA's blocks [blk0, blk1) into sort keys (fs.key_addr) and the
-// level-1 histogram. Warp w takes blocks blk0 + w, blk0 + w + NW, ...
-template <int NCHUNK, bool NORM>
-__device__ __forceinline__ void score_slice(const uint8_t* __restrict__ ids_pair,
-                                            const __half* __restrict__ norms_pair, int L, int N, int blk0,
-                                            int blk1, const FusedSmem& fs, uint32_t* hist1) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  uint32_t col_addr[NCHUNK];
+// Fills every chunk table from the first copies built by the cluster: the
+// 4-column group starting at table 4g is owned by CTA (4g) / per; it is read
+// from the owner (distributed shared memory, 16-byte loads) and written to all
+// 64 / S_c copies of its columns in this CTA.
+template <int LP>
+__device__ __forceinline__ void pull_and_replicate_tables(cg::cluster_group& cluster, float* t0, float* t1, int L,
+                                                          int P, int per, int rank) {
+  const int nbk = 1 << P;
 #pragma unroll
-  for (int c = 0; c < NCHUNK; ++c) col_addr[c] = fs.tbl + 4u * (32 * c + lane);
-  const int nb = (blk1 - blk0 - warp + nw - 1) / nw;
-  IdBlock<NCHUNK> buf[SCORE_PF];
-#pragma unroll
-  for (int u = 0; u < SCORE_PF; ++u) {
-    if (u < nb) {
-      const int blk = blk0 + warp + u * nw;
-      load_id_block<NCHUNK, NORM>(buf[u], ids_pair + (size_t)blk * 32 * L, norms_pair + (size_t)blk * 32, L, lane);
+  for (int c = 0; c < table_chunks(LP); ++c) {
+    float* t = c ? t1 : t0;
+    const int S = id_chunk_size(L, c);
+    const int groups = S / 4;
+    for (int e = threadIdx.x; e < 256 * groups; e += blockDim.x) {
+      const int bb = e / groups, g = e % groups;
+      const int l = 32 * c + 4 * g;                        // first table of the group
+      const int owner = l < L ? l / per : rank;            // padding groups are zero everywhere
+      float* src = t + bb * TABLE_COLS + 4 * g;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (bb < nbk) v = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(src, (unsigned)owner));
+      for (int x = 4 * g; x < TABLE_COLS; x += S) *reinterpret_cast<uint4*>(t + bb * TABLE_COLS + x) = v;
     }
   }
+}
+
+// Scores keys of blocks blk0 + warp + i * NW (i < nb) into sort keys and the
+// level-0 histogram. buf holds the first SCORE_PF blocks, already requested.
+template <int LP, bool NORM>
+__device__ __forceinline__ void score_blocks(KeyIds<LP> (&buf)[SCORE_PF], const uint8_t* __restrict__ ids_pair,
+                                             const __half* __restrict__ norms_pair, int N, int blk0, int nb,
+                                             uint32_t col0, uint32_t col1, const FusedKeys keys, uint32_t* hist0) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int it = 0; it < nb; it += SCORE_PF) {
 #pragma unroll
     for (int u = 0; u < SCORE_PF; ++u) {
       const int i = it + u;
       if (i < nb) {
-        const IdBlock<NCHUNK> cur = buf[u];
+        const KeyIds<LP> cur = buf[u];
         if (i + SCORE_PF < nb) {
-          const int blk = blk0 + warp + (i + SCORE_PF) * nw;
-          load_id_block<NCHUNK, NORM>(buf[u], ids_pair + (size_t)blk * 32 * L, norms_pair + (size_t)blk * 32, L,
-                                      lane);
+          const int key = (blk0 + warp + (i + SCORE_PF) * nw) * 32 + lane;
+          load_key_ids<LP, NORM>(buf[u], ids_pair + (size_t)key * LP, norms_pair + key);
         }
-        const float s = score_id_block<NCHUNK, NORM>(cur, col_addr, lane);
-        const int blk = blk0 + warp + i * nw;
-        const int gkey = blk * 32 + lane;
+        const float s = score_key<LP, NORM>(cur, col0, col1);
+        const int gkey = (blk0 + warp + i * nw) * 32 + lane;
         if (gkey < N) {
           const uint32_t key = key_of(s);
           const uint32_t li = (uint32_t)(gkey - blk0 * 32);
-          asm volatile("st.shared.u32 [%0], %1;" :: "r"(fs.key_addr(li)), "r"(key) : "memory");
-          atomicAdd(&hist1[key >> 20], 1u);
+          asm volatile("st.shared.u32 [%0], %1;" ::"r"(keys.addr(li)), "r"(key) : "memory");
+          atomicAdd(&hist0[key >> 20], 1u);
         }
       }
     }
   }
 }
 
-// ---------------------------------------------------------------- fused decode
-// One cluster of C CTAs per (batch, KV-head) pair; grid = pairs * C.
-// HATA = false: SOCKET soft-LSH scores (ids/norms cache, tables l = rank mod C).
-// HATA = true: hard-hash scores from 128-bit codes (16 byte tables, no norm),
-// with R holding the 128 code hyperplanes and ids the codes.
-template <int D, int NCHUNK, typename KVT, bool HATA>
-__global__ void __launch_bounds__(FUSED_THREADS, 1) socket_decode_fused_kernel(const FusedParams p) {
+template <int LP, bool NORM>
+__device__ __forceinline__ void prefetch_blocks(KeyIds<LP> (&buf)[SCORE_PF], const uint8_t* __restrict__ ids_pair,
+                                                const __half* __restrict__ norms_pair, int blk0, int nb) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+#pragma unroll
+  for (int u = 0; u < SCORE_PF; ++u) {
+    if (u < nb) {
+      const int key = (blk0 + warp + u * nw) * 32 + lane;
+      load_key_ids<LP, NORM>(buf[u], ids_pair + (size_t)key * LP, norms_pair + key);
+    }
+  }
+}
+
+// Shared-memory plan of the attention stage: query stage, one mbarrier and
+// phase word per warp slot, warp slots, per-warp partials.
+struct AttendSmem {
+  uint32_t qs;             // query rows (bf16 path)
+  uint32_t mbar0;          // 8 bytes per slot
+  uint32_t phases;         // 4 bytes per slot
+  uint32_t slot0;          // warp w's slot: slot0 + w * slot_stride
+  uint32_t slot_stride;
+  int nslots;
+  uint32_t partials;
+};
+
+// Exact attention of cnt keys (keys(i), i < cnt) into merged per-CTA results
+// (cM, cL, cO) using warps 0..ncw-1; all threads call it. For bf16 the caller
+// has staged Q at as.qs, initialised the slot mbarriers and zeroed phases.
+template <int D, typename KVT, typename KeyFn>
+__device__ __forceinline__ void attend_and_merge(unsigned char* dyn, uint32_t base, const AttendSmem& as,
+                                                 const KVT* Qg, const KVT* Kp, const KVT* Vp, int G, float scale,
+                                                 KeyFn keys, int cnt, int nrows, float*& cM, float*& cL, float*& cO) {
+  const int ncw = as.nslots;
+  const PartialView pv = partial_view(sptr<float>(dyn, base, as.partials), ncw, G, D, cM, cL, cO);
+  if constexpr (sizeof(KVT) == 2) {
+    attend_tiles_bf16<D>(reinterpret_cast<const __nv_bfloat16*>(Kp), reinterpret_cast<const __nv_bfloat16*>(Vp), keys,
+                         cnt, nrows, G, scale, as.qs, as.slot0, as.slot_stride, as.mbar0,
+                         sptr<uint32_t>(dyn, base, as.phases), ncw, pv);
+  } else {
+    attend_keys_f32<D>(reinterpret_cast<const float*>(Qg), reinterpret_cast<const float*>(Kp),
+                       reinterpret_cast<const float*>(Vp), keys, cnt, nrows, G, scale, ncw, pv);
+  }
+  __syncthreads();
+  merge_partials(pv, ncw, cM, cL, cO);
+}
+
+// Sets up the attention stage: stages Q (bf16), initialises one mbarrier per
+// slot and zeroes the phase words. Ends with __syncthreads().
+template <int D, typename KVT>
+__device__ __forceinline__ void attend_setup(unsigned char* dyn, uint32_t base, const AttendSmem& as, const KVT* Qg,
+                                             int G) {
+  if constexpr (sizeof(KVT) == 2) {
+    stage_q<D>(reinterpret_cast<const __nv_bfloat16*>(Qg), G, sptr<unsigned char>(dyn, base, as.qs));
+    if (threadIdx.x < as.nslots) {
+      mbar_init(as.mbar0 + 8u * threadIdx.x, 1);
+      sptr<uint32_t>(dyn, base, as.phases)[threadIdx.x] = 0u;
+    }
+    if (threadIdx.x == 0) fence_mbar_init();
+  }
+  __syncthreads();
+}
+
+// ---------------------------------------------------------------- selection kernel
+// One cluster of C CTAs per (batch, KV-head) pair; grid = pairs * C. CTA r
+// scores the keys of blocks [r * blocks_per_cta, ...); the cluster then finds
+// the exact top-k and writes the pair's ascending index list to p.idx_out.
+// HATA = false: SOCKET soft-LSH scores from the ids/norms cache.
+// HATA = true: hard-hash scores from 128-bit codes (16 byte-tables, no norm);
+// R holds the 128 code hyperplanes and ids the codes.
+template <int D, int LP, typename QT, bool HATA>
+__global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const FusedParams p) {
   extern __shared__ __align__(1024) unsigned char dyn[];
+  cg::cluster_group cluster = cg::this_cluster();
+  constexpr int NCH = table_chunks(LP);
   const int C = p.C;
   const int rank = (int)cluster_ctarank();
   const int pair = blockIdx.x / C;
   const int G = p.Hq / p.Hkv;
   const int b = pair / p.Hkv, kvh = pair % p.Hkv;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
   uint32_t dyn_size;
   asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_size));
   FusedSmem fs;
-  fs.plan(smem_u32(dyn), dyn_size);
+  fs.plan(smem_u32(dyn), dyn_size, NCH);
+  // The host sizes slices from the same plan; a mismatch (a host bug) is
+  // flagged and every CTA of the grid leaves here (the test is uniform).
+  if (fs.segB > fs.segB_end || (uint32_t)p.blocks_per_cta * 32u > fs.key_capacity()) {
+    if (tid == 0) atomicOr(&g_error_word, ERR_LAYOUT);
+    return;
+  }
+  stamp(p.phase_ts, 0);
   SelShared* sh = sptr<SelShared>(dyn, fs.base, fs.sel);
-  uint32_t* hist[3] = {sptr<uint32_t>(dyn, fs.base, fs.hist1), sptr<uint32_t>(dyn, fs.base, fs.hist2),
-                       sptr<uint32_t>(dyn, fs.base, fs.hist3)};
+  uint32_t* hist[3] = {sptr<uint32_t>(dyn, fs.base, fs.hist0), sptr<uint32_t>(dyn, fs.base, fs.hist1),
+                       sptr<uint32_t>(dyn, fs.base, fs.hist2)};
+  float* tab0 = sptr<float>(dyn, fs.base, fs.tbl0);
+  float* tab1 = sptr<float>(dyn, fs.base, fs.tbl1);
 
   const int nblk_pair = (p.N + 31) / 32;
   const int blk0 = min(nblk_pair, rank * p.blocks_per_cta);
   const int blk1 = min(nblk_pair, blk0 + p.blocks_per_cta);
   const int n_local = max(0, min(p.N, blk1 * 32) - blk0 * 32);
-  // The host sizes slices from the same plan; a mismatch (a host bug) is flagged
-  // and the kernel then selects and gathers nothing. The test is the same in every
-  // CTA of the cluster.
-  const bool fits = fs.tbl + TABLE_BYTES <= fs.base + dyn_size &&
-                    (uint32_t)p.blocks_per_cta * 32u <= fs.key_capacity();
-  if (!fits) {              // uniform across the cluster: every CTA leaves here
-    if (tid == 0) atomicOr(&g_error_word, ERR_LAYOUT);
-    return;
-  }
-
-  // ---- setup: zero histograms and table padding; let peers know we started
-  for (int i = tid; i < (1 << HIST1_BITS); i += blockDim.x) hist[0][i] = 0u;
-  for (int i = tid; i < (1 << HIST2_BITS); i += blockDim.x) hist[1][i] = 0u;
-  for (int i = tid; i < (1 << HIST3_BITS); i += blockDim.x) hist[2][i] = 0u;
-  zero_table_padding(dyn, fs.base, fs.tbl, p.L, p.P);
-  cluster_sync();
-
-  // ---- SOCKET step 2: this CTA's share of the bucket tables, written to every CTA
-  const KVT* Qg = reinterpret_cast<const KVT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
-  {
-    const uint32_t tbl = fs.tbl;
-    auto store = [&](int bb, int l, float v) {
-      const uint32_t a = tbl + (uint32_t)bb * 256u + 4u * (uint32_t)l;
-      for (int r = 0; r < C; ++r) st_cluster_f32(mapa(a, r), v);
-    };
-    if constexpr (HATA) {
-      build_hamming_table(Qg, G, D, p.R, rank, C, sptr<uint32_t>(dyn, fs.base, fs.segB), store);
-    } else {
-      build_bucket_table(Qg, G, D, p.R, p.L, p.P, p.tau, rank, C, sptr<double>(dyn, fs.base, fs.segB), store);
-    }
-  }
-  cluster_sync();
-
-  // ---- SOCKET step 3: scores of this CTA's slice (kept on chip) + level-1 histogram
+  const int nb = max(0, (blk1 - blk0 - warp + FUSED_WARPS - 1) / FUSED_WARPS);
   const size_t pair_keys = (size_t)pair * p.Ncap;
+  const uint8_t* ids_pair = p.ids + pair_keys * LP;
+  const __half* norms_pair = p.norms + pair_keys;
+
+  // ---- setup: zero histograms and table padding; all CTAs started before any remote access
+  for (int i = tid; i < hist_words(0); i += blockDim.x) hist[0][i] = 0u;
+  for (int i = tid; i < hist_words(1); i += blockDim.x) hist[1][i] = 0u;
+  for (int i = tid; i < hist_words(2); i += blockDim.x) hist[2][i] = 0u;
+  zero_table_padding<LP>(tab0, tab1, p.L, p.P);
+  if (rank == 0 && tid == 0 && p.counters) p.counters[pair] = 0u;     // for the attention kernel's merge
+  cluster_sync();
+  stamp(p.phase_ts, 8);
+
+  // ---- SOCKET step 2: this CTA builds a range of tables (4-table aligned) into
+  // its own first copy; after the barrier every CTA pulls the other ranges.
+  const QT* Qg = reinterpret_cast<const QT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
+  const int per = ((p.L + C - 1) / C + 3) & ~3;
   {
-    const uint8_t* ids_pair = p.ids + pair_keys * p.L;
-    const __half* norms_pair = p.norms + pair_keys;
-    score_slice<NCHUNK, !HATA>(ids_pair, norms_pair, p.L, p.N, blk0, blk1, fs, hist[0]);
+    const int l0 = min(p.L, rank * per);
+    const int nl = min(p.L, l0 + per) - l0;
+    auto store = [=](int bb, int l, float v) {
+      const int c = l >= 32 ? 1 : 0;
+      (c ? tab1 : tab0)[bb * TABLE_COLS + (l - 32 * c)] = v;
+    };
+    void* scratch = sptr<void>(dyn, fs.base, fs.keysA);
+    if (nl > 0) {
+      if constexpr (HATA) build_hamming_table<D>(Qg, G, p.R, l0, nl, scratch, store);
+      else build_bucket_table<D>(Qg, G, p.R, p.P, p.tau, l0, nl, scratch, store, p.phase_ts);
+    }
   }
+  stamp(p.phase_ts, 9);
+  cluster_sync();
+  stamp(p.phase_ts, 10);
+  KeyIds<LP> buf[SCORE_PF];
+  prefetch_blocks<LP, !HATA>(buf, ids_pair, norms_pair, blk0, nb);
+  pull_and_replicate_tables<LP>(cluster, tab0, tab1, p.L, p.P, per, rank);
+  __syncthreads();
+  stamp(p.phase_ts, 1);
+
+  // ---- SOCKET step 3: scores of this CTA's slice (kept on chip) + level-0 histogram
+  const FusedKeys keys = fs.keys();
+  score_blocks<LP, !HATA>(buf, ids_pair, norms_pair, p.N, blk0, nb, fs.tbl0 + 4u * lane, fs.tbl1 + 4u * lane, keys,
+                          hist[0]);
+  stamp(p.phase_ts, 11);
   __syncthreads();
   cluster_sync();
+  stamp(p.phase_ts, 2);
 
-  // ---- SOCKET step 4a: exact top-k across the cluster
-  DigitLevel lv[3];
-  f32_levels(lv);
-  auto key_at = [&](int i) -> uint32_t { return lds_u32(fs.key_addr((uint32_t)i)); };
-  const int nl = n_local;
-  const SelPlan plan = cluster_select(key_at, nl, lv, 3, hist, (uint32_t)p.k, C, rank, sh);
-  // emit: the position's owner CTA gathers it; idx_out gets the ascending list
-  const int chunk = p.chunk;
-  const uint32_t list = fs.tbl;                       // table is dead: index list
-  int* idx_out = p.idx_out ? p.idx_out + (size_t)pair * p.k : nullptr;
-  ordered_compact(key_at, nl, plan, sh, [&](uint32_t pos, int i) {
-    if (pos >= (uint32_t)p.k) return;       // cannot happen for a consistent plan
-    const int g = blk0 * 32 + i;
-    const uint32_t owner = pos / (uint32_t)chunk;
-    const uint32_t slot = pos - owner * (uint32_t)chunk;
-    st_cluster_u32(mapa(list + 4u * slot, owner), (uint32_t)g);
-    if (idx_out) idx_out[pos] = g;
-  });
-  cluster_sync();
-
-  // ---- SOCKET step 4b: exact attention over this CTA's share of the selection
-  const int my_begin = rank * chunk;
-  const int cnt = max(0, min(p.k - my_begin, chunk));
-  const int* my_list = sptr<int>(dyn, fs.base, list);
-  // partial slots and the CTA result live in segment B (sort keys are dead)
-  PartialView pv;
-  pv.G = G;
-  pv.D = D;
-  float* pbase = sptr<float>(dyn, fs.base, fs.segB);
-  pv.pm = pbase;
-  pv.pl = pv.pm + FUSED_WARPS * G;
-  pv.po = pv.pl + FUSED_WARPS * G;
-  float* cM = pv.po + (size_t)FUSED_WARPS * G * D;
-  float* cL = cM + G;
-  float* cO = cL + G;
-  const KVT* Kp = reinterpret_cast<const KVT*>(p.K) + pair_keys * D;
-  const KVT* Vp = reinterpret_cast<const KVT*>(p.V) + pair_keys * D;
-  const float scale_log2 = p.scale * LOG2E;
-  const int nrows = p.N;
-  if constexpr (sizeof(KVT) == 2) {
-    const bool packed = G <= 4;
-    uint32_t qb[D / 32][4];
-    load_q_frag<D>(qb, reinterpret_cast<const __nv_bfloat16*>(Qg), G, lane);
-    MmaAttendState<D> st;
-    st.init();
-    const int ntiles = (cnt + 15) / 16;
-    KVTile<D> cur, nxt;
-    int t = warp;
-    if (t < ntiles) {
-      load_kv_tile<D>(cur, reinterpret_cast<const __nv_bfloat16*>(Kp), reinterpret_cast<const __nv_bfloat16*>(Vp),
-                      [&](int i) { return my_list[t * 16 + i]; }, min(16, cnt - t * 16), nrows, lane);
-    }
-    for (; t < ntiles; t += FUSED_WARPS) {
-      const int tn = t + FUSED_WARPS;
-      if (tn < ntiles) {
-        load_kv_tile<D>(nxt, reinterpret_cast<const __nv_bfloat16*>(Kp), reinterpret_cast<const __nv_bfloat16*>(Vp),
-                        [&](int i) { return my_list[tn * 16 + i]; }, min(16, cnt - tn * 16), nrows, lane);
-      }
-      mma_attend_tile<D>(st, cur, qb, scale_log2, packed, lane);
-      cur = nxt;
-    }
-    store_mma_partial<D>(st, pv, warp, packed, lane);
-  } else {
-    float q[8][D / 32];
-#pragma unroll
-    for (int h = 0; h < 8; ++h)
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i)
-        q[h][i] = h < G ? reinterpret_cast<const float*>(Qg)[h * D + lane + 32 * i] * scale_log2 : 0.f;
-    SimtAttendState<D> st;
-    st.init();
-    for (int j = warp; j < cnt; j += FUSED_WARPS) {
-      const int row = min(max(my_list[j], 0), nrows - 1);
-      simt_attend_key<D>(st, reinterpret_cast<const float*>(Kp) + (size_t)row * D,
-                         reinterpret_cast<const float*>(Vp) + (size_t)row * D, q, G, lane);
-    }
-    store_simt_partial<D>(st, pv, warp, lane);
-  }
-  __syncthreads();
-  merge_partials(pv, FUSED_WARPS, cM, cL, cO);
-  cluster_sync();
-
-  // ---- cross-CTA merge: CTA `rank` finalises heads h with h % C == rank
-  const uint32_t aM = smem_u32(cM), aL = smem_u32(cL), aO = smem_u32(cO);
-  for (int h = rank; h < G; h += C) {
-    float mm = -INFINITY;
-    for (int r = 0; r < C; ++r) mm = fmaxf(mm, ld_cluster_f32(mapa(aM + 4u * h, r)));
-    float lsum = 0.f;
-    for (int r = 0; r < C; ++r) {
-      const float mr = ld_cluster_f32(mapa(aM + 4u * h, r));
-      if (mr != -INFINITY) lsum += exp2f(mr - mm) * ld_cluster_f32(mapa(aL + 4u * h, r));
-    }
-    for (int e = tid; e < D; e += blockDim.x) {
-      float o = 0.f;
-      for (int r = 0; r < C; ++r) {
-        const float mr = ld_cluster_f32(mapa(aM + 4u * h, r));
-        if (mr != -INFINITY) o += exp2f(mr - mm) * ld_cluster_f32(mapa(aO + 4u * (h * D + e), r));
-      }
-      p.O[((size_t)b * p.Hq + kvh * G + h) * D + e] = o / lsum;
-    }
-  }
+  // ---- SOCKET step 4a: exact top-k across the cluster, ascending indices to idx_out
+  auto key_at = [=](int i) -> uint32_t { return lds_u32(keys.addr((uint32_t)i)); };
+  const SelThreshold th = cluster_threshold<FUSED_THREADS>(key_at, n_local, hist, (uint32_t)p.k, C, sh, p.phase_ts);
+  stamp(p.phase_ts, 3);
+  int* idx_out = p.idx_out + (size_t)pair * p.k;
+  const int kk = p.k, g0 = blk0 * 32;
+  ordered_compact(key_at, n_local, th, C, rank, sh, [=](uint32_t pos, int i) {
+    if (pos < (uint32_t)kk) idx_out[pos] = g0 + i;
+  }, p.phase_ts);
+  stamp(p.phase_ts, 12);
+  // the attention kernel may start once every CTA has written its indices
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   cluster_sync();   // peers may still read this CTA's shared memory until here
+  stamp(p.phase_ts, 7);
 }
 
 // ---------------------------------------------------------------- unfused chain
 struct TableParams {
   const void* Q;
   const __nv_bfloat16* R;
-  float* T;            // [pairs][256][64]
-  int Hq, Hkv, d, L, P;
+  float* T;            // [pairs][nch][256][64], the shared-memory table image
+  int Hq, Hkv, L, P;
   float tau;
 };
 
-template <typename QT>
+// grid = (pairs, ny): CTA y computes a contiguous range of tables and writes
+// every copy of its entries; CTA y = 0 also writes the zero padding.
+template <int D, int LP, typename QT>
 __global__ void __launch_bounds__(256) bucket_table_kernel(const TableParams p) {
   extern __shared__ __align__(1024) unsigned char dyn[];
+  constexpr int NCH = table_chunks(LP);
   const int pair = blockIdx.x;
   const int G = p.Hq / p.Hkv;
   const int b = pair / p.Hkv, kvh = pair % p.Hkv;
-  const QT* Qg = reinterpret_cast<const QT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * p.d;
-  float* T = p.T + (size_t)pair * 256 * TABLE_COLS;
-  // padding (rows >= 2^P, columns >= L) is zero; CTA y = 0 writes it
+  const QT* Qg = reinterpret_cast<const QT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
+  float* T = p.T + (size_t)pair * NCH * 256 * TABLE_COLS;
   if (blockIdx.y == 0) {
-    const int nb = 1 << p.P;
-    for (int e = threadIdx.x; e < 256 * TABLE_COLS; e += blockDim.x) {
-      const int bb = e / TABLE_COLS, l = e % TABLE_COLS;
-      if (bb >= nb || l >= p.L) T[e] = 0.f;
+    const int nbk = 1 << p.P;
+    for (int e = threadIdx.x; e < NCH * 256 * TABLE_COLS; e += blockDim.x) {
+      const int c = e / (256 * TABLE_COLS), bb = (e / TABLE_COLS) % 256, x = e % TABLE_COLS;
+      if (bb >= nbk || column_table(p.L, c, x) >= p.L) T[e] = 0.f;
     }
   }
-  build_bucket_table(Qg, G, p.d, p.R, p.L, p.P, p.tau, (int)blockIdx.y, (int)gridDim.y,
-                     reinterpret_cast<double*>(dyn),
-                     [&](int bb, int l, float v) { T[bb * TABLE_COLS + l] = v; });
+  const int per = (p.L + gridDim.y - 1) / gridDim.y;
+  const int l0 = min(p.L, (int)blockIdx.y * per);
+  const int nl = min(p.L, l0 + per) - l0;
+  if (nl <= 0) return;
+  build_bucket_table<D>(Qg, G, p.R, p.P, p.tau, l0, nl, reinterpret_cast<double*>(dyn),
+                        [&](int bb, int l, float v) {
+                          const int c = l >= 32 ? 1 : 0;
+                          const int S = id_chunk_size(p.L, c);
+                          float* row = T + ((size_t)c * 256 + bb) * TABLE_COLS;
+                          for (int x = l - 32 * c; x < TABLE_COLS; x += S) row[x] = v;
+                        });
 }
 
 struct ScoreParams {
@@ -341,42 +380,39 @@ struct ScoreParams {
   const uint8_t* ids;
   const __half* norms;
   float* scores;
-  int Ncap, N, L, blocks_per_cta;
+  int Ncap, N, blocks_per_cta;
 };
 
-// grid = (pairs, chunks); the 64 KB table of the pair is copied to a 64 KB-aligned
-// shared address, then each warp scores 32-key blocks.
-template <int NCHUNK>
-__global__ void __launch_bounds__(256, 1) socket_score_kernel(const ScoreParams p) {
+// grid = (pairs, chunks); the pair's table image is copied to 64 KB-aligned
+// shared memory, then each lane scores one key.
+template <int LP>
+__global__ void __launch_bounds__(FUSED_THREADS, 1) socket_score_kernel(const ScoreParams p) {
   extern __shared__ __align__(1024) unsigned char dyn[];
+  constexpr int NCH = table_chunks(LP);
   const int pair = blockIdx.x;
   const uint32_t base = smem_u32(dyn);
   const uint32_t tbl = (base + 65535u) & ~65535u;
   uint32_t dyn_size;
   asm volatile("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn_size));
-  if (tbl + TABLE_BYTES > base + dyn_size) {     // uniform over the grid
+  if (tbl + NCH * TABLE_BYTES > base + dyn_size) {     // uniform over the grid
     if (threadIdx.x == 0) atomicOr(&g_error_word, ERR_LAYOUT);
     return;
   }
   float* t = sptr<float>(dyn, base, tbl);
-  const float4* src = reinterpret_cast<const float4*>(p.T + (size_t)pair * 256 * TABLE_COLS);
-  for (int e = threadIdx.x; e < 256 * TABLE_COLS / 4; e += blockDim.x)
+  const float4* src = reinterpret_cast<const float4*>(p.T + (size_t)pair * NCH * 256 * TABLE_COLS);
+  for (int e = threadIdx.x; e < NCH * 256 * TABLE_COLS / 4; e += blockDim.x)
     reinterpret_cast<float4*>(t)[e] = __ldg(src + e);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  uint32_t col_addr[NCHUNK];
-#pragma unroll
-  for (int c = 0; c < NCHUNK; ++c) col_addr[c] = tbl + 4u * (32 * c + lane);
   const size_t pair_keys = (size_t)pair * p.Ncap;
   const int nblk = (p.N + 31) / 32;
   const int blk0 = blockIdx.y * p.blocks_per_cta;
   const int blk1 = min(nblk, blk0 + p.blocks_per_cta);
   for (int blk = blk0 + warp; blk < blk1; blk += nw) {
-    IdBlock<NCHUNK> ib;
-    load_id_block(ib, p.ids + (pair_keys + (size_t)blk * 32) * p.L, p.norms + pair_keys + (size_t)blk * 32, p.L,
-                  lane);
-    const float s = score_id_block(ib, col_addr, lane);
     const int key = blk * 32 + lane;
+    KeyIds<LP> k;
+    load_key_ids<LP, true>(k, p.ids + (pair_keys + key) * LP, p.norms + pair_keys + key);
+    const float s = score_key<LP, true>(k, tbl + 4u * lane, tbl + TABLE_BYTES + 4u * lane);
     if (key < p.N) p.scores[pair_keys + key] = s;
   }
 }
@@ -387,20 +423,20 @@ struct TopkParams {
   int Ncap, N, k, C, keys_per_cta;
 };
 
-// One cluster of C CTAs per pair; CTA r holds keys [r*keys_per_cta, ...).
+// One cluster of C CTAs per pair; CTA r holds keys [r * keys_per_cta, ...).
 __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_topk_kernel(const TopkParams p) {
   extern __shared__ __align__(1024) unsigned char dyn[];
   const int C = p.C;
   const int rank = (int)cluster_ctarank();
   const int pair = blockIdx.x / C;
   SelShared* sh = reinterpret_cast<SelShared*>(dyn);
-  uint32_t* h1 = reinterpret_cast<uint32_t*>(dyn + ((sizeof(SelShared) + 15) & ~15));
-  uint32_t* h2 = h1 + (1 << HIST1_BITS);
-  uint32_t* h3 = h2 + (1 << HIST2_BITS);
-  uint32_t* keys = h3 + (1 << HIST3_BITS);
-  for (int i = threadIdx.x; i < (1 << HIST1_BITS); i += blockDim.x) h1[i] = 0u;
-  for (int i = threadIdx.x; i < (1 << HIST2_BITS); i += blockDim.x) h2[i] = 0u;
-  for (int i = threadIdx.x; i < (1 << HIST3_BITS); i += blockDim.x) h3[i] = 0u;
+  uint32_t* h0 = reinterpret_cast<uint32_t*>(dyn + ((sizeof(SelShared) + 15) & ~15));
+  uint32_t* h1 = h0 + hist_words(0);
+  uint32_t* h2 = h1 + hist_words(1);
+  uint32_t* keys = h2 + hist_words(2);
+  for (int i = threadIdx.x; i < hist_words(0); i += blockDim.x) h0[i] = 0u;
+  for (int i = threadIdx.x; i < hist_words(1); i += blockDim.x) h1[i] = 0u;
+  for (int i = threadIdx.x; i < hist_words(2); i += blockDim.x) h2[i] = 0u;
   __syncthreads();
   const int k0 = rank * p.keys_per_cta;
   const int n_local = max(0, min(p.N - k0, p.keys_per_cta));
@@ -408,17 +444,15 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_topk_kernel(const Top
   for (int i = threadIdx.x; i < n_local; i += blockDim.x) {
     const uint32_t key = key_of(fmaxf(src[i], 0.0f));
     keys[i] = key;
-    atomicAdd(&h1[key >> 20], 1u);
+    atomicAdd(&h0[key >> 20], 1u);
   }
   __syncthreads();
   cluster_sync();
-  DigitLevel lv[3];
-  f32_levels(lv);
-  uint32_t* hist[3] = {h1, h2, h3};
+  uint32_t* hist[3] = {h0, h1, h2};
   auto key_at = [&](int i) -> uint32_t { return keys[i]; };
-  const SelPlan plan = cluster_select(key_at, n_local, lv, 3, hist, (uint32_t)p.k, C, rank, sh);
+  const SelThreshold th = cluster_threshold<FUSED_THREADS>(key_at, n_local, hist, (uint32_t)p.k, C, sh);
   int* out = p.idx + (size_t)pair * p.k;
-  ordered_compact(key_at, n_local, plan, sh, [&](uint32_t pos, int i) {
+  ordered_compact(key_at, n_local, th, C, rank, sh, [&](uint32_t pos, int i) {
     if (pos < (uint32_t)p.k) out[pos] = k0 + i;
   });
   cluster_sync();
@@ -428,111 +462,109 @@ struct AttendParams {
   const void* Q;
   const void* K;
   const void* V;
-  const int* idx;        // [pairs][k] (sparse) or nullptr (dense: keys 0..n-1)
-  float* part;           // [pairs][splits][G][D + 2]: (m, l, o[D]) per head
+  const int* idx;          // [pairs][n] key list (sparse) or nullptr (dense: keys 0..n-1)
+  float* part;             // [pairs][splits][G][D + 2]: (m, l, o[D]) per head
+  unsigned int* counters;  // [pairs], zero on entry; left zero on exit
+  float* O;                // [B][Hq][D]
   int Hq, Hkv, Ncap, n, keys_per_split, splits;
   float scale;
 };
 
-// grid = (pairs, splits). Each CTA attends over its range of the key list and
-// writes one partial (m, l, unnormalised o) per head.
+// Shared bytes of socket_attend_kernel: query stage, mbarriers and phases,
+// warp slots, partials, the CTA's index list, a flag word.
+template <int D>
+__host__ __device__ inline size_t attend_smem_bytes(int G, int keys_per_split) {
+  return q_stage_bytes<D>() + 8 * 32 + 4 * 32 + (size_t)ATTEND_WARPS * kv_slot_bytes<D>() +
+         partial_bytes(ATTEND_WARPS, G, D) + (((size_t)keys_per_split * 4 + 15) & ~(size_t)15) + 16;
+}
+
+// Exact attention over a key list, split over keys: grid = (pairs, splits).
+// Each CTA attends over its range and writes one partial (m, l, o) per head;
+// the last CTA of a pair to finish (counted with an atomic) merges the
+// pair's partials in split order and writes O, so the result does not depend
+// on the order the CTAs ran. Launched after the selection kernel with
+// programmatic dependent launch: everything before griddepcontrol.wait
+// overlaps that kernel's tail.
 template <int D, typename KVT>
-__global__ void __launch_bounds__(FUSED_THREADS) attend_split_kernel(const AttendParams p) {
+__global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const AttendParams p) {
   extern __shared__ __align__(1024) unsigned char dyn[];
   const int pair = blockIdx.x, split = blockIdx.y;
   const int G = p.Hq / p.Hkv;
   const int b = pair / p.Hkv, kvh = pair % p.Hkv;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int i0 = split * p.keys_per_split;
   const int cnt = max(0, min(p.n - i0, p.keys_per_split));
-  const int* list = p.idx ? p.idx + (size_t)pair * p.n + i0 : nullptr;
   const size_t pair_keys = (size_t)pair * p.Ncap;
   const KVT* Qg = reinterpret_cast<const KVT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
+  const uint32_t base = smem_u32(dyn);
+  AttendSmem as;
+  {
+    uint32_t a = base;
+    as.qs = a;       a += q_stage_bytes<D>();
+    as.mbar0 = a;    a += 8u * 32u;
+    as.phases = a;   a += 4u * 32u;
+    as.slot0 = a;
+    as.slot_stride = kv_slot_bytes<D>();
+    a += ATTEND_WARPS * kv_slot_bytes<D>();
+    as.nslots = ATTEND_WARPS;
+    as.partials = a;
+  }
+  const size_t smem_total = attend_smem_bytes<D>(G, p.idx ? p.keys_per_split : 0);
+  uint32_t* last_flag = reinterpret_cast<uint32_t*>(dyn + (smem_total - 16));
+  int* list_s = reinterpret_cast<int*>(dyn + (as.partials - base) + partial_bytes(ATTEND_WARPS, G, D));
+  attend_setup<D, KVT>(dyn, base, as, Qg, G);
+  asm volatile("griddepcontrol.wait;" ::: "memory");   // the key list is complete from here on
   const KVT* Kp = reinterpret_cast<const KVT*>(p.K) + pair_keys * D;
   const KVT* Vp = reinterpret_cast<const KVT*>(p.V) + pair_keys * D;
-  PartialView pv;
-  pv.G = G;
-  pv.D = D;
-  pv.pm = reinterpret_cast<float*>(dyn);
-  pv.pl = pv.pm + FUSED_WARPS * G;
-  pv.po = pv.pl + FUSED_WARPS * G;
-  float* cM = pv.po + (size_t)FUSED_WARPS * G * D;
-  float* cL = cM + G;
-  float* cO = cL + G;
-  const float scale_log2 = p.scale * LOG2E;
-  const int nrows = p.Ncap;
-  auto row_of = [&](int j) { return list ? list[j] : i0 + j; };
-  if constexpr (sizeof(KVT) == 2) {
-    const bool packed = G <= 4;
-    uint32_t qb[D / 32][4];
-    load_q_frag<D>(qb, reinterpret_cast<const __nv_bfloat16*>(Qg), G, lane);
-    MmaAttendState<D> st;
-    st.init();
-    const int ntiles = (cnt + 15) / 16;
-    KVTile<D> cur, nxt;
-    int t = warp;
-    if (t < ntiles) {
-      load_kv_tile<D>(cur, reinterpret_cast<const __nv_bfloat16*>(Kp), reinterpret_cast<const __nv_bfloat16*>(Vp),
-                      [&](int i) { return row_of(t * 16 + i); }, min(16, cnt - t * 16), nrows, lane);
-    }
-    for (; t < ntiles; t += FUSED_WARPS) {
-      const int tn = t + FUSED_WARPS;
-      if (tn < ntiles) {
-        load_kv_tile<D>(nxt, reinterpret_cast<const __nv_bfloat16*>(Kp), reinterpret_cast<const __nv_bfloat16*>(Vp),
-                        [&](int i) { return row_of(tn * 16 + i); }, min(16, cnt - tn * 16), nrows, lane);
-      }
-      mma_attend_tile<D>(st, cur, qb, scale_log2, packed, lane);
-      cur = nxt;
-    }
-    store_mma_partial<D>(st, pv, warp, packed, lane);
+  float *cM, *cL, *cO;
+  if (p.idx) {
+    const int* list = p.idx + (size_t)pair * p.n + i0;      // one coalesced load of this CTA's indices
+    for (int i = threadIdx.x; i < cnt; i += blockDim.x) list_s[i] = __ldcg(list + i);
+    __syncthreads();
+    attend_and_merge<D, KVT>(dyn, base, as, Qg, Kp, Vp, G, p.scale, [=](int i) { return list_s[i]; }, cnt, p.Ncap,
+                             cM, cL, cO);
   } else {
-    float q[8][D / 32];
-#pragma unroll
-    for (int h = 0; h < 8; ++h)
-#pragma unroll
-      for (int i = 0; i < D / 32; ++i)
-        q[h][i] = h < G ? reinterpret_cast<const float*>(Qg)[h * D + lane + 32 * i] * scale_log2 : 0.f;
-    SimtAttendState<D> st;
-    st.init();
-    for (int j = warp; j < cnt; j += FUSED_WARPS) {
-      const int row = min(max(row_of(j), 0), nrows - 1);
-      simt_attend_key<D>(st, reinterpret_cast<const float*>(Kp) + (size_t)row * D,
-                         reinterpret_cast<const float*>(Vp) + (size_t)row * D, q, G, lane);
-    }
-    store_simt_partial<D>(st, pv, warp, lane);
+    attend_and_merge<D, KVT>(dyn, base, as, Qg, Kp, Vp, G, p.scale, [=](int i) { return i0 + i; }, cnt, p.Ncap, cM,
+                             cL, cO);
   }
-  __syncthreads();
-  merge_partials(pv, FUSED_WARPS, cM, cL, cO);
-  float* out = p.part + ((size_t)pair * p.splits + split) * G * (D + 2);
+  float* mine = p.part + ((size_t)pair * p.splits + split) * G * (D + 2);
   for (int e = threadIdx.x; e < G * (D + 2); e += blockDim.x) {
     const int h = e / (D + 2), j = e % (D + 2);
-    out[e] = j == 0 ? cM[h] : j == 1 ? cL[h] : cO[h * D + j - 2];
+    mine[e] = j == 0 ? cM[h] : j == 1 ? cL[h] : cO[h * D + j - 2];
   }
-}
-
-// grid = pairs * G; block = D threads. Merges the splits of one head in order.
-__global__ void merge_splits_kernel(const float* __restrict__ part, float* __restrict__ O, int Hq, int Hkv, int D,
-                                    int splits) {
-  const int G = Hq / Hkv;
-  const int pair = blockIdx.x / G, h = blockIdx.x % G;
-  const int b = pair / Hkv, kvh = pair % Hkv;
-  const float* base = part + (size_t)pair * splits * G * (D + 2) + (size_t)h * (D + 2);
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) *last_flag = (atomicAdd(&p.counters[pair], 1u) == (unsigned)p.splits - 1u) ? 1u : 0u;
+  __syncthreads();
+  if (*last_flag == 0u) return;
+  // ---- last CTA of the pair: merge the splits in order, one head at a time:
+  // the head's partials are copied into shared memory (the warp slots are
+  // free; splits <= ATTEND_MAX_SPLITS keeps them in bounds) with independent
+  // loads, then combined there.
+  __threadfence();
+  const float* part = p.part + (size_t)pair * p.splits * G * (D + 2);
   const size_t stride = (size_t)G * (D + 2);
-  float mm = -INFINITY;
-  for (int s = 0; s < splits; ++s) mm = fmaxf(mm, base[s * stride]);
-  float lsum = 0.f;
-  for (int s = 0; s < splits; ++s) {
-    const float m = base[s * stride];
-    if (m != -INFINITY) lsum += exp2f(m - mm) * base[s * stride + 1];
-  }
-  for (int e = threadIdx.x; e < D; e += blockDim.x) {
-    float o = 0.f;
-    for (int s = 0; s < splits; ++s) {
-      const float m = base[s * stride];
-      if (m != -INFINITY) o += exp2f(m - mm) * base[s * stride + 2 + e];
+  float* ps = reinterpret_cast<float*>(dyn + (as.slot0 - base));
+  for (int h = 0; h < G; ++h) {
+    for (int e = threadIdx.x; e < p.splits * (D + 2); e += blockDim.x)
+      ps[e] = __ldcg(part + (size_t)(e / (D + 2)) * stride + (size_t)h * (D + 2) + e % (D + 2));
+    __syncthreads();
+    for (int dv = threadIdx.x; dv < D; dv += blockDim.x) {
+      float mm = -INFINITY;
+      for (int sp = 0; sp < p.splits; ++sp) mm = fmaxf(mm, ps[sp * (D + 2)]);
+      float lsum = 0.f, o = 0.f;
+      for (int sp = 0; sp < p.splits; ++sp) {
+        const float m = ps[sp * (D + 2)];
+        if (m != -INFINITY) {
+          const float w = exp2f(m - mm);
+          lsum += w * ps[sp * (D + 2) + 1];
+          o += w * ps[sp * (D + 2) + 2 + dv];
+        }
+      }
+      p.O[((size_t)b * p.Hq + kvh * G + h) * D + dv] = o / lsum;
     }
-    O[((size_t)b * Hq + kvh * G + h) * D + e] = o / lsum;
+    __syncthreads();
   }
+  if (threadIdx.x == 0) p.counters[pair] = 0u;
 }
 
 }  // namespace hst

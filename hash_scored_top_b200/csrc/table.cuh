@@ -19,10 +19,14 @@
 
 namespace hst {
 
-// Number of float64 scratch words build_bucket_table needs.
-__host__ __device__ inline int table_scratch_doubles(int G, int d, int n_my_tables, int P) {
+// Bytes of shared scratch build_bucket_table needs for nl tables: float64
+// words for the unit queries, bit factors and lo/hi products, then the
+// staged bf16 hyperplane rows.
+__host__ __device__ inline size_t table_scratch_bytes(int G, int d, int nl, int P) {
   const int plo = P / 2, phi = P - plo;
-  return G * d + G * n_my_tables * P * 2 + G * n_my_tables * ((1 << plo) + (1 << phi));
+  size_t dbl = (size_t)G * (d + 8) + (size_t)G * nl * P * 2 + (size_t)G * nl * ((1 << plo) + (1 << phi) + 2);
+  dbl = (dbl + 1) & ~(size_t)1;                         // keep the bf16 rows 16-byte aligned
+  return dbl * 8 + (size_t)nl * P * d * 2;
 }
 
 __device__ __forceinline__ double load_q(const float* q, int i) { return (double)q[i]; }
@@ -30,82 +34,144 @@ __device__ __forceinline__ double load_q(const __nv_bfloat16* q, int i) {
   return (double)__bfloat162float(q[i]);
 }
 
-// Computes T_l(b) for the tables l = l_first + t * l_step (t = 0, 1, ...) < L
-// and every bucket b < 2^P, calling store(b, l, value_f32) once per entry.
-// Qg points at the G query rows of the pair (row stride d). All threads of
-// the block must call this; it ends with __syncthreads().
-template <typename QT, typename Store>
-__device__ void build_bucket_table(const QT* __restrict__ Qg, int G, int d,
-                                   const __nv_bfloat16* __restrict__ R, int L, int P, float tau,
-                                   int l_first, int l_step, double* scratch, Store store) {
-  const int tid = threadIdx.x, nthr = blockDim.x;
-  const int nl = (L - l_first + l_step - 1) / l_step;   // tables handled here
-  const int plo = P / 2, phi = P - plo;
-  const int nlo = 1 << plo, nhi = 1 << phi;
-  double* qhat = scratch;                               // [G][d]
-  double* sig = qhat + G * d;                           // [G][nl][P][2]: P(bit=0), P(bit=1)
-  double* lo = sig + G * nl * P * 2;                    // [G][nl][nlo]
-  double* hi = lo + G * nl * nlo;                       // [G][nl][nhi]
+// Unit query rows are stored with each of the 8 segments of D / 8 values
+// followed by one padding word, so the 8 lanes that read the 8 segments hit
+// different banks.
+template <int D>
+__host__ __device__ constexpr int qpad_row() { return D + 8; }
+template <int D>
+__device__ __forceinline__ int qpad_index(int h, int c) {
+  return h * qpad_row<D>() + (c / (D / 8)) * (D / 8 + 1) + c % (D / 8);
+}
 
-  // 1. unit query rows (one warp per head)
-  const int warp = tid >> 5, lane = tid & 31, nwarps = nthr >> 5;
-  for (int h = warp; h < G; h += nwarps) {
-    double ss = 0.0;
-    for (int c = lane; c < d; c += 32) {
-      const double x = load_q(Qg + (size_t)h * d, c);
-      ss = fma(x, x, ss);
+// Projections z[item] = q_hat_h . r_m for items (h, m) with m = row0 + mi,
+// mi < nrows, computed as eight partial dot products of D / 8 terms (one per
+// lane of an aligned group of 8 lanes, two independent chains each, added in a
+// fixed butterfly order) in float64: short dependency chains, since float64
+// latency is long. Calls out(item, z) once per item from the group's first
+// lane. qhat: G padded rows (qpad_index); rs: [nrows][D] bf16 rows.
+template <int D, typename Out>
+__device__ __forceinline__ void project_rows(const double* qhat, int G, const __nv_bfloat16* rs, int nrows, Out out) {
+  const int nitems = G * nrows;
+  for (int base = 0; base < 8 * nitems; base += blockDim.x) {
+    const int e = base + threadIdx.x;
+    const bool valid = e < 8 * nitems;
+    const int item = valid ? e >> 3 : 0, part = e & 7;
+    const int h = item / nrows, mi = item % nrows;
+    const double* qh = qhat + h * qpad_row<D>() + part * (D / 8 + 1);
+    const uint4* rr = reinterpret_cast<const uint4*>(rs + (size_t)mi * D + part * (D / 8));
+    double z0 = 0.0, z1 = 0.0;
+#pragma unroll
+    for (int c8 = 0; c8 < D / 64; ++c8) {
+      const uint4 w = rr[c8];
+      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        z0 = fma(qh[c8 * 8 + 2 * k], (double)bf16lo_to_f32(ws[k]), z0);
+        z1 = fma(qh[c8 * 8 + 2 * k + 1], (double)bf16hi_to_f32(ws[k]), z1);
+      }
     }
+    double z = z0 + z1;
+    z += __shfl_xor_sync(FULL, z, 1);
+    z += __shfl_xor_sync(FULL, z, 2);
+    z += __shfl_xor_sync(FULL, z, 4);
+    if (valid && part == 0) out(item, z);
+  }
+}
+
+// Unit query rows (one warp per head) into qhat (padded rows, qpad_index),
+// float64. Each lane loads its D / 32 values once, then normalises them.
+template <int D, typename QT>
+__device__ __forceinline__ void unit_queries(const QT* __restrict__ Qg, int G, double* qhat) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  for (int h = warp; h < G; h += nwarps) {
+    double x[D / 32];
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) x[i] = load_q(Qg + (size_t)h * D, lane + 32 * i);
+    double ss = 0.0;
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) ss = fma(x[i], x[i], ss);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
-    const double nrm = sqrt(ss);
-    for (int c = lane; c < d; c += 32) qhat[h * d + c] = load_q(Qg + (size_t)h * d, c) / nrm;
+    const double inv = 1.0 / sqrt(ss);
+#pragma unroll
+    for (int i = 0; i < D / 32; ++i) qhat[qpad_index<D>(h, lane + 32 * i)] = x[i] * inv;
   }
+}
+
+// Copies hyperplane rows [row0, row0 + nrows) (bf16, D wide) to shared rs.
+template <int D>
+__device__ __forceinline__ void stage_rows(const __nv_bfloat16* __restrict__ R, int row0, int nrows,
+                                           __nv_bfloat16* rs) {
+  const uint4* src = reinterpret_cast<const uint4*>(R + (size_t)row0 * D);
+  uint4* dst = reinterpret_cast<uint4*>(rs);
+  for (int e = threadIdx.x; e < nrows * (D / 8); e += blockDim.x) dst[e] = __ldg(src + e);
+}
+
+// Computes T_l(b) for the tables l in [l0, l0 + nl) and every bucket b < 2^P,
+// calling store(b, l, value_f32) once per entry. Qg points at the G query
+// rows of the pair (row stride D); scratch holds table_scratch_bytes. All
+// threads of the block must call this; it ends with __syncthreads().
+template <int D, typename QT, typename Store>
+__device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_bfloat16* __restrict__ R, int P,
+                                   float tau, int l0, int nl, void* scratch, Store store,
+                                   unsigned long long* ts = nullptr) {
+  auto tstamp = [&](int ph) {
+    if (ts != nullptr && threadIdx.x == 0) {
+      unsigned long long t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      ts[blockIdx.x * 24 + ph] = t;
+    }
+  };
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const int plo = P / 2, phi = P - plo;
+  const int nlo = 1 << plo, nhi = 1 << phi;
+  // lo/hi rows are padded by one word (17 or 9 words) so that the lanes of a
+  // warp, which read different rows, hit different banks
+  const int slo = nlo + 1, shi = nhi + 1;
+  double* qhat = reinterpret_cast<double*>(scratch);   // G padded rows
+  double* sig = qhat + G * qpad_row<D>();               // [G][nl][P][2]: P(bit=0), P(bit=1)
+  double* lo = sig + G * nl * P * 2;                    // [G][nl][slo]
+  double* hi = lo + G * nl * slo;                       // [G][nl][shi]
+  const int ndbl = (G * qpad_row<D>() + G * nl * P * 2 + G * nl * (slo + shi) + 1) & ~1;   // 16-byte aligned rows
+  __nv_bfloat16* rs = reinterpret_cast<__nv_bfloat16*>(qhat + ndbl);                       // [nl * P][D]
+
+  // 1. unit query rows; this CTA's hyperplane rows
+  unit_queries<D>(Qg, G, qhat);
+  stage_rows<D>(R, l0 * P, nl * P, rs);
   __syncthreads();
+  tstamp(5);
 
   // 2. projections z and the per-bit factors sigmoid(+-2z/tau)
   const double two_over_tau = 2.0 / (double)tau;
-  for (int item = tid; item < G * nl * P; item += nthr) {
-    const int j = item % P;
-    const int li = (item / P) % nl;
-    const int h = item / (P * nl);
-    const int l = l_first + li * l_step;
-    const uint4* rrow = reinterpret_cast<const uint4*>(R + (size_t)(l * P + j) * d);
-    const double* qh = qhat + h * d;
-    double z = 0.0;
-    for (int c8 = 0; c8 < d / 8; ++c8) {
-      const uint4 w = __ldg(rrow + c8);
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        z = fma(qh[c8 * 8 + 2 * e], (double)bf16lo_to_f32(ws[e]), z);
-        z = fma(qh[c8 * 8 + 2 * e + 1], (double)bf16hi_to_f32(ws[e]), z);
-      }
-    }
+  project_rows<D>(qhat, G, rs, nl * P, [&](int item, double z) {
     const double x = two_over_tau * z;                  // logit gap between bit=1 and bit=0
     const double e = exp(-fabs(x));
     const double p_big = 1.0 / (1.0 + e);               // sigmoid(|x|)
     const double p_small = e / (1.0 + e);               // sigmoid(-|x|)
     sig[item * 2 + 1] = x >= 0.0 ? p_big : p_small;     // bit j = 1
     sig[item * 2 + 0] = x >= 0.0 ? p_small : p_big;     // bit j = 0
-  }
+  });
   __syncthreads();
+  tstamp(6);
 
   // 3. products over the low / high bits
   for (int item = tid; item < G * nl * (nlo + nhi); item += nthr) {
     const int m = item % (nlo + nhi);
     const int hl = item / (nlo + nhi);                  // h * nl + li
-    const double* s = sig + (size_t)hl * P * 2;
+    const double* sg = sig + (size_t)hl * P * 2;
     double prod = 1.0;
     if (m < nlo) {
-      for (int j = 0; j < plo; ++j) prod *= s[j * 2 + ((m >> j) & 1)];
-      lo[hl * nlo + m] = prod;
+      for (int j = 0; j < plo; ++j) prod *= sg[j * 2 + ((m >> j) & 1)];
+      lo[hl * slo + m] = prod;
     } else {
       const int mh = m - nlo;
-      for (int j = 0; j < phi; ++j) prod *= s[(plo + j) * 2 + ((mh >> j) & 1)];
-      hi[hl * nhi + mh] = prod;
+      for (int j = 0; j < phi; ++j) prod *= sg[(plo + j) * 2 + ((mh >> j) & 1)];
+      hi[hl * shi + mh] = prod;
     }
   }
   __syncthreads();
+  tstamp(13);
 
   // 4. table entries, summed over the group's heads
   const int nb = 1 << P;
@@ -115,9 +181,9 @@ __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, int d,
     double t = 0.0;
     for (int h = 0; h < G; ++h) {
       const int hl = h * nl + li;
-      t = fma(lo[hl * nlo + (b & (nlo - 1))], hi[hl * nhi + (b >> plo)], t);
+      t = fma(lo[hl * slo + (b & (nlo - 1))], hi[hl * shi + (b >> plo)], t);
     }
-    store(b, l_first + li * l_step, (float)t);
+    store(b, l0 + li, (float)t);
   }
   __syncthreads();
 }

@@ -35,13 +35,16 @@
  *   R      [L*P][d]            bf16; row l*P + j is hyperplane j of table l
  *   R128   [128][d]            bf16; hyperplanes of the 128-bit hard-hash codes
  *   norms  [B][Hkv][Ncap]      f16; cached |v| of each key
- *   ids    per pair, key-block interleaved: the bucket ID of key n in table l
- *          of pair p is byte  p*Ncap*L + (n/32)*32*L + l*32 + (n%32)  (uint8;
- *          P <= 8, so a table has at most 256 buckets).
- *   codes  per pair, key-block interleaved like ids with 16 "tables": byte m
- *          of the 128-bit code of key n of pair p is at
- *          p*Ncap*16 + (n/32)*512 + m*32 + (n%32); code bit c is bit c%8 of
- *          byte c/8.
+ *   ids    [B][Hkv][Ncap][LP] uint8, LP = 16 (L <= 16), 32 (L <= 32),
+ *          48 (L <= 48) or 64 (L <= 64) bytes per key, in chunks of S_0, S_1
+ *          tables: [16], [32], [32, 16] or [32, 32]. Inside chunk c (tables
+ *          32c, 32c+1, ...), byte 32c + j of key n holds the bucket ID of table
+ *          32c + (j + n) mod S_c, and 0 where that table is >= L ("rotated
+ *          key-major": 32 consecutive keys read 32 different tables at every
+ *          byte position). P <= 8, so an ID is one byte.
+ *   codes  [B][Hkv][Ncap][16] uint8 in the same layout with 16 "tables": byte
+ *          j of key n holds byte (j + n) mod 16 of its 128-bit code; code bit c
+ *          is bit c % 8 of code byte c / 8.
  *   scores [B][Hkv][Ncap]      f32 (only the first N per pair are written)
  *   idx    [B][Hkv][k]         int32, ascending key indices
  */
@@ -180,6 +183,14 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
  * up, SK_ERR_UNSUPPORTED if a kernel found its shared-memory plan did not fit
  * (it then wrote nothing); SK_ERR_CUDA on a pending CUDA error; else SK_OK. */
 int sk_check_status(void* stream);
+
+/* Profiling hook: while `device_buffer` is non-NULL, every fused decode
+ * launch (socket_decode, hata_decode) writes %globaltimer stamps per CTA to
+ * device_buffer[cta * 24 + phase] (phases: start, tables built, scores done,
+ * threshold found, indices scattered, attention done, CTA merge done, exit).
+ * The buffer must hold 24 entries per CTA of the launch (at most 16 * B * Hkv
+ * CTAs). Pass NULL to turn it off. Costs one store per phase per CTA. */
+int sk_profile_phases(unsigned long long* device_buffer);
 
 /* Thread-local description of the last non-OK return (never NULL). */
 const char* sk_last_error(void);

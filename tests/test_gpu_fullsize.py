@@ -47,7 +47,7 @@ def test_socket_fullsize_sampled(api, wname, nsample):
     pairs = _sample_pairs(w, nsample)
     ref_nat, ref_norms, proj = pa.oracle_socket_cache(inp, w, pairs)
     R = inp["R"].double().cpu().numpy()
-    nat = api.ids_to_natural(ids)
+    nat = api.ids_to_natural(ids, w.L)
     for b, h in pairs:
         K = inp["K"][b, h, : w.N].double().cpu().numpy()
         robust = pa.sign_band(K, R, proj[(b, h)]).reshape(w.N, w.L, w.P).all(axis=2)
@@ -88,7 +88,7 @@ def test_hata_fullsize_sampled(api):
     pairs = _sample_pairs(w, 3)
     ref, proj = pa.oracle_codes(inp, w, pairs)
     R = inp["R128"].double().cpu().numpy()
-    nat = api.ids_to_natural(codes)
+    nat = api.ids_to_natural(codes, 16)
     for b, h in pairs:
         K = inp["K"][b, h, : w.N].double().cpu().numpy()
         robust = pa.sign_band(K, R, proj[(b, h)]).reshape(w.N, 16, 8).all(axis=2)

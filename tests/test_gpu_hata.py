@@ -37,7 +37,7 @@ def test_codes_match_oracle(api, name):
     codes = api.empty_codes(w.B, w.Hkv, Ncap, DEV)
     api.hata_hash_keys(inp["K"], inp["R128"], codes)
     torch.cuda.synchronize()
-    got = api.ids_to_natural(codes).cpu().numpy()
+    got = api.ids_to_natural(codes, 16).cpu().numpy()
     ref, proj = pa.oracle_codes(inp, w)
     R = inp["R128"].double().cpu().numpy()
     for b in range(w.B):

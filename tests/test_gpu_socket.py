@@ -55,7 +55,7 @@ def test_hash_keys_match_oracle(api, name):
     norms = api.empty_norms(w.B, w.Hkv, Ncap, DEV)
     api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, norms)
     torch.cuda.synchronize()
-    gpu_nat = api.ids_to_natural(ids).cpu().numpy()
+    gpu_nat = api.ids_to_natural(ids, w.L).cpu().numpy()
     ref_nat, ref_norms, proj = pa.oracle_socket_cache(inp, w)
     R = inp["R"].double().cpu().numpy()
     total_robust = 0
@@ -83,7 +83,7 @@ def test_hash_keys_append_touches_only_the_range(api):
     api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, full_ids, full_norms, 0, w.N)
     torch.cuda.synchronize()
     assert torch.equal(ids, full_ids) and torch.equal(norms, full_norms)
-    nat_b, nat_a = api.ids_to_natural(before_ids), api.ids_to_natural(ids)
+    nat_b, nat_a = api.ids_to_natural(before_ids, w.L), api.ids_to_natural(ids, w.L)
     assert torch.equal(nat_b[:, :, : w.N - 1], nat_a[:, :, : w.N - 1])
     assert torch.equal(nat_a[:, :, w.N:], torch.zeros_like(nat_a[:, :, w.N:]))
 

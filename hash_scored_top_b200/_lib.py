@@ -28,6 +28,8 @@ SIGNATURES = {
     "socket_score": (_i, [_p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _z, _p]),
     "socket_topk": (_i, [_p, _i, _i, _i, _i, _i, _p, _p, _z, _p]),
     "socket_sparse_attend": (_i, [_p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p, _z, _p]),
+    "socket_sparse_attend_noalloc": (_i, [_p, _p, _p, _i, _p, _i, _i, _i, _i, _i, _i, _f, _p, _p]),
+    "sk_noalloc_scratch_bytes": (_z, []),
     "socket_decode": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _f, _p, _p, _p, _z,
                            _p]),
     "hata_hash_keys": (_i, [_p, _i, _p, _i, _i, _i, _i, _i, _i, _p, _p]),

@@ -175,6 +175,32 @@ def socket_sparse_attend(Q, K, V, idx, scale: float, O, ws=None):
     _check(rc, "socket_sparse_attend")
 
 
+def socket_sparse_attend_noalloc(Q, K, V, idx, scale: float, O):
+    """socket_sparse_attend for callers that cannot allocate device memory.
+
+    The library keeps a fixed static device scratch (``noalloc_scratch_bytes()``
+    bytes per GPU) for the attention partials, so this call allocates nothing;
+    shapes that do not fit raise RuntimeError. All calls on a GPU share that
+    scratch: calls that overlap on the GPU race. The first call on a device
+    looks up the scratch address; make it before any stream capture.
+    """
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = K.shape
+    k = idx.shape[-1]
+    _want(K, Q.dtype, K.shape, "K")
+    _want(V, Q.dtype, K.shape, "V")
+    _want(idx, torch.int32, (B, Hkv, k), "idx")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    rc = _lib.lib.socket_sparse_attend_noalloc(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(idx), B, Hq, Hkv,
+                                               Ncap, d, k, ctypes.c_float(scale), _ptr(O), _stream())
+    _check(rc, "socket_sparse_attend_noalloc")
+
+
+def noalloc_scratch_bytes() -> int:
+    """Bytes of the static scratch socket_sparse_attend_noalloc uses."""
+    return int(_lib.lib.sk_noalloc_scratch_bytes())
+
+
 def socket_decode(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k: int, scale: float, O, idx_out=None,
                   ws=None):
     """The fused decode step (SOCKET steps 2-4)."""

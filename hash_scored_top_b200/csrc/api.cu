@@ -537,6 +537,75 @@ int socket_sparse_attend(const void* Q, const void* K, const void* V, sk_dtype k
                        as_stream(stream));
 }
 
+}  // extern "C"
+
+namespace {
+
+// Fixed scratch of socket_sparse_attend_noalloc: the attention partials and
+// the per-pair merge counters. It lives in the library's own device image, so
+// every GPU that loads the library holds these bytes until the process exits,
+// and every call of the entry point on that GPU shares them.
+constexpr size_t kNoAllocScratchBytes = (size_t)4 << 20;
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on the current device. In host code the
+// array's name stands for a host-side shadow symbol, not device memory, so the
+// address must come from the runtime; it is looked up once per device (with
+// that device current) and cached.
+int noalloc_scratch_address(void** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static void* addr[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return fail(SK_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return fail(SK_ERR_UNSUPPORTED, "device ordinal %d >= %d", dev, kMaxDevices);
+  std::lock_guard<std::mutex> lock(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return fail(SK_ERR_CUDA, "static scratch address on device %d: %s", dev, cudaGetErrorString(e));
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return SK_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sk_noalloc_scratch_bytes(void) { return kNoAllocScratchBytes; }
+
+int socket_sparse_attend_noalloc(const void* Q, const void* K, const void* V, sk_dtype kv, const int* idx, int B,
+                                 int Hq, int Hkv, int Ncap, int d, int k, float scale, float* O, void* stream) {
+  SK_NONNULL(Q);
+  SK_NONNULL(K);
+  SK_NONNULL(V);
+  SK_NONNULL(idx);
+  SK_NONNULL(O);
+  SK_TRY(check_dtype(kv));
+  SK_TRY(check_heads(B, Hq, Hkv, d));
+  if (Ncap < 32 || Ncap % 32) return fail(SK_ERR_INVALID_ARG, "Ncap=%d must be a positive multiple of 32", Ncap);
+  if (k < 1) return fail(SK_ERR_INVALID_ARG, "k=%d must be >= 1", k);
+  const int pairs = B * Hkv, G = Hq / Hkv;
+  if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
+  // same split count as socket_sparse_attend, hence the same partial layout
+  const size_t need = attend_ws_bytes(pairs, attend_splits(k, pairs, false), G, d);
+  if (need > kNoAllocScratchBytes)
+    return fail(SK_ERR_WORKSPACE,
+                "socket_sparse_attend_noalloc: B=%d Hkv=%d G=%d d=%d needs %zu bytes of scratch, above the fixed "
+                "%zu-byte static scratch; call socket_sparse_attend with a caller workspace instead",
+                B, Hkv, G, d, need, kNoAllocScratchBytes);
+  void* scratch = nullptr;
+  SK_TRY(noalloc_scratch_address(&scratch));
+  // zero_counters: the merge counters keep the previous call's contents and
+  // must start at zero; the partials are written before they are read
+  return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, scratch, kNoAllocScratchBytes, false,
+                       true, as_stream(stream));
+}
+
 namespace {
 
 // The decode step: selection kernel (tables, scores, exact top-k -> index list)

@@ -130,6 +130,37 @@ int socket_sparse_attend(const void* Q, const void* K, const void* V, sk_dtype k
                          void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * socket_sparse_attend without a workspace argument, for callers that cannot
+ * allocate device memory: a host whose memory manager has already reserved
+ * the free HBM (a serving engine that pre-sizes its KV cache, for instance),
+ * or code on a latency-critical path where cudaMalloc / cudaFree, which can
+ * synchronise the device, are not allowed. The paper has no counterpart: it
+ * is a packaging of the same attention, not a step of the method.
+ *
+ * Same arguments, layout and result as socket_sparse_attend minus ws and
+ * ws_bytes. Instead of a caller buffer it uses one fixed static device array
+ * of sk_noalloc_scratch_bytes() bytes (4 MiB) inside the library, which every
+ * GPU that loads the library holds until the process exits. It allocates
+ * nothing. Shapes whose partials exceed that size (roughly B*Hkv above ~1000
+ * pairs at G = 8, d = 128) return SK_ERR_WORKSPACE with a message naming the
+ * needed and the available bytes, launching nothing.
+ *
+ * The first call on a device looks up the array's device address (with that
+ * device current) and caches it; make that first call before any stream
+ * capture. Each call clears the merge counters it needs on `stream` before
+ * the kernel runs. Every call on a device shares the one array: calls whose
+ * kernels overlap on the GPU (different streams, or threads that do not
+ * order their streams) race on it and give wrong results. Order them on one
+ * stream, or use socket_sparse_attend with a buffer per stream.
+ */
+int socket_sparse_attend_noalloc(const void* Q, const void* K, const void* V, sk_dtype kv, const int* idx,
+                                 int B, int Hq, int Hkv, int Ncap, int d, int k, float scale, float* O,
+                                 void* stream);
+
+/* Size in bytes of the static scratch socket_sparse_attend_noalloc uses. */
+size_t sk_noalloc_scratch_bytes(void);
+
+/*
  * The fused decode step, SOCKET steps 2-4 in one launch: bucket table,
  * scores, exact top-k and attention over the selection, one thread-block
  * cluster per pair with the scores kept on chip. The result equals

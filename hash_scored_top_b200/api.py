@@ -18,7 +18,8 @@ import torch
 from . import _lib
 
 SK_F32, SK_BF16 = 0, 1
-OP_HASH_KEYS, OP_SCORE, OP_TOPK, OP_SPARSE_ATTEND, OP_DECODE, OP_HATA_HASH, OP_HATA_DECODE, OP_DENSE_DECODE = range(8)
+(OP_HASH_KEYS, OP_SCORE, OP_TOPK, OP_SPARSE_ATTEND, OP_DECODE, OP_HATA_HASH, OP_HATA_DECODE, OP_DENSE_DECODE,
+ OP_SELECT) = range(9)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -219,6 +220,20 @@ def socket_decode(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k:
                                 Ncap, N, d, L, P, ctypes.c_float(tau), k, ctypes.c_float(scale), _ptr(O),
                                 _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
     _check(rc, "socket_decode")
+
+
+def socket_select(Q, R, ids, norms, N: int, L: int, P: int, tau: float, k: int, idx, ws=None):
+    """SOCKET steps 2-4 without the attention: idx [B, Hkv, k] int32 ascending."""
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = ids.shape
+    _want(R, torch.bfloat16, (L * P, d), "R")
+    _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
+    _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
+    _want(idx, torch.int32, (B, Hkv, k), "idx")
+    ws = _workspace(workspace_bytes(OP_SELECT, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    rc = _lib.lib.socket_select(_ptr(Q), _dtype_code(Q), _ptr(R), _ptr(ids), _ptr(norms), B, Hq, Hkv, Ncap, N, d, L,
+                                P, ctypes.c_float(tau), k, _ptr(idx), _ptr(ws), _ws_bytes(ws), _stream())
+    _check(rc, "socket_select")
 
 
 def hata_hash_keys(K, R128, codes, n_begin: int = 0, n_count: int | None = None):

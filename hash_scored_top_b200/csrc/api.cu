@@ -422,6 +422,13 @@ size_t chain_ws_bytes(int B, int Hq, int Hkv, int Ncap, int d, int L, int k) {
   return align256(table_image_bytes(pairs, L)) + align256((size_t)pairs * Ncap * 4) + decode_ws_bytes(B, Hq, Hkv, k, d);
 }
 
+// Workspace of the selection alone: none when it runs as one cluster kernel,
+// else the unfused chain's tables and scores.
+size_t select_ws_bytes(const FusedPlan& fp, int pairs, int Ncap, int L) {
+  if (fp.C > 0) return 0;
+  return align256(table_image_bytes(pairs, L)) + align256((size_t)pairs * Ncap * 4);
+}
+
 constexpr int kAppendMaxKeys = 16;
 
 int hash_launch(const void* K, const void* V, sk_dtype kv, const void* R, int B, int Hkv, int Ncap, int n_begin,
@@ -613,13 +620,15 @@ namespace {
 // chain when the selection cannot keep a pair's keys on chip.
 int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, const void* ids,
                 const void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k,
-                float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, bool hata, cudaStream_t s) {
+                float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, bool hata, bool attend,
+                cudaStream_t s) {
   const int pairs = B * Hkv, G = Hq / Hkv;
   if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
   const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, hata, max_cluster_size());
   if (fp.C == 0 && hata) return fail(SK_ERR_UNSUPPORTED, "hard-hash decode: N=%d too large for one cluster", N);
-  const size_t need = fp.C > 0 ? decode_ws_bytes(B, Hq, Hkv, k, d) : chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
-  if (ws == nullptr || ws_bytes < need)
+  const size_t need = !attend ? select_ws_bytes(fp, pairs, Ncap, L)
+                      : fp.C > 0 ? decode_ws_bytes(B, Hq, Hkv, k, d) : chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
+  if (need > 0 && (ws == nullptr || ws_bytes < need))
     return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
   char* w = reinterpret_cast<char*>(ws);
   if (fp.C == 0) {        // unfused chain through the workspace
@@ -632,14 +641,17 @@ int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const 
     SK_TRY(launch_tables(Q, kv, R, B, Hq, Hkv, d, L, P, tau, T, s));
     SK_TRY(launch_score(T, ids, norms, pairs, Ncap, N, L, scores, s));
     SK_TRY(launch_topk(scores, pairs, Ncap, N, k, idx, s));
+    if (!attend) return SK_OK;
     return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, w,
                          attend_ws_bytes(pairs, attend_splits(k, pairs, false), G, d), false, true, s);
   }
   int* idx = idx_out ? idx_out : reinterpret_cast<int*>(w);
-  w += align256((size_t)pairs * k * 4);
   const int splits = attend_splits(k, pairs, false);
-  unsigned int* counters = reinterpret_cast<unsigned int*>(
-      w + align256((size_t)pairs * splits * G * (d + 2) * sizeof(float)));
+  unsigned int* counters = nullptr;
+  if (attend) {
+    w += align256((size_t)pairs * k * 4);
+    counters = reinterpret_cast<unsigned int*>(w + align256((size_t)pairs * splits * G * (d + 2) * sizeof(float)));
+  }
   FusedParams p;
   p.Q = Q;
   p.K = K;
@@ -664,6 +676,7 @@ int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const 
   p.tau = tau;
   p.scale = scale;
   SK_TRY(launch_select(p, pairs, d, kv, hata, s));
+  if (!attend) return SK_OK;
   return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, w, attend_ws_bytes(pairs, splits, G, d),
                        true, false, s);
 }
@@ -686,7 +699,24 @@ int socket_decode(const void* Q, const void* K, const void* V, sk_dtype kv, cons
   SK_TRY(check_tables(L, P, tau));
   if (k < 1 || k > N) return fail(SK_ERR_INVALID_ARG, "k=%d must be in [1, N=%d]", k, N);
   return decode_impl(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, scale, O, idx_out, ws, ws_bytes,
-                     false, as_stream(stream));
+                     false, true, as_stream(stream));
+}
+
+int socket_select(const void* Q, sk_dtype q, const void* R, const void* ids, const void* norms, int B, int Hq, int Hkv,
+                  int Ncap, int N, int d, int L, int P, float tau, int k, int* idx, void* ws, size_t ws_bytes,
+                  void* stream) {
+  SK_NONNULL(Q);
+  SK_NONNULL(R);
+  SK_NONNULL(ids);
+  SK_NONNULL(norms);
+  SK_NONNULL(idx);
+  SK_TRY(check_dtype(q));
+  SK_TRY(check_heads(B, Hq, Hkv, d));
+  SK_TRY(check_cache(Ncap, N));
+  SK_TRY(check_tables(L, P, tau));
+  if (k < 1 || k > N) return fail(SK_ERR_INVALID_ARG, "k=%d must be in [1, N=%d]", k, N);
+  return decode_impl(Q, nullptr, nullptr, q, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, 0.f, nullptr, idx,
+                     ws, ws_bytes, false, false, as_stream(stream));
 }
 
 int hata_hash_keys(const void* K, sk_dtype kv, const void* R128, int B, int Hkv, int Ncap, int n_begin, int n_count,
@@ -721,7 +751,7 @@ int hata_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const 
   if (Hq / Hkv > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", Hq / Hkv);
   // 128 code bits = 16 byte-tables of 8 hyperplanes; no norms
   return decode_impl(Q, K, V, kv, R128, codes, codes, B, Hq, Hkv, Ncap, N, d, 16, 8, 1.f, k, scale, O, idx_out, ws,
-                     ws_bytes, true, as_stream(stream));
+                     ws_bytes, true, true, as_stream(stream));
 }
 
 int dense_decode(const void* Q, const void* K, const void* V, sk_dtype kv, int B, int Hq, int Hkv, int Ncap, int N,
@@ -755,6 +785,10 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
     case SK_OP_DENSE_DECODE:
       if (N < 1) return bad;
       return attend_ws_bytes(pairs, attend_splits(N, pairs, true), G, d);
+    case SK_OP_SELECT: {
+      if (k < 1 || N < 1 || G > 8 || L < 1 || L > kMaxL || P < 1 || P > 8) return bad;
+      return select_ws_bytes(plan_select(pairs, N, k, G, d, L, P, false, 8), pairs, Ncap, L);
+    }
     case SK_OP_DECODE:
     case SK_OP_HATA_DECODE: {
       if (k < 1 || N < 1 || G > 8) return bad;

@@ -77,7 +77,8 @@ typedef enum {
   SK_OP_DECODE = 4,
   SK_OP_HATA_HASH = 5,
   SK_OP_HATA_DECODE = 6,
-  SK_OP_DENSE_DECODE = 7
+  SK_OP_DENSE_DECODE = 7,
+  SK_OP_SELECT = 8
 } sk_op;
 
 /*
@@ -161,19 +162,36 @@ int socket_sparse_attend_noalloc(const void* Q, const void* K, const void* V, sk
 size_t sk_noalloc_scratch_bytes(void);
 
 /*
- * The fused decode step, SOCKET steps 2-4 in one launch: bucket table,
- * scores, exact top-k and attention over the selection, one thread-block
- * cluster per pair with the scores kept on chip. The result equals
- * socket_score -> socket_topk -> socket_sparse_attend. idx_out (nullable)
- * receives the selected indices [B][Hkv][k] ascending. Shapes the fused
- * kernel cannot hold on chip run that unfused chain instead (same results).
- * Requires 1 <= P <= 8, 1 <= L <= 64, 1 <= k <= N, tau > 0.
- * ws: sk_workspace_bytes(SK_OP_DECODE, ...) bytes.
+ * The decode step, SOCKET steps 2-4: bucket tables, scores, exact top-k and
+ * attention over the selection. Two kernels on `stream`: a selection kernel
+ * (one thread-block cluster per pair; the pair's scores stay in the
+ * cluster's shared memory, never in HBM) writes the index list, and an
+ * attention kernel, launched as its programmatic dependent, gathers the
+ * selected K/V rows and merges its key splits in a fixed order. The result
+ * equals socket_score -> socket_topk -> socket_sparse_attend. idx_out
+ * (nullable) receives the selected indices [B][Hkv][k] ascending. Shapes
+ * whose keys do not fit one cluster's shared memory run that unfused chain
+ * instead (same results). Requires 1 <= P <= 8, 1 <= L <= 64, 1 <= k <= N,
+ * tau > 0, G <= 8. ws: sk_workspace_bytes(SK_OP_DECODE, ...) bytes.
  */
 int socket_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R,
                   const void* ids, const void* norms, int B, int Hq, int Hkv, int Ncap, int N,
                   int d, int L, int P, float tau, int k, float scale, float* O, int* idx_out,
                   void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Selection only, SOCKET steps 2-4 without the attention: the index list of
+ * socket_decode (bucket tables, scores, exact top-k with ties to the lower
+ * index), written ascending to idx [B][Hkv][k], for callers that run their
+ * own attention over the selected keys. Q: [B][Hq][d] in dtype q. One
+ * cluster kernel; shapes it cannot hold on chip run socket_score ->
+ * socket_topk through ws. ws: sk_workspace_bytes(SK_OP_SELECT, ...) bytes
+ * (0 when the cluster kernel runs; ws may then be NULL).
+ * Requires 1 <= P <= 8, 1 <= L <= 64, 1 <= k <= N, tau > 0, G <= 8.
+ */
+int socket_select(const void* Q, sk_dtype q, const void* R, const void* ids, const void* norms,
+                  int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k,
+                  int* idx, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Hard-hash codes (HATA digest, section 3, with seeded random hyperplanes
@@ -215,12 +233,13 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
  * (it then wrote nothing); SK_ERR_CUDA on a pending CUDA error; else SK_OK. */
 int sk_check_status(void* stream);
 
-/* Profiling hook: while `device_buffer` is non-NULL, every fused decode
- * launch (socket_decode, hata_decode) writes %globaltimer stamps per CTA to
- * device_buffer[cta * 24 + phase] (phases: start, tables built, scores done,
- * threshold found, indices scattered, attention done, CTA merge done, exit).
- * The buffer must hold 24 entries per CTA of the launch (at most 16 * B * Hkv
- * CTAs). Pass NULL to turn it off. Costs one store per phase per CTA. */
+/* Profiling hook: while `device_buffer` is non-NULL, every selection kernel
+ * launch (socket_decode, socket_select, hata_decode) writes %globaltimer
+ * stamps per CTA to device_buffer[cta * 24 + phase] (phases such as start,
+ * tables built, scores done, histogram levels, threshold found, indices
+ * written, exit; slots 22-23 hold clock64 at start and exit). The buffer must
+ * hold 24 entries per CTA of the launch (at most 16 * B * Hkv CTAs). Pass
+ * NULL to turn it off. Costs one store per phase per CTA. */
 int sk_profile_phases(unsigned long long* device_buffer);
 
 /* Thread-local description of the last non-OK return (never NULL). */

@@ -215,6 +215,29 @@ def test_fused_decode_matches_oracle(api, name):
     assert torch.equal(idx, idx2)
 
 
+@pytest.mark.parametrize("name", ["tiny_f32", "llama8b_needles", "qwen_l48_g8", "g2_small_n"])
+def test_select_only_matches_decode_and_oracle(api, name):
+    """socket_select returns the decode step's index list: a valid top-k of the
+    oracle's scores, identical to what socket_decode selects."""
+    w = _w(name)
+    inp = wl.make_inputs(w, DEV)
+    ids, nrm, ids_nat, norms, _ = _cache(api, w, inp)
+    sel = torch.full((w.B, w.Hkv, w.k), -1, dtype=torch.int32, device=DEV)
+    api.socket_select(inp["Q"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, w.k, sel)
+    O = torch.empty(w.B, w.Hq, w.d, device=DEV)
+    idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=DEV)
+    api.socket_decode(inp["Q"], inp["K"], inp["V"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, w.k, w.scale, O, idx)
+    api.check_status()
+    assert torch.equal(sel, idx)
+    R = inp["R"].double().cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            Qg = inp["Q"][b, h * w.G:(h + 1) * w.G].double().cpu().numpy()
+            s_ref = so.soft_collision_scores(so.group_bucket_table(Qg, R, w.L, w.P, w.tau), ids_nat[b, h, : w.N],
+                                             norms[b, h, : w.N])
+            assert pa.check_selection(s_ref, sel[b, h].cpu().numpy(), w.k) == [], (b, h)
+
+
 def test_fused_decode_is_deterministic(api):
     w = _w("llama8b_needles")
     inp = wl.make_inputs(w, DEV)

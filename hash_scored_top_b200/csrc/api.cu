@@ -2,6 +2,7 @@
 // launches. Every entry point validates on the host before launching
 // anything, allocates nothing, and runs asynchronously on the caller's stream.
 #include <cstdarg>
+#include <cstdint>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -110,6 +111,13 @@ int check_dtype(sk_dtype t) {
     if ((ptr) == nullptr) return fail(SK_ERR_INVALID_ARG, "%s is NULL", #ptr);   \
   } while (0)
 
+// Alignment the kernels' vector loads and bulk copies rely on.
+#define SK_ALIGNED(ptr, bytes)                                                                   \
+  do {                                                                                           \
+    if (reinterpret_cast<uintptr_t>(ptr) % (bytes))                                              \
+      return fail(SK_ERR_INVALID_ARG, "%s must be %d-byte aligned", #ptr, (int)(bytes));         \
+  } while (0)
+
 // ---------------------------------------------------------------- plans
 // Splits over keys of the attention kernel: one wave of ~2 CTAs per SM
 // (sparse) or several waves (dense), at least 16 keys each.
@@ -144,7 +152,7 @@ constexpr uint32_t kFixedBytes = ((sizeof(SelShared) + 15u) & ~15u) + 4u * (hist
                                                                              hist_words(2));
 constexpr uint32_t kSegAFree = kTableAddr - SMEM_BASE_EXPECTED - kFixedBytes;
 uint32_t seg_b_bytes(int nch) { return SMEM_BASE_EXPECTED + SMEM_DYN_MAX - kTableAddr - nch * TABLE_BYTES; }
-uint32_t fused_key_capacity(int nch) { return kSegAFree / 4u + seg_b_bytes(nch) / 4u; }
+uint32_t fused_key_capacity(int nch) { return ((kSegAFree / 4u) & ~127u) + seg_b_bytes(nch) / 4u; }
 
 FusedPlan plan_select(int pairs, int N, int k, int G, int d, int L, int P, bool hata, int max_c) {
   FusedPlan fp;
@@ -157,7 +165,7 @@ FusedPlan plan_select(int pairs, int N, int k, int G, int d, int L, int P, bool 
     const int per = ((L + c - 1) / c + 3) & ~3;
     const int nl = per < L ? per : L;
     const size_t scratch = hata ? hamming_scratch_bytes(G, d, nl) : table_scratch_bytes(G, d, nl, P);
-    if ((uint32_t)bpc * 32u <= fused_key_capacity(nch) && scratch <= kSegAFree) {
+    if ((((uint32_t)bpc * 32u + 127u) & ~127u) <= fused_key_capacity(nch) && scratch <= kSegAFree) {
       fp.C = c;
       fp.blocks_per_cta = bpc;
       fp.chunk = (k + c - 1) / c;
@@ -352,32 +360,94 @@ int launch_topk(const float* scores, int pairs, int Ncap, int N, int k, int* idx
   return check_launch("socket_topk_kernel");
 }
 
+// Clusters of S CTAs (1, S, 1) that fit on the GPU at once with this launch
+// shape, from the occupancy API (cached per kernel, S and shared size).
+template <typename Kern>
+int attend_active_clusters(Kern kern, int pairs, int S, size_t smem) {
+  struct Rec {
+    const void* fn;
+    int S;
+    size_t smem;
+    int n;
+  };
+  static std::mutex mu;
+  static std::vector<Rec> cache;
+  const void* fn = reinterpret_cast<const void*>(kern);
+  std::lock_guard<std::mutex> lock(mu);
+  for (const Rec& r : cache)
+    if (r.fn == fn && r.S == S && r.smem == smem) return r.n;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pairs, S, 1);
+  cfg.blockDim = dim3(ATTEND_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = (unsigned)S;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+  cudaGetLastError();
+  cache.push_back(Rec{fn, S, smem, n});
+  return n;
+}
+
 template <int D, typename KVT>
-int launch_attend_t(const AttendParams& ap, int pairs, int G, bool pdl, cudaStream_t s) {
+int launch_attend_t(AttendParams ap, int pairs, int G, bool pdl, bool cluster, cudaStream_t s) {
+  auto kern = cluster ? socket_attend_kernel<D, KVT, true> : socket_attend_kernel<D, KVT, false>;
+  if (cluster) {
+    // the largest cluster (at most the planned split count) whose clusters,
+    // one per pair, all fit on the GPU at once
+    const int s0 = ap.splits;
+    int S = s0;
+    for (;;) {
+      const size_t sm = attend_smem_bytes<D>(G, (ap.n + S - 1) / S);
+      if (set_kernel_smem(kern, sm, S > 8) != cudaSuccess) return check_launch("cudaFuncSetAttribute(attend smem)");
+      if (S == 1 || attend_active_clusters(kern, pairs, S, sm) >= pairs) break;
+      S = S > 8 ? 8 : S / 2;
+    }
+    ap.splits = S;
+    ap.keys_per_split = (ap.n + S - 1) / S;
+  }
   const size_t smem = attend_smem_bytes<D>(G, ap.idx ? ap.keys_per_split : 0);
-  auto kern = socket_attend_kernel<D, KVT>;
-  if (set_kernel_smem(kern, smem) != cudaSuccess) return check_launch("cudaFuncSetAttribute(attend smem)");
+  if (set_kernel_smem(kern, smem, cluster && ap.splits > 8) != cudaSuccess)
+    return check_launch("cudaFuncSetAttribute(attend smem)");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(pairs, ap.splits, 1);
   cfg.blockDim = dim3(ATTEND_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cudaLaunchAttribute attr[2];
+  int na = 0;
+  if (pdl) {
+    attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[na].val.programmaticStreamSerializationAllowed = 1;
+    ++na;
+  }
+  if (cluster) {                       // the splits of a pair form one cluster
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = 1;
+    attr[na].val.clusterDim.y = (unsigned)ap.splits;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+  }
   cfg.attrs = attr;
-  cfg.numAttrs = pdl ? 1 : 0;
+  cfg.numAttrs = na;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ap);
   if (e != cudaSuccess) return fail(SK_ERR_CUDA, "attention launch: %s", cudaGetErrorString(e));
   return check_launch("socket_attend_kernel");
 }
 
-// Attention over idx (sparse, n = k) or all keys (dense, idx = NULL, n = N)
-// through workspace ws (partials + counters). zero_counters: clear the
-// counters first (standalone calls); otherwise the selection kernel did.
+// Attention over idx (sparse, n = k) or all keys (dense, idx = NULL, n = N).
+// Sparse attention with allow_cluster merges its splits inside a cluster
+// (at most max_cluster_size() splits); otherwise the splits merge through
+// workspace ws (partials + counters). zero_counters: clear the counters first
+// (standalone calls); otherwise the selection kernel did.
 int launch_attend(const void* Q, const void* K, const void* V, sk_dtype kv, const int* idx, int B, int Hq, int Hkv,
                   int Ncap, int n, int d, float scale, float* O, void* ws, size_t ws_bytes, bool pdl,
-                  bool zero_counters, cudaStream_t s) {
+                  bool zero_counters, cudaStream_t s, bool allow_cluster = true) {
   const int pairs = B * Hkv, G = Hq / Hkv;
   if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
   AttendParams ap;
@@ -391,22 +461,25 @@ int launch_attend(const void* Q, const void* K, const void* V, sk_dtype kv, cons
   ap.Ncap = Ncap;
   ap.n = n;
   ap.splits = attend_splits(n, pairs, idx == nullptr);
+  const bool cluster = allow_cluster && idx != nullptr;
+  if (cluster) ap.splits = std::min(ap.splits, max_cluster_size());
   ap.keys_per_split = (n + ap.splits - 1) / ap.splits;
   ap.scale = scale;
+  ap.phase_ts = g_phase_ts ? g_phase_ts + (size_t)16 * pairs * PHASES : nullptr;   // after the selection's CTAs
   const size_t need = attend_ws_bytes(pairs, ap.splits, G, d);
   if (ws == nullptr || ws_bytes < need)
     return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
   ap.part = reinterpret_cast<float*>(ws);
   ap.counters = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(ws) +
                                                 align256((size_t)pairs * ap.splits * G * (d + 2) * sizeof(float)));
-  if (zero_counters) {
+  if (zero_counters && !cluster) {
     const cudaError_t e = cudaMemsetAsync(ap.counters, 0, (size_t)pairs * 4, s);
     if (e != cudaSuccess) return fail(SK_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
   }
-  if (d == 128) return kv == SK_BF16 ? launch_attend_t<128, __nv_bfloat16>(ap, pairs, G, pdl, s)
-                                     : launch_attend_t<128, float>(ap, pairs, G, pdl, s);
-  return kv == SK_BF16 ? launch_attend_t<64, __nv_bfloat16>(ap, pairs, G, pdl, s)
-                       : launch_attend_t<64, float>(ap, pairs, G, pdl, s);
+  if (d == 128) return kv == SK_BF16 ? launch_attend_t<128, __nv_bfloat16>(ap, pairs, G, pdl, cluster, s)
+                                     : launch_attend_t<128, float>(ap, pairs, G, pdl, cluster, s);
+  return kv == SK_BF16 ? launch_attend_t<64, __nv_bfloat16>(ap, pairs, G, pdl, cluster, s)
+                       : launch_attend_t<64, float>(ap, pairs, G, pdl, cluster, s);
 }
 
 // Workspace of a decode step: the index list (when idx_out is NULL) then the
@@ -484,6 +557,11 @@ int socket_hash_keys(const void* K, const void* V, sk_dtype kv, const void* R, i
   SK_NONNULL(R);
   SK_NONNULL(ids);
   SK_NONNULL(norms);
+  SK_ALIGNED(K, 16);
+  SK_ALIGNED(V, 16);
+  SK_ALIGNED(R, 16);
+  SK_ALIGNED(ids, 32);
+  SK_ALIGNED(norms, 2);
   SK_TRY(check_dtype(kv));
   SK_TRY(check_heads(B, Hkv, Hkv, d));
   if (Ncap < 32 || Ncap % 32) return fail(SK_ERR_INVALID_ARG, "Ncap=%d must be a positive multiple of 32", Ncap);
@@ -503,6 +581,9 @@ int socket_score(const void* Q, sk_dtype q, const void* R, const void* ids, cons
   SK_NONNULL(ids);
   SK_NONNULL(norms);
   SK_NONNULL(scores);
+  SK_ALIGNED(R, 16);
+  SK_ALIGNED(ids, 32);
+  SK_ALIGNED(norms, 2);
   SK_TRY(check_dtype(q));
   SK_TRY(check_heads(B, Hq, Hkv, d));
   SK_TRY(check_cache(Ncap, N));
@@ -536,6 +617,9 @@ int socket_sparse_attend(const void* Q, const void* K, const void* V, sk_dtype k
   SK_NONNULL(V);
   SK_NONNULL(idx);
   SK_NONNULL(O);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(K, 16);
+  SK_ALIGNED(V, 16);
   SK_TRY(check_dtype(kv));
   SK_TRY(check_heads(B, Hq, Hkv, d));
   if (Ncap < 32 || Ncap % 32) return fail(SK_ERR_INVALID_ARG, "Ncap=%d must be a positive multiple of 32", Ncap);
@@ -592,6 +676,9 @@ int socket_sparse_attend_noalloc(const void* Q, const void* K, const void* V, sk
   SK_NONNULL(V);
   SK_NONNULL(idx);
   SK_NONNULL(O);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(K, 16);
+  SK_ALIGNED(V, 16);
   SK_TRY(check_dtype(kv));
   SK_TRY(check_heads(B, Hq, Hkv, d));
   if (Ncap < 32 || Ncap % 32) return fail(SK_ERR_INVALID_ARG, "Ncap=%d must be a positive multiple of 32", Ncap);
@@ -610,7 +697,7 @@ int socket_sparse_attend_noalloc(const void* Q, const void* K, const void* V, sk
   // zero_counters: the merge counters keep the previous call's contents and
   // must start at zero; the partials are written before they are read
   return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, scratch, kNoAllocScratchBytes, false,
-                       true, as_stream(stream));
+                       true, as_stream(stream), false);
 }
 
 namespace {
@@ -693,6 +780,12 @@ int socket_decode(const void* Q, const void* K, const void* V, sk_dtype kv, cons
   SK_NONNULL(ids);
   SK_NONNULL(norms);
   SK_NONNULL(O);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(K, 16);
+  SK_ALIGNED(V, 16);
+  SK_ALIGNED(R, 16);
+  SK_ALIGNED(ids, 32);
+  SK_ALIGNED(norms, 2);
   SK_TRY(check_dtype(kv));
   SK_TRY(check_heads(B, Hq, Hkv, d));
   SK_TRY(check_cache(Ncap, N));
@@ -710,6 +803,9 @@ int socket_select(const void* Q, sk_dtype q, const void* R, const void* ids, con
   SK_NONNULL(ids);
   SK_NONNULL(norms);
   SK_NONNULL(idx);
+  SK_ALIGNED(R, 16);
+  SK_ALIGNED(ids, 32);
+  SK_ALIGNED(norms, 2);
   SK_TRY(check_dtype(q));
   SK_TRY(check_heads(B, Hq, Hkv, d));
   SK_TRY(check_cache(Ncap, N));
@@ -724,6 +820,9 @@ int hata_hash_keys(const void* K, sk_dtype kv, const void* R128, int B, int Hkv,
   SK_NONNULL(K);
   SK_NONNULL(R128);
   SK_NONNULL(codes);
+  SK_ALIGNED(K, 16);
+  SK_ALIGNED(R128, 16);
+  SK_ALIGNED(codes, 16);
   SK_TRY(check_dtype(kv));
   SK_TRY(check_heads(B, Hkv, Hkv, d));
   if (Ncap < 32 || Ncap % 32) return fail(SK_ERR_INVALID_ARG, "Ncap=%d must be a positive multiple of 32", Ncap);
@@ -744,6 +843,11 @@ int hata_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const 
   SK_NONNULL(R128);
   SK_NONNULL(codes);
   SK_NONNULL(O);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(K, 16);
+  SK_ALIGNED(V, 16);
+  SK_ALIGNED(R128, 16);
+  SK_ALIGNED(codes, 16);
   SK_TRY(check_dtype(kv));
   SK_TRY(check_heads(B, Hq, Hkv, d));
   SK_TRY(check_cache(Ncap, N));
@@ -760,6 +864,9 @@ int dense_decode(const void* Q, const void* K, const void* V, sk_dtype kv, int B
   SK_NONNULL(K);
   SK_NONNULL(V);
   SK_NONNULL(O);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(K, 16);
+  SK_ALIGNED(V, 16);
   SK_TRY(check_dtype(kv));
   SK_TRY(check_heads(B, Hq, Hkv, d));
   SK_TRY(check_cache(Ncap, N));

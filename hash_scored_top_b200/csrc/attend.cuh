@@ -285,10 +285,13 @@ __device__ __forceinline__ void store_empty_partial(const PartialView& pv, int w
   }
 }
 
-// bf16 attention of `cnt` listed keys by warps 0..ncw-1 (warp w owns slot
-// `slot0 + w * slot_stride` and mbarrier `mbar0 + 8 w`, phase bits in
-// phases[w]); results go to partial slots 0..ncw-1. Other warps do nothing.
-template <int D, typename KeyFn>
+// bf16 attention of `cnt` listed keys by warps 0..ncw-1. Warp w takes the
+// 16-key tiles w, w + ncw, ... and cycles through its NBUF slots (slot
+// w * NBUF + s at slot0 + (w * NBUF + s) * slot_stride, mbarrier
+// mbar0 + 8 (w * NBUF + s), phase bit in phases[w * NBUF + s]): the copies of
+// the next NBUF - 1 tiles are in flight while a tile is computed. Results go
+// to partial slots 0..ncw-1. Other warps do nothing.
+template <int D, int NBUF, typename KeyFn>
 __device__ void attend_tiles_bf16(const __nv_bfloat16* __restrict__ Kp, const __nv_bfloat16* __restrict__ Vp,
                                   KeyFn keys, int cnt, int nrows, int G, float scale, uint32_t qs, uint32_t slot0,
                                   uint32_t slot_stride, uint32_t mbar0, uint32_t* phases, int ncw,
@@ -299,23 +302,47 @@ __device__ void attend_tiles_bf16(const __nv_bfloat16* __restrict__ Kp, const __
   const float scale_log2 = scale * LOG2E;
   MmaAttendState<D> st;
   st.init();
-  const uint32_t slot = slot0 + (uint32_t)warp * slot_stride;
-  const uint32_t mbar = mbar0 + 8u * warp;
-  uint32_t phase = phases[warp];
   const int ntiles = (cnt + 15) / 16;
-  bool ok = true;
-  for (int t = warp; t < ntiles && ok; t += ncw) {
+  const int nt = ntiles > warp ? (ntiles - warp + ncw - 1) / ncw : 0;   // this warp's tiles
+  uint32_t ph = 0;                          // bit s: phase of slot s
+#pragma unroll
+  for (int s = 0; s < NBUF; ++s) ph |= (phases[warp * NBUF + s] & 1u) << s;
+  auto slot_of = [&](int s) { return slot0 + (uint32_t)(warp * NBUF + s) * slot_stride; };
+  auto mbar_of = [&](int s) { return mbar0 + 8u * (uint32_t)(warp * NBUF + s); };
+  auto issue = [&](int j) {
+    const int t = warp + j * ncw;
     const int nvalid = min(16, cnt - 16 * t);
-    issue_tile_copies<D>(slot, mbar, Kp, Vp, [&](int i) { return keys(16 * t + i); }, nvalid, nrows, lane);
-    ok = mbar_wait_bounded(mbar, phase);
-    phase ^= 1u;
-    if (ok) mma_attend_slot<D>(st, slot, qs, nvalid, scale_log2, packed, lane);
+    issue_tile_copies<D>(slot_of(j % NBUF), mbar_of(j % NBUF), Kp, Vp, [&](int i) { return keys(16 * t + i); },
+                         nvalid, nrows, lane);
+  };
+  for (int j = 0; j < NBUF && j < nt; ++j) issue(j);
+  bool ok = true;
+  int j = 0;
+  for (; j < nt && ok; ++j) {
+    const int s = j % NBUF;
+    ok = mbar_wait_bounded(mbar_of(s), (ph >> s) & 1u);
+    ph ^= 1u << s;
+    if (ok) {
+      const int t = warp + j * ncw;
+      mma_attend_slot<D>(st, slot_of(s), qs, min(16, cnt - 16 * t), scale_log2, packed, lane);
+    }
     __syncwarp();
+    if (ok && j + NBUF < nt) issue(j + NBUF);
   }
-  if (!ok) {           // a copy never completed: wait once more (bounded) so none is left in flight
-    mbar_wait_bounded(mbar, phase ^ 1u);
+  if (!ok) {
+    // a copy never completed: wait once more (bounded) for it and for the
+    // tiles issued after it, so that none is left in flight
+    const int jf = j - 1;
+    mbar_wait_bounded(mbar_of(jf % NBUF), ((ph >> (jf % NBUF)) & 1u) ^ 1u);
+    for (int jj = jf + 1; jj < jf + NBUF && jj < nt; ++jj) {
+      mbar_wait_bounded(mbar_of(jj % NBUF), (ph >> (jj % NBUF)) & 1u);
+      ph ^= 1u << (jj % NBUF);
+    }
   }
-  if (lane == 0) phases[warp] = phase;
+  if (lane == 0) {
+#pragma unroll
+    for (int s = 0; s < NBUF; ++s) phases[warp * NBUF + s] = (ph >> s) & 1u;
+  }
   store_mma_partial<D>(st, pv, warp, packed, lane);
 }
 

@@ -52,6 +52,13 @@ __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   return r;
 }
 
+// 32 bytes in one request (sm_100 256-bit load); p must be 32-byte aligned.
+__device__ __forceinline__ void ldg_stream32(const void* p, uint4& lo, uint4& hi) {
+  asm volatile("ld.global.nc.L1::no_allocate.v8.u32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+               : "=r"(lo.x), "=r"(lo.y), "=r"(lo.z), "=r"(lo.w), "=r"(hi.x), "=r"(hi.y), "=r"(hi.z), "=r"(hi.w)
+               : "l"(p));
+}
+
 __device__ __forceinline__ uint16_t ldg_u16(const void* p) {
   unsigned short r;
   asm volatile("ld.global.nc.u16 %0, [%1];" : "=h"(r) : "l"(p));

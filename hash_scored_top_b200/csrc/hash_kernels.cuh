@@ -178,9 +178,9 @@ __host__ __device__ inline size_t hamming_scratch_bytes(int G, int d, int nm) {
   return (size_t)G * (d + 8) * 8 + (size_t)G * 16 * 4 + (size_t)nm * 8 * d * 2;
 }
 
-template <int D, typename QT, typename Store>
+template <int D, typename QT, typename Store, typename Hook = NoHook>
 __device__ void build_hamming_table(const QT* __restrict__ Qg, int G, const __nv_bfloat16* __restrict__ R128,
-                                    int m0, int nm, void* scratch, Store store) {
+                                    int m0, int nm, void* scratch, Store store, Hook before_store = Hook()) {
   const int tid = threadIdx.x;
   double* qd = reinterpret_cast<double*>(scratch);                 // G padded rows (not normalised: the sign is enough)
   uint32_t* qbyte = reinterpret_cast<uint32_t*>(qd + G * qpad_row<D>());  // [G][16]
@@ -194,6 +194,7 @@ __device__ void build_hamming_table(const QT* __restrict__ Qg, int G, const __nv
     if (z > 0.0) atomicOr(&qbyte[h * 16 + m0 + mi / 8], 1u << (mi % 8));
   });
   __syncthreads();
+  before_store();
   for (int item = tid; item < 256 * nm; item += blockDim.x) {
     const int x = item % 256;
     const int m = m0 + item / 256;

@@ -34,11 +34,20 @@ struct KeyIds {
   uint16_t norm;
 };
 
+// One key's IDs (and norm). Key rows of 32 and 64 bytes are read with 32-byte
+// loads, so each request of a warp covers whole 32-byte sectors; 16- and
+// 48-byte rows with 16-byte loads. ids_key is aligned to its row size's
+// largest power-of-two divisor (up to 32 bytes).
 template <int LP, bool NORM>
 __device__ __forceinline__ void load_key_ids(KeyIds<LP>& k, const uint8_t* __restrict__ ids_key,
                                              const __half* __restrict__ norm_key) {
+  if constexpr (LP % 32 == 0) {
 #pragma unroll
-  for (int i = 0; i < LP / 16; ++i) k.w[i] = ldg_stream(ids_key + 16 * i);
+    for (int i = 0; i < LP / 32; ++i) ldg_stream32(ids_key + 32 * i, k.w[2 * i], k.w[2 * i + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < LP / 16; ++i) k.w[i] = ldg_stream(ids_key + 16 * i);
+  }
   if (NORM) k.norm = ldg_u16(norm_key);
 }
 

@@ -43,6 +43,12 @@ struct SelShared {
   uint32_t cnt_w[32][2];         // compaction: per-warp (greater, equal) counts
   uint32_t off_w[32][2];         // compaction: per-warp (selected, equal) offsets
   uint32_t counts[SEL_MAX_C][2]; // (greater, equal) published by every CTA of the cluster
+  uint32_t coarse[SEL_MAX_C][64]; // binned path: coarse histogram sums of every CTA of the cluster
+  uint32_t over[SEL_MAX_C];      // binned path: keys above the bins' range, per CTA
+  uint32_t selc[SEL_MAX_C];      // binned path: selected boundary candidates of every CTA
+  uint32_t over_local;           // binned path: this CTA's keys above the range
+  uint32_t ncand;                // binned path: boundary candidates of this CTA
+  uint32_t pad2[2];
 };
 
 // Block-wide exclusive scan of one value per thread (thread order).
@@ -145,9 +151,7 @@ __device__ __forceinline__ void histogram_pass(KeyAt key_at, int n, int shift, i
 
 __device__ __forceinline__ void sel_stamp(unsigned long long* ts, int phase) {
   if (ts != nullptr && threadIdx.x == 0) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    ts[blockIdx.x * 24 + phase] = t;
+    ts[blockIdx.x * 24 + phase] = (unsigned long long)clock64();
   }
 }
 
@@ -284,6 +288,290 @@ __device__ void ordered_compact(KeyAt key_at, int n, const SelThreshold& th, int
     eq_run += __popc(meq);
   }
   __syncthreads();
+}
+
+
+// ---------------------------------------------------------------- binned path
+// The usual selection: while the scores are computed, every CTA counts its
+// keys into a histogram of fixed bins (f32 keys: one bin per 2^16 bit
+// patterns, i.e. 1/128 of an octave, over scores in [2^-16, 2^16); integer
+// keys: one bin per value). At the barrier after scoring every CTA has pushed
+// 64 coarse sums of its histogram and its count of keys above the range into
+// every CTA of the cluster. One warp then finds the coarse bin, and within it
+// (reading 64 fine bins of each CTA) the bin b* that holds the k-th largest
+// key. Keys above b* are all taken; the keys of b* (few) are gathered from
+// every CTA and ordered exactly (key descending, index ascending); the emit
+// pass writes the selection in index order. If the k-th key is outside the
+// range or b* holds more than BIN_CAND_CAP keys, the exact radix select above
+// runs instead (the decision is the same in every CTA).
+constexpr int BIN_COUNT = 4096;
+constexpr int BIN_COARSE = 64;                 // coarse bins, of 64 fine bins each
+constexpr int BIN_CAND_CAP = 256;
+constexpr uint32_t BIN_F32_BASE = 111u << 7;   // (key >> 16) of the f32 2^-16
+
+// Bin of a sort key: < 0 below the range, >= BIN_COUNT above it.
+template <bool INT_KEYS>
+__device__ __forceinline__ int key_bin(uint32_t key) {
+  if (INT_KEYS) return (int)min(key, (uint32_t)BIN_COUNT);
+  return (int)(key >> 16) - (int)BIN_F32_BASE;
+}
+
+// Smallest and largest key of bin b.
+template <bool INT_KEYS>
+__device__ __forceinline__ uint32_t bin_lo(int b) {
+  return INT_KEYS ? (uint32_t)b : ((uint32_t)b + BIN_F32_BASE) << 16;
+}
+template <bool INT_KEYS>
+__device__ __forceinline__ uint32_t bin_hi(int b) {
+  return INT_KEYS ? (uint32_t)b : (((uint32_t)b + BIN_F32_BASE + 1u) << 16) - 1u;
+}
+
+// Counts one key into this CTA's histogram (BIN_COUNT words) or its
+// above-range counter.
+template <bool INT_KEYS>
+__device__ __forceinline__ void bin_count(uint32_t key, uint32_t* hist, SelShared* sh) {
+  const int b = key_bin<INT_KEYS>(key);
+  if (b >= BIN_COUNT) atomicAdd(&sh->over_local, 1u);
+  else if (b >= 0) atomicAdd(&hist[b], 1u);
+}
+
+// Words of scratch binned_select needs: own and gathered candidates, flags.
+__host__ __device__ constexpr int bin_scratch_words() { return 2 * BIN_CAND_CAP * 2 + BIN_CAND_CAP; }
+
+// Stores this CTA's coarse sums and above-range count into every CTA of the
+// cluster. Call with all 1024 threads after the histogram is complete and
+// before the cluster barrier that follows scoring.
+__device__ __forceinline__ void publish_coarse(const uint32_t* hist, int C, int rank, SelShared* sh) {
+  const int t = threadIdx.x;
+  uint32_t v = 0;
+  if (t < BIN_COUNT / 4) {
+    const uint4 q = reinterpret_cast<const uint4*>(hist)[t];
+    v = q.x + q.y + q.z + q.w;
+  }
+#pragma unroll
+  for (int o = 1; o < 16; o <<= 1) v += __shfl_xor_sync(FULL, v, o);
+  if ((t & 15) == 0 && t < BIN_COUNT / 4) {
+    const uint32_t a = smem_u32(&sh->coarse[rank][t >> 4]);
+    for (int c = 0; c < C; ++c) st_cluster_u32(mapa(a, (uint32_t)c), v);
+  }
+  if (t == 0) {
+    const uint32_t a = smem_u32(&sh->over[rank]);
+    for (int c = 0; c < C; ++c) st_cluster_u32(mapa(a, (uint32_t)c), sh->over_local);
+  }
+}
+
+// One warp: over 64 bins in descending order (bin = hi - 2 * lane - j, j < 2,
+// counts cnt(bin)), finds the bin holding the need-th key after `before`
+// keys. Returns true and sets (bin, before keys above it, its count) if found.
+__device__ __forceinline__ bool warp_pick_desc(uint32_t c_hi, uint32_t c_lo, uint32_t before, uint32_t need, int hi,
+                                               int& bin, uint32_t& above, uint32_t& cnt) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t pair = c_hi + c_lo;
+  uint32_t incl = pair;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t y = __shfl_up_sync(FULL, incl, o);
+    if (lane >= o) incl += y;
+  }
+  const uint32_t ex = before + incl - pair;
+  const bool in_hi = ex < need && need <= ex + c_hi;
+  const bool in_lo = !in_hi && ex + c_hi < need && need <= ex + pair;
+  const uint32_t m = __ballot_sync(FULL, in_hi || in_lo);
+  if (m == 0u) return false;
+  const int src = __ffs(m) - 1;
+  const int b = in_hi ? hi - 2 * lane : hi - 2 * lane - 1;
+  const uint32_t a = in_hi ? ex : ex + c_hi;
+  const uint32_t c = in_hi ? c_hi : c_lo;
+  bin = __shfl_sync(FULL, b, src);
+  above = __shfl_sync(FULL, a, src);
+  cnt = __shfl_sync(FULL, c, src);
+  return true;
+}
+
+template <typename KeyAddr>
+__device__ __forceinline__ uint4 lds_key4(KeyAddr key_addr, int i) {
+  uint4 v;
+  asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(key_addr(i)));
+  return v;
+}
+
+// Returns false (having changed nothing) when the exact radix path must run
+// instead. key_at(i) / key_addr(i): local key i < n and its shared address
+// (keys are read four at a time from 128-key chunks, which lie in one
+// contiguous 16-byte aligned run; keys past n up to the chunk end may hold
+// anything). hist: this CTA's histogram, at the same offset in every CTA.
+// g0_of(c): first global index of CTA c. emit(pos, i) as in ordered_compact.
+// scratch: bin_scratch_words() words, the same offset in every CTA. The
+// cluster has synchronised since publish_coarse.
+template <bool INT_KEYS, typename KeyAt, typename KeyAddr, typename G0Of, typename Emit>
+__device__ bool binned_select(KeyAt key_at, KeyAddr key_addr, int n, uint32_t k, int C, int rank, G0Of g0_of,
+                              const uint32_t* hist, SelShared* sh, uint32_t* scratch, Emit emit,
+                              unsigned long long* ts = nullptr) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+  uint2* own = reinterpret_cast<uint2*>(scratch);            // [BIN_CAND_CAP] (key, local index)
+  uint2* all = own + BIN_CAND_CAP;                            // [BIN_CAND_CAP] (key, global index)
+  uint32_t* flag = reinterpret_cast<uint32_t*>(all + BIN_CAND_CAP);
+  // resolve (warp 0): coarse bins, then the fine bins of the chosen coarse bin
+  if (warp == 0) {
+    uint32_t over = 0, ch = 0, cl = 0;
+    for (int c = 0; c < C; ++c) {
+      over += sh->over[c];
+      ch += sh->coarse[c][63 - 2 * lane];
+      cl += sh->coarse[c][62 - 2 * lane];
+    }
+    int cb = -1, bstar = -1;
+    uint32_t before = 0, ccnt = 0, above = 0, in_bin = 0;
+    bool ok = over < k && warp_pick_desc(ch, cl, over, k, 63, cb, before, ccnt);
+    if (ok) {
+      const int f_hi = cb * 64 + 63 - 2 * lane;
+      uint32_t fh = 0, fl = 0;
+      for (int c = 0; c < C; ++c) {
+        const uint32_t* h = cluster.map_shared_rank(hist, c);
+        fh += h[f_hi];
+        fl += h[f_hi - 1];
+      }
+      ok = warp_pick_desc(fh, fl, before, k, cb * 64 + 63, bstar, above, in_bin);
+    }
+    if (lane == 0) {
+      sh->bin = ok ? (uint32_t)bstar : 0xffffffffu;
+      sh->above = above;
+      sh->total_in_bin = in_bin;
+      sh->ncand = 0u;
+    }
+  }
+  if (tid < SEL_MAX_C) sh->selc[tid] = 0u;
+  __syncthreads();
+  sel_stamp(ts, 19);
+  if (sh->bin == 0xffffffffu) return false;                           // the k-th key is outside the range
+  const int bstar = (int)sh->bin;
+  const uint32_t above = sh->above, in_bin = sh->total_in_bin;
+  if (!INT_KEYS && in_bin > (uint32_t)BIN_CAND_CAP) return false;     // too many keys at the boundary
+  const uint32_t need = k - above;                                    // 1 <= need <= in_bin
+  if (INT_KEYS) {
+    // every key of bin b* has the value b*: take the first `need` of them in index order
+    SelThreshold th;
+    th.t = bin_lo<true>(bstar);
+    th.take_eq = need == in_bin ? 0xffffffffu : need;   // whole bin: every key >= t
+    ordered_compact(key_at, n, th, C, rank, sh, emit, ts);
+    return true;
+  }
+  const uint32_t lo = bin_lo<false>(bstar), hi = bin_hi<false>(bstar);
+  // pass 1 (four keys per lane): per-warp counts of keys above b*; this CTA's candidates
+  const int nchunks = (n + 127) / 128;
+  const int per_warp = (nchunks + nw - 1) / nw;
+  const int c0 = warp * per_warp, c1 = min(nchunks, c0 + per_warp);
+  uint32_t n_above = 0;
+  for (int chk = c0; chk < c1; ++chk) {
+    const int i0 = chk * 128 + 4 * lane;
+    const uint4 q = lds_key4(key_addr, i0);
+    const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
+    bool any = false;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool valid = i0 + j < n;
+      n_above += (valid && kv[j] > hi) ? 1u : 0u;
+      any |= valid && kv[j] >= lo && kv[j] <= hi;
+    }
+    if (__any_sync(FULL, any)) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        if (i0 + j < n && kv[j] >= lo && kv[j] <= hi) {
+          const uint32_t slot = atomicAdd(&sh->ncand, 1u);
+          if (slot < (uint32_t)BIN_CAND_CAP) own[slot] = make_uint2(kv[j], (uint32_t)(i0 + j));
+        }
+      }
+    }
+  }
+  n_above = __reduce_add_sync(FULL, n_above);
+  if (lane == 0) sh->cnt_w[warp][0] = n_above;
+  __syncthreads();
+  if (tid < C) {
+    uint32_t a = 0;
+    for (int w = 0; w < nw; ++w) a += sh->cnt_w[w][0];
+    uint32_t* dst = cluster.map_shared_rank(&sh->counts[rank][0], (unsigned)tid);
+    dst[0] = a;
+    dst[1] = sh->ncand;
+  }
+  sel_stamp(ts, 16);
+  cluster_sync();
+  sel_stamp(ts, 17);
+  // gather every CTA's candidates (in_bin of them in total)
+  const int m = (int)in_bin;
+  for (int e = tid; e < m; e += blockDim.x) {
+    int c = 0, off = 0;
+    while (c < C - 1 && e >= off + (int)sh->counts[c][1]) off += (int)sh->counts[c++][1];
+    const uint2 v = *cluster.map_shared_rank(own + (e - off), (unsigned)c);
+    all[e] = make_uint2(v.x, (uint32_t)g0_of(c) + v.y);
+  }
+  __syncthreads();
+  sel_stamp(ts, 20);
+  // exact order among the candidates: key descending, then index ascending
+  for (int e = tid; e < m; e += blockDim.x) {
+    const uint2 me = all[e];
+    uint32_t ahead = 0;
+    for (int j = 0; j < m; ++j) {
+      const uint2 o = all[j];
+      ahead += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1u : 0u;
+    }
+    const uint32_t take = ahead < need ? 1u : 0u;
+    flag[e] = take;
+    if (take) {
+      int c = 0, off = 0;
+      while (c < C - 1 && e >= off + (int)sh->counts[c][1]) off += (int)sh->counts[c++][1];
+      atomicAdd(&sh->selc[c], 1u);
+    }
+  }
+  __syncthreads();
+  sel_stamp(ts, 21);
+  // this CTA's candidates: taken ones become all ones (> hi), the rest 0 (< lo)
+  {
+    int off = 0;
+    for (int c = 0; c < rank; ++c) off += (int)sh->counts[c][1];
+    const int mine = (int)sh->counts[rank][1];
+    const uint32_t g0 = (uint32_t)g0_of(rank);
+    for (int e = tid; e < mine; e += blockDim.x) {
+      const uint32_t i = all[off + e].y - g0;
+      const uint32_t take = flag[off + e];
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(key_addr((int)i)), "r"(take ? 0xffffffffu : 0u) : "memory");
+      if (take) atomicAdd(&sh->cnt_w[((int)i / 128) / per_warp][0], 1u);
+    }
+  }
+  __syncthreads();
+  sel_stamp(ts, 4);
+  if (tid == 0) {
+    uint32_t run = 0;
+    for (int c = 0; c < rank; ++c) run += sh->counts[c][0] + sh->selc[c];
+    for (int w = 0; w < nw; ++w) {
+      sh->off_w[w][0] = run;
+      run += sh->cnt_w[w][0];
+    }
+  }
+  __syncthreads();
+  sel_stamp(ts, 18);
+  // pass 2: emit keys > hi in index order (four per lane, warp-wide prefix)
+  uint32_t run = sh->off_w[warp][0];
+  for (int chk = c0; chk < c1; ++chk) {
+    const int i0 = chk * 128 + 4 * lane;
+    const uint4 q = lds_key4(key_addr, i0);
+    const bool t0 = i0 < n && q.x > hi, t1 = i0 + 1 < n && q.y > hi;
+    const bool t2 = i0 + 2 < n && q.z > hi, t3 = i0 + 3 < n && q.w > hi;
+    const uint32_t cnt = (uint32_t)t0 + (uint32_t)t1 + (uint32_t)t2 + (uint32_t)t3;
+    uint32_t incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t y = __shfl_up_sync(FULL, incl, o);
+      if (lane >= o) incl += y;
+    }
+    uint32_t pos = run + incl - cnt;
+    if (t0) emit(pos++, i0);
+    if (t1) emit(pos++, i0 + 1);
+    if (t2) emit(pos++, i0 + 2);
+    if (t3) emit(pos, i0 + 3);
+    run += __shfl_sync(FULL, incl, 31);
+  }
+  __syncthreads();
+  return true;
 }
 
 }  // namespace hst

@@ -26,9 +26,16 @@ constexpr int FUSED_WARPS = FUSED_THREADS / 32;
 constexpr int SCORE_PF = 2;                      // 32-key blocks in flight per warp
 constexpr int ATTEND_THREADS = 256;              // the attention kernel
 constexpr int ATTEND_WARPS = ATTEND_THREADS / 32;
+constexpr int ATTEND_BUFS = 2;                    // bf16: K/V slots per computing warp
+constexpr int ATTEND_MMA_WARPS = ATTEND_WARPS / ATTEND_BUFS;   // bf16: computing warps
 constexpr int ATTEND_MAX_SPLITS = 128;           // one head's partials fit in the warp slots
 
 __device__ __forceinline__ uint32_t key_of(float s) { return __float_as_uint(s); }
+
+static_assert(bin_scratch_words() * 4 <= TABLE_BYTES, "the selection scratch lives in the first table");
+static_assert(hist_words(0) + hist_words(1) >= BIN_COUNT, "the selection bins live in the first two radix histograms");
+static_assert(FUSED_THREADS * 4 == BIN_COUNT, "publish_coarse reads four bins per thread");
+static_assert(ATTEND_MMA_WARPS * ATTEND_BUFS == ATTEND_WARPS, "the bf16 slots are the warp slots, regrouped");
 
 __host__ __device__ constexpr int table_chunks(int LP) { return LP > 32 ? 2 : 1; }
 
@@ -42,19 +49,23 @@ struct FusedParams {
   float* O;
   int* idx_out;                   // [pairs][k] ascending (always written)
   unsigned int* counters;         // [pairs] zeroed here for the attention kernel's merge (may be null)
-  unsigned long long* phase_ts;   // optional: [grid][PHASES] globaltimer stamps (profiling)
+  unsigned long long* phase_ts;   // optional: [grid][PHASES] clock stamps (profiling)
   int Hq, Hkv, Ncap, N, L, P, k, C, blocks_per_cta, chunk;
   float tau, scale;
 };
 
 constexpr int PHASES = 24;
 
+// Profiling stamps (see sk_profile_phases): the SM clock at each phase, and
+// the global timer at the start (slot 22) and the exit (slot 23).
 __device__ __forceinline__ void stamp(unsigned long long* ts, int phase) {
   if (ts != nullptr && threadIdx.x == 0) {
-    unsigned long long t;
-    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-    ts[blockIdx.x * PHASES + phase] = t;
-    if (phase == 0 || phase == 7) ts[blockIdx.x * PHASES + 22 + (phase == 7)] = (unsigned long long)clock64();
+    ts[blockIdx.x * PHASES + phase] = (unsigned long long)clock64();
+    if (phase == 0 || phase == 7) {
+      unsigned long long t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      ts[blockIdx.x * PHASES + 22 + (phase == 7)] = t;
+    }
   }
 }
 
@@ -85,7 +96,7 @@ struct FusedSmem {
     hist1 = a; a += 4u * hist_words(1);
     hist2 = a; a += 4u * hist_words(2);
     keysA = a;
-    nA = (segA_end > a) ? (segA_end - a) / 4u : 0u;
+    nA = (segA_end > a) ? ((segA_end - a) / 4u) & ~127u : 0u;   // whole 128-key chunks
     keysB = segB;
   }
   __device__ uint32_t key_capacity() const { return nA + (segB_end > segB ? (segB_end - segB) / 4u : 0u); }
@@ -97,53 +108,32 @@ __device__ __forceinline__ T* sptr(unsigned char* dyn, uint32_t base, uint32_t a
   return reinterpret_cast<T*>(dyn + (addr - base));
 }
 
-// Zeroes, in the first copy of every chunk table (columns x < S_c), the cells
-// of rows >= 2^P and of tables >= L.
+// Zeroes every copy of the padding cells of the chunk tables: rows >= 2^P
+// and columns whose table is >= L. The other cells are written by the table
+// build of the cluster.
 template <int LP>
-__device__ __forceinline__ void zero_table_padding(float* t0, float* t1, int L, int P) {
+__device__ __forceinline__ void zero_table_padding_all(float* t0, float* t1, int L, int P) {
   const int nb = 1 << P;
 #pragma unroll
   for (int c = 0; c < table_chunks(LP); ++c) {
     float* t = c ? t1 : t0;
     const int S = id_chunk_size(L, c);
-    for (int e = threadIdx.x; e < 256 * S; e += blockDim.x) {
-      const int b = e / S, x = e % S;
-      if (b >= nb || 32 * c + x >= L) t[b * TABLE_COLS + x] = 0.f;
+    if (nb == 256 && 32 * c + S <= L) continue;       // no padding in this chunk
+    for (int e = threadIdx.x; e < 256 * TABLE_COLS; e += blockDim.x) {
+      const int b = e / TABLE_COLS, x = e % TABLE_COLS;
+      if (b >= nb || 32 * c + x % S >= L) t[e] = 0.f;
     }
   }
 }
 
-// Fills every chunk table from the first copies built by the cluster: the
-// 4-column group starting at table 4g is owned by CTA (4g) / per; it is read
-// from the owner (distributed shared memory, 16-byte loads) and written to all
-// 64 / S_c copies of its columns in this CTA.
-template <int LP>
-__device__ __forceinline__ void pull_and_replicate_tables(cg::cluster_group& cluster, float* t0, float* t1, int L,
-                                                          int P, int per, int rank) {
-  const int nbk = 1 << P;
-#pragma unroll
-  for (int c = 0; c < table_chunks(LP); ++c) {
-    float* t = c ? t1 : t0;
-    const int S = id_chunk_size(L, c);
-    const int groups = S / 4;
-    for (int e = threadIdx.x; e < 256 * groups; e += blockDim.x) {
-      const int bb = e / groups, g = e % groups;
-      const int l = 32 * c + 4 * g;                        // first table of the group
-      const int owner = l < L ? l / per : rank;            // padding groups are zero everywhere
-      float* src = t + bb * TABLE_COLS + 4 * g;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (bb < nbk) v = *reinterpret_cast<const uint4*>(cluster.map_shared_rank(src, (unsigned)owner));
-      for (int x = 4 * g; x < TABLE_COLS; x += S) *reinterpret_cast<uint4*>(t + bb * TABLE_COLS + x) = v;
-    }
-  }
-}
-
-// Scores keys of blocks blk0 + warp + i * NW (i < nb) into sort keys and the
-// level-0 histogram. buf holds the first SCORE_PF blocks, already requested.
+// Scores keys of blocks blk0 + warp + i * NW (i < nb) into sort keys in
+// shared memory and counts them into the CTA's selection histogram. buf holds
+// the first SCORE_PF blocks, already requested.
 template <int LP, bool NORM>
 __device__ __forceinline__ void score_blocks(KeyIds<LP> (&buf)[SCORE_PF], const uint8_t* __restrict__ ids_pair,
                                              const __half* __restrict__ norms_pair, int N, int blk0, int nb,
-                                             uint32_t col0, uint32_t col1, const FusedKeys keys, uint32_t* hist0) {
+                                             uint32_t col0, uint32_t col1, const FusedKeys keys, uint32_t* hist,
+                                             SelShared* sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   for (int it = 0; it < nb; it += SCORE_PF) {
 #pragma unroll
@@ -158,10 +148,11 @@ __device__ __forceinline__ void score_blocks(KeyIds<LP> (&buf)[SCORE_PF], const 
         const float s = score_key<LP, NORM>(cur, col0, col1);
         const int gkey = (blk0 + warp + i * nw) * 32 + lane;
         if (gkey < N) {
-          const uint32_t key = key_of(s);
+          // soft scores sort by their f32 bits; hard-hash scores are small integers
+          const uint32_t key = NORM ? key_of(s) : (uint32_t)s;
           const uint32_t li = (uint32_t)(gkey - blk0 * 32);
           asm volatile("st.shared.u32 [%0], %1;" ::"r"(keys.addr(li)), "r"(key) : "memory");
-          atomicAdd(&hist0[key >> 20], 1u);
+          bin_count<!NORM>(key, hist, sh);
         }
       }
     }
@@ -189,7 +180,8 @@ struct AttendSmem {
   uint32_t phases;         // 4 bytes per slot
   uint32_t slot0;          // warp w's slot: slot0 + w * slot_stride
   uint32_t slot_stride;
-  int nslots;
+  int ncw;                 // computing warps (one partial each)
+  int nbuf;                // slots per computing warp (bf16)
   uint32_t partials;
 };
 
@@ -200,12 +192,13 @@ template <int D, typename KVT, typename KeyFn>
 __device__ __forceinline__ void attend_and_merge(unsigned char* dyn, uint32_t base, const AttendSmem& as,
                                                  const KVT* Qg, const KVT* Kp, const KVT* Vp, int G, float scale,
                                                  KeyFn keys, int cnt, int nrows, float*& cM, float*& cL, float*& cO) {
-  const int ncw = as.nslots;
+  const int ncw = as.ncw;
   const PartialView pv = partial_view(sptr<float>(dyn, base, as.partials), ncw, G, D, cM, cL, cO);
   if constexpr (sizeof(KVT) == 2) {
-    attend_tiles_bf16<D>(reinterpret_cast<const __nv_bfloat16*>(Kp), reinterpret_cast<const __nv_bfloat16*>(Vp), keys,
-                         cnt, nrows, G, scale, as.qs, as.slot0, as.slot_stride, as.mbar0,
-                         sptr<uint32_t>(dyn, base, as.phases), ncw, pv);
+    attend_tiles_bf16<D, ATTEND_BUFS>(reinterpret_cast<const __nv_bfloat16*>(Kp),
+                                      reinterpret_cast<const __nv_bfloat16*>(Vp), keys, cnt, nrows, G, scale, as.qs,
+                                      as.slot0, as.slot_stride, as.mbar0, sptr<uint32_t>(dyn, base, as.phases), ncw,
+                                      pv);
   } else {
     attend_keys_f32<D>(reinterpret_cast<const float*>(Qg), reinterpret_cast<const float*>(Kp),
                        reinterpret_cast<const float*>(Vp), keys, cnt, nrows, G, scale, ncw, pv);
@@ -221,7 +214,7 @@ __device__ __forceinline__ void attend_setup(unsigned char* dyn, uint32_t base, 
                                              int G) {
   if constexpr (sizeof(KVT) == 2) {
     stage_q<D>(reinterpret_cast<const __nv_bfloat16*>(Qg), G, sptr<unsigned char>(dyn, base, as.qs));
-    if (threadIdx.x < as.nslots) {
+    if ((int)threadIdx.x < as.ncw * as.nbuf) {
       mbar_init(as.mbar0 + 8u * threadIdx.x, 1);
       sptr<uint32_t>(dyn, base, as.phases)[threadIdx.x] = 0u;
     }
@@ -255,7 +248,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
   fs.plan(smem_u32(dyn), dyn_size, NCH);
   // The host sizes slices from the same plan; a mismatch (a host bug) is
   // flagged and every CTA of the grid leaves here (the test is uniform).
-  if (fs.segB > fs.segB_end || (uint32_t)p.blocks_per_cta * 32u > fs.key_capacity()) {
+  if (fs.segB > fs.segB_end || (((uint32_t)p.blocks_per_cta * 32u + 127u) & ~127u) > fs.key_capacity()) {
     if (tid == 0) atomicOr(&g_error_word, ERR_LAYOUT);
     return;
   }
@@ -265,6 +258,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
                        sptr<uint32_t>(dyn, fs.base, fs.hist2)};
   float* tab0 = sptr<float>(dyn, fs.base, fs.tbl0);
   float* tab1 = sptr<float>(dyn, fs.base, fs.tbl1);
+  uint32_t* tab0u = sptr<uint32_t>(dyn, fs.base, fs.tbl0);   // selection scratch once scoring is done
 
   const int nblk_pair = (p.N + 31) / 32;
   const int blk0 = min(nblk_pair, rank * p.blocks_per_cta);
@@ -275,59 +269,86 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
   const uint8_t* ids_pair = p.ids + pair_keys * LP;
   const __half* norms_pair = p.norms + pair_keys;
 
-  // ---- setup: zero histograms and table padding; all CTAs started before any remote access
-  for (int i = tid; i < hist_words(0); i += blockDim.x) hist[0][i] = 0u;
-  for (int i = tid; i < hist_words(1); i += blockDim.x) hist[1][i] = 0u;
-  for (int i = tid; i < hist_words(2); i += blockDim.x) hist[2][i] = 0u;
-  zero_table_padding<LP>(tab0, tab1, p.L, p.P);
+  // ---- setup. The cluster barrier is split: this arrive, and the wait just
+  // before the first store into another CTA (the tables), so the barrier's
+  // latency hides behind the table build. The first key blocks are requested
+  // now; they arrive while the tables are built.
+  cluster_arrive_relaxed();
+  KeyIds<LP> buf[SCORE_PF];
+  prefetch_blocks<LP, !HATA>(buf, ids_pair, norms_pair, blk0, nb);
+  if (tid == 0) sh->over_local = 0u;
+  for (int i = tid; i < BIN_COUNT; i += blockDim.x) hist[0][i] = 0u;     // hist0 + hist1: the selection bins
+  zero_table_padding_all<LP>(tab0, tab1, p.L, p.P);
   if (rank == 0 && tid == 0 && p.counters) p.counters[pair] = 0u;     // for the attention kernel's merge
-  cluster_sync();
   stamp(p.phase_ts, 8);
 
-  // ---- SOCKET step 2: this CTA builds a range of tables (4-table aligned) into
-  // its own first copy; after the barrier every CTA pulls the other ranges.
+  // ---- SOCKET step 2: this CTA builds a range of tables (4-table aligned) and
+  // stores every entry into all its column copies in every CTA of the cluster.
   const QT* Qg = reinterpret_cast<const QT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
   const int per = ((p.L + C - 1) / C + 3) & ~3;
   {
     const int l0 = min(p.L, rank * per);
     const int nl = min(p.L, l0 + per) - l0;
+    const uint32_t t0a = fs.tbl0, t1a = fs.tbl1;
+    const int L = p.L;
     auto store = [=](int bb, int l, float v) {
       const int c = l >= 32 ? 1 : 0;
-      (c ? tab1 : tab0)[bb * TABLE_COLS + (l - 32 * c)] = v;
+      const int S = id_chunk_size(L, c);
+      const uint32_t row = (c ? t1a : t0a) + (uint32_t)bb * (TABLE_COLS * 4u);
+      for (int x = l - 32 * c; x < TABLE_COLS; x += S)
+        for (int r = 0; r < C; ++r) st_cluster_f32(mapa(row + 4u * x, (uint32_t)r), v);
     };
+    auto before_store = [] { cluster_wait(); };    // every CTA of the cluster has started
     void* scratch = sptr<void>(dyn, fs.base, fs.keysA);
     if (nl > 0) {
-      if constexpr (HATA) build_hamming_table<D>(Qg, G, p.R, l0, nl, scratch, store);
-      else build_bucket_table<D>(Qg, G, p.R, p.P, p.tau, l0, nl, scratch, store, p.phase_ts);
+      if constexpr (HATA) build_hamming_table<D>(Qg, G, p.R, l0, nl, scratch, store, before_store);
+      else build_bucket_table<D>(Qg, G, p.R, p.P, p.tau, l0, nl, scratch, store, p.phase_ts, before_store);
+    } else {
+      cluster_wait();
     }
   }
   stamp(p.phase_ts, 9);
-  cluster_sync();
-  stamp(p.phase_ts, 10);
-  KeyIds<LP> buf[SCORE_PF];
-  prefetch_blocks<LP, !HATA>(buf, ids_pair, norms_pair, blk0, nb);
-  pull_and_replicate_tables<LP>(cluster, tab0, tab1, p.L, p.P, per, rank);
-  __syncthreads();
+  cluster_sync();     // every table entry has landed in every CTA
   stamp(p.phase_ts, 1);
 
-  // ---- SOCKET step 3: scores of this CTA's slice (kept on chip) + level-0 histogram
+  // ---- SOCKET step 3: scores of this CTA's slice, kept on chip
   const FusedKeys keys = fs.keys();
   score_blocks<LP, !HATA>(buf, ids_pair, norms_pair, p.N, blk0, nb, fs.tbl0 + 4u * lane, fs.tbl1 + 4u * lane, keys,
-                          hist[0]);
+                          hist[0], sh);
   stamp(p.phase_ts, 11);
   __syncthreads();
-  cluster_sync();
+  publish_coarse(hist[0], C, rank, sh);
+  cluster_sync();     // every CTA's scores and histogram sums are final; the tables are no longer read
   stamp(p.phase_ts, 2);
 
   // ---- SOCKET step 4a: exact top-k across the cluster, ascending indices to idx_out
   auto key_at = [=](int i) -> uint32_t { return lds_u32(keys.addr((uint32_t)i)); };
-  const SelThreshold th = cluster_threshold<FUSED_THREADS>(key_at, n_local, hist, (uint32_t)p.k, C, sh, p.phase_ts);
-  stamp(p.phase_ts, 3);
+  auto key_addr = [=](int i) -> uint32_t { return keys.addr((uint32_t)i); };
+  const int bpc = p.blocks_per_cta;
+  auto g0_of = [=](int c) -> int { return min(nblk_pair, c * bpc) * 32; };
   int* idx_out = p.idx_out + (size_t)pair * p.k;
   const int kk = p.k, g0 = blk0 * 32;
-  ordered_compact(key_at, n_local, th, C, rank, sh, [=](uint32_t pos, int i) {
+  auto emit = [=](uint32_t pos, int i) {
     if (pos < (uint32_t)kk) idx_out[pos] = g0 + i;
-  }, p.phase_ts);
+  };
+  const bool done = binned_select<HATA>(key_at, key_addr, n_local, (uint32_t)p.k, C, rank, g0_of, hist[0], sh, tab0u,
+                                       emit, p.phase_ts);
+  if (!done) {
+    // exact radix select over the whole key range; every CTA has finished
+    // reading the other CTAs' bins before any reuses its own
+    cluster_sync();
+    for (int i = tid; i < hist_words(0); i += blockDim.x) hist[0][i] = 0u;
+    for (int i = tid; i < hist_words(1); i += blockDim.x) hist[1][i] = 0u;
+    for (int i = tid; i < hist_words(2); i += blockDim.x) hist[2][i] = 0u;
+    __syncthreads();
+    histogram_pass(key_at, n_local, sel_shift(0), sel_bits(0), 32, 0u, hist[0]);
+    __syncthreads();
+    cluster_sync();
+    const SelThreshold th = cluster_threshold<FUSED_THREADS>(key_at, n_local, hist, (uint32_t)p.k, C, sh,
+                                                             p.phase_ts);
+    stamp(p.phase_ts, 3);
+    ordered_compact(key_at, n_local, th, C, rank, sh, emit, p.phase_ts);
+  }
   stamp(p.phase_ts, 12);
   // the attention kernel may start once every CTA has written its indices
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -466,9 +487,22 @@ struct AttendParams {
   float* part;             // [pairs][splits][G][D + 2]: (m, l, o[D]) per head
   unsigned int* counters;  // [pairs], zero on entry; left zero on exit
   float* O;                // [B][Hq][D]
+  unsigned long long* phase_ts;  // optional: [pairs * splits][PHASES] clock stamps (profiling)
   int Hq, Hkv, Ncap, n, keys_per_split, splits;
   float scale;
 };
+
+__device__ __forceinline__ void attend_stamp(unsigned long long* ts, int phase) {
+  if (ts != nullptr && threadIdx.x == 0) {
+    const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+    ts[cta * PHASES + phase] = (unsigned long long)clock64();
+    if (phase == 0 || phase == 7) {
+      unsigned long long t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      ts[cta * PHASES + 22 + (phase == 7)] = t;
+    }
+  }
+}
 
 // Shared bytes of socket_attend_kernel: query stage, mbarriers and phases,
 // warp slots, partials, the CTA's index list, a flag word.
@@ -479,15 +513,19 @@ __host__ __device__ inline size_t attend_smem_bytes(int G, int keys_per_split) {
 }
 
 // Exact attention over a key list, split over keys: grid = (pairs, splits).
-// Each CTA attends over its range and writes one partial (m, l, o) per head;
-// the last CTA of a pair to finish (counted with an atomic) merges the
-// pair's partials in split order and writes O, so the result does not depend
-// on the order the CTAs ran. Launched after the selection kernel with
-// programmatic dependent launch: everything before griddepcontrol.wait
-// overlaps that kernel's tail.
-template <int D, typename KVT>
+// Each CTA attends over its range and forms one partial (m, l, o) per head.
+// CLUSTER = true: the splits of a pair form one thread-block cluster; after a
+// cluster barrier CTA r merges heads r, r + splits, ... reading every CTA's
+// partial from its shared memory (split order). CLUSTER = false: the partial
+// goes to the workspace and the last CTA of a pair to finish (counted with an
+// atomic) merges the pair's partials in split order. Either way the result
+// does not depend on the order the CTAs ran. Launched after the selection
+// kernel with programmatic dependent launch: everything before
+// griddepcontrol.wait overlaps that kernel's tail.
+template <int D, typename KVT, bool CLUSTER>
 __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const AttendParams p) {
   extern __shared__ __align__(1024) unsigned char dyn[];
+  attend_stamp(p.phase_ts, 0);
   const int pair = blockIdx.x, split = blockIdx.y;
   const int G = p.Hq / p.Hkv;
   const int b = pair / p.Hkv, kvh = pair % p.Hkv;
@@ -505,14 +543,17 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
     as.slot0 = a;
     as.slot_stride = kv_slot_bytes<D>();
     a += ATTEND_WARPS * kv_slot_bytes<D>();
-    as.nslots = ATTEND_WARPS;
+    as.ncw = sizeof(KVT) == 2 ? ATTEND_MMA_WARPS : ATTEND_WARPS;
+    as.nbuf = ATTEND_BUFS;
     as.partials = a;
   }
   const size_t smem_total = attend_smem_bytes<D>(G, p.idx ? p.keys_per_split : 0);
   uint32_t* last_flag = reinterpret_cast<uint32_t*>(dyn + (smem_total - 16));
   int* list_s = reinterpret_cast<int*>(dyn + (as.partials - base) + partial_bytes(ATTEND_WARPS, G, D));
   attend_setup<D, KVT>(dyn, base, as, Qg, G);
+  attend_stamp(p.phase_ts, 1);
   asm volatile("griddepcontrol.wait;" ::: "memory");   // the key list is complete from here on
+  attend_stamp(p.phase_ts, 2);
   const KVT* Kp = reinterpret_cast<const KVT*>(p.K) + pair_keys * D;
   const KVT* Vp = reinterpret_cast<const KVT*>(p.V) + pair_keys * D;
   float *cM, *cL, *cO;
@@ -520,11 +561,38 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
     const int* list = p.idx + (size_t)pair * p.n + i0;      // one coalesced load of this CTA's indices
     for (int i = threadIdx.x; i < cnt; i += blockDim.x) list_s[i] = __ldcg(list + i);
     __syncthreads();
+    attend_stamp(p.phase_ts, 3);
     attend_and_merge<D, KVT>(dyn, base, as, Qg, Kp, Vp, G, p.scale, [=](int i) { return list_s[i]; }, cnt, p.Ncap,
                              cM, cL, cO);
   } else {
     attend_and_merge<D, KVT>(dyn, base, as, Qg, Kp, Vp, G, p.scale, [=](int i) { return i0 + i; }, cnt, p.Ncap, cM,
                              cL, cO);
+  }
+  attend_stamp(p.phase_ts, 4);
+  if constexpr (CLUSTER) {
+    cg::cluster_group cluster = cg::this_cluster();
+    cluster_sync();            // every split's partial is final
+    attend_stamp(p.phase_ts, 5);
+    for (int h = split; h < G; h += p.splits) {
+      for (int dv = threadIdx.x; dv < D; dv += blockDim.x) {
+        float mm = -INFINITY;
+        for (int sp = 0; sp < p.splits; ++sp) mm = fmaxf(mm, *cluster.map_shared_rank(cM + h, sp));
+        float lsum = 0.f, o = 0.f;
+        for (int sp = 0; sp < p.splits; ++sp) {
+          const float m = *cluster.map_shared_rank(cM + h, sp);
+          if (m != -INFINITY) {
+            const float w = exp2f(m - mm);
+            lsum += w * *cluster.map_shared_rank(cL + h, sp);
+            o += w * *cluster.map_shared_rank(cO + h * D + dv, sp);
+          }
+        }
+        p.O[((size_t)b * p.Hq + kvh * G + h) * D + dv] = o / lsum;
+      }
+    }
+    attend_stamp(p.phase_ts, 6);
+    cluster_sync();            // the other CTAs read this CTA's partial until here
+    attend_stamp(p.phase_ts, 7);
+    return;
   }
   float* mine = p.part + ((size_t)pair * p.splits + split) * G * (D + 2);
   for (int e = threadIdx.x; e < G * (D + 2); e += blockDim.x) {
@@ -535,7 +603,11 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
   __syncthreads();
   if (threadIdx.x == 0) *last_flag = (atomicAdd(&p.counters[pair], 1u) == (unsigned)p.splits - 1u) ? 1u : 0u;
   __syncthreads();
-  if (*last_flag == 0u) return;
+  attend_stamp(p.phase_ts, 5);
+  if (*last_flag == 0u) {
+    attend_stamp(p.phase_ts, 7);
+    return;
+  }
   // ---- last CTA of the pair: merge the splits in order, one head at a time:
   // the head's partials are copied into shared memory (the warp slots are
   // free; splits <= ATTEND_MAX_SPLITS keeps them in bounds) with independent
@@ -565,6 +637,8 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
     __syncthreads();
   }
   if (threadIdx.x == 0) p.counters[pair] = 0u;
+  attend_stamp(p.phase_ts, 6);
+  attend_stamp(p.phase_ts, 7);
 }
 
 }  // namespace hst

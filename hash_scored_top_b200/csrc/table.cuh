@@ -108,19 +108,22 @@ __device__ __forceinline__ void stage_rows(const __nv_bfloat16* __restrict__ R, 
   for (int e = threadIdx.x; e < nrows * (D / 8); e += blockDim.x) dst[e] = __ldg(src + e);
 }
 
+struct NoHook {
+  __device__ void operator()() const {}
+};
+
 // Computes T_l(b) for the tables l in [l0, l0 + nl) and every bucket b < 2^P,
 // calling store(b, l, value_f32) once per entry. Qg points at the G query
 // rows of the pair (row stride D); scratch holds table_scratch_bytes. All
-// threads of the block must call this; it ends with __syncthreads().
-template <int D, typename QT, typename Store>
+// threads of the block must call this; it calls before_store() (all threads,
+// converged) just before the first store and ends with __syncthreads().
+template <int D, typename QT, typename Store, typename Hook = NoHook>
 __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_bfloat16* __restrict__ R, int P,
                                    float tau, int l0, int nl, void* scratch, Store store,
-                                   unsigned long long* ts = nullptr) {
+                                   unsigned long long* ts = nullptr, Hook before_store = Hook()) {
   auto tstamp = [&](int ph) {
     if (ts != nullptr && threadIdx.x == 0) {
-      unsigned long long t;
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-      ts[blockIdx.x * 24 + ph] = t;
+      ts[blockIdx.x * 24 + ph] = (unsigned long long)clock64();
     }
   };
   const int tid = threadIdx.x, nthr = blockDim.x;
@@ -148,7 +151,7 @@ __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_
     const double x = two_over_tau * z;                  // logit gap between bit=1 and bit=0
     const double e = exp(-fabs(x));
     const double p_big = 1.0 / (1.0 + e);               // sigmoid(|x|)
-    const double p_small = e / (1.0 + e);               // sigmoid(-|x|)
+    const double p_small = e * p_big;                   // sigmoid(-|x|)
     sig[item * 2 + 1] = x >= 0.0 ? p_big : p_small;     // bit j = 1
     sig[item * 2 + 0] = x >= 0.0 ? p_small : p_big;     // bit j = 0
   });
@@ -174,6 +177,7 @@ __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_
   tstamp(13);
 
   // 4. table entries, summed over the group's heads
+  before_store();
   const int nb = 1 << P;
   for (int item = tid; item < nb * nl; item += nthr) {
     const int li = item % nl;

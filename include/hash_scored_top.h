@@ -12,7 +12,9 @@
  * Conventions shared by every entry point
  * ---------------------------------------
  * - All tensor arguments are DEVICE pointers to contiguous memory owned by
- *   the caller. The library allocates nothing and frees nothing; scratch
+ *   the caller. Alignment: ids 32 bytes; codes, Q, K, V, R, R128 16 bytes;
+ *   norms 2 bytes (cudaMalloc and torch allocations satisfy all of these);
+ *   a misaligned pointer is rejected with SK_ERR_INVALID_ARG. The library allocates nothing and frees nothing; scratch
  *   memory is passed in as `ws` / `ws_bytes` (query the size with
  *   sk_workspace_bytes). `stream` is a cudaStream_t (NULL = legacy default).
  * - Calls are asynchronous on `stream`. Arguments are validated on the host
@@ -234,12 +236,15 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
 int sk_check_status(void* stream);
 
 /* Profiling hook: while `device_buffer` is non-NULL, every selection kernel
- * launch (socket_decode, socket_select, hata_decode) writes %globaltimer
- * stamps per CTA to device_buffer[cta * 24 + phase] (phases such as start,
- * tables built, scores done, histogram levels, threshold found, indices
- * written, exit; slots 22-23 hold clock64 at start and exit). The buffer must
- * hold 24 entries per CTA of the launch (at most 16 * B * Hkv CTAs). Pass
- * NULL to turn it off. Costs one store per phase per CTA. */
+ * launch (socket_decode, socket_select, hata_decode) writes, per CTA, the SM
+ * clock (clock64) at each phase to device_buffer[cta * 24 + phase] (phases
+ * such as start, tables built, scores done, histogram, candidates, indices
+ * written, exit) and the global timer (ns) at start and exit to slots 22 and
+ * 23. The attention kernel of those calls and of socket_sparse_attend
+ * stamps its CTAs (pair-major within each split) from entry 16 * B * Hkv * 24
+ * on. The buffer must hold 24 entries per CTA: 16 * B * Hkv for the
+ * selection plus B * Hkv * splits (at most 128 splits) for the attention.
+ * Pass NULL to turn it off. One store per phase per CTA. */
 int sk_profile_phases(unsigned long long* device_buffer);
 
 /* Thread-local description of the last non-OK return (never NULL). */

@@ -64,7 +64,7 @@ def _rc_and_msg(lib, fn, *args):
 
 def test_host_validation_rejects_without_launching(lib):
     L = lib.lib
-    p = ctypes.c_void_p(16)          # never dereferenced: validation fails first
+    p = ctypes.c_void_p(256)         # never dereferenced: validation fails first
     null = None
     # socket_decode: NULL query
     rc, msg = _rc_and_msg(lib, L.socket_decode, null, p, p, 1, p, p, p, 1, 4, 1, 64, 64, 128, 8, 4, 0.5, 8, 0.1, p,
@@ -108,6 +108,14 @@ def test_host_validation_rejects_without_launching(lib):
     # hard-hash decode with a group of 16 heads
     rc, msg = _rc_and_msg(lib, L.hata_decode, p, p, p, 1, p, p, 1, 16, 1, 64, 64, 128, 8, 0.1, p, null, null, 0, null)
     assert rc == 2 and "G=16" in msg
+    # bucket IDs must allow 32-byte loads
+    rc, msg = _rc_and_msg(lib, L.socket_select, p, 1, p, ctypes.c_void_p(272), p, 1, 4, 1, 64, 64, 128, 8, 4, 0.5, 8,
+                          p, null, 0, null)
+    assert rc == 1 and "ids must be 32-byte aligned" in msg
+    # K rows are bulk-copied: 16-byte alignment
+    rc, msg = _rc_and_msg(lib, L.socket_sparse_attend, p, ctypes.c_void_p(264), p, 1, p, 1, 4, 1, 64, 128, 8, 0.1, p,
+                          p, 1 << 20, null)
+    assert rc == 1 and "K must be 16-byte aligned" in msg
     # unknown dtype
     rc, msg = _rc_and_msg(lib, L.dense_decode, p, p, p, 7, 1, 4, 1, 64, 64, 128, 0.1, p, p, 1 << 20, null)
     assert rc == 1 and "dtype" in msg

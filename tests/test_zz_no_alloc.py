@@ -79,7 +79,7 @@ def test_noalloc_rejects_shapes_beyond_the_static_scratch(lib):
     """Too many pairs for the fixed scratch: a workspace error, nothing launched
     (the pointers are never dereferenced, so this runs without a GPU)."""
     assert lib.lib.sk_noalloc_scratch_bytes() == 4 << 20
-    p = ctypes.c_void_p(16)
+    p = ctypes.c_void_p(256)
     rc = lib.lib.socket_sparse_attend_noalloc(p, p, p, 1, p, 2048, 8, 1, 32, 128, 1, ctypes.c_float(0.1), p, None)
     msg = lib.last_error()
     assert rc == 5 and "static scratch" in msg and "4194304" in msg

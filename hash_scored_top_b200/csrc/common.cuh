@@ -45,6 +45,12 @@ __host__ __device__ inline int id_byte_table(int L, int b, int n) {
 }
 
 // ---------------------------------------------------------------- loads
+// Asks the TMA unit to bring [p, p + bytes) into L2 (no completion to wait
+// for). p and bytes must be multiples of 16.
+__device__ __forceinline__ void prefetch_l2_bulk(const void* p, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ uint4 ldg_stream(const void* p) {
   uint4 r;
   asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
@@ -118,6 +124,11 @@ __device__ __forceinline__ uint32_t mapa(uint32_t addr, uint32_t rank) {
 
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
   asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(addr), "f"(v) : "memory");
+}
+
+__device__ __forceinline__ void st_cluster_v4f32(uint32_t addr, const float* v) {
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "f"(v[0]), "f"(v[1]), "f"(v[2]),
+               "f"(v[3]) : "memory");
 }
 
 __device__ __forceinline__ void st_cluster_u32(uint32_t addr, uint32_t v) {

@@ -335,8 +335,9 @@ __device__ __forceinline__ void bin_count(uint32_t key, uint32_t* hist, SelShare
   else if (b >= 0) atomicAdd(&hist[b], 1u);
 }
 
-// Words of scratch binned_select needs: own and gathered candidates, flags.
-__host__ __device__ constexpr int bin_scratch_words() { return 2 * BIN_CAND_CAP * 2 + BIN_CAND_CAP; }
+// Words of scratch binned_select needs: own and gathered candidates, flags,
+// per-thread counts.
+__host__ __device__ constexpr int bin_scratch_words() { return 2 * BIN_CAND_CAP * 2 + BIN_CAND_CAP + 1024; }
 
 // Stores this CTA's coarse sums and above-range count into every CTA of the
 // cluster. Call with all 1024 threads after the histogram is complete and
@@ -398,15 +399,19 @@ __device__ __forceinline__ uint4 lds_key4(KeyAddr key_addr, int i) {
 // Returns false (having changed nothing) when the exact radix path must run
 // instead. key_at(i) / key_addr(i): local key i < n and its shared address
 // (keys are read four at a time from 128-key chunks, which lie in one
-// contiguous 16-byte aligned run; keys past n up to the chunk end may hold
-// anything). hist: this CTA's histogram, at the same offset in every CTA.
+// contiguous 16-byte aligned run; keys past n up to the chunk end must be 0,
+// which is below every bin of f32 keys). hist: this CTA's histogram, at the same offset in every CTA.
 // g0_of(c): first global index of CTA c. emit(pos, i) as in ordered_compact.
 // scratch: bin_scratch_words() words, the same offset in every CTA. The
 // cluster has synchronised since publish_coarse.
+// The selection is written to out[0..k) (the pair's index list, global
+// index = g0_of(rank) + local index): through `stage` (stage_cap words of
+// shared memory) and coalesced stores when this CTA's part fits, else with
+// emit(pos, i) directly.
 template <bool INT_KEYS, typename KeyAt, typename KeyAddr, typename G0Of, typename Emit>
 __device__ bool binned_select(KeyAt key_at, KeyAddr key_addr, int n, uint32_t k, int C, int rank, G0Of g0_of,
-                              const uint32_t* hist, SelShared* sh, uint32_t* scratch, Emit emit,
-                              unsigned long long* ts = nullptr) {
+                              const uint32_t* hist, SelShared* sh, uint32_t* scratch, Emit emit, int* out,
+                              uint32_t* stage, uint32_t stage_cap, unsigned long long* ts = nullptr) {
   cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
   uint2* own = reinterpret_cast<uint2*>(scratch);            // [BIN_CAND_CAP] (key, local index)
@@ -457,32 +462,37 @@ __device__ bool binned_select(KeyAt key_at, KeyAddr key_addr, int n, uint32_t k,
     return true;
   }
   const uint32_t lo = bin_lo<false>(bstar), hi = bin_hi<false>(bstar);
-  // pass 1 (four keys per lane): per-warp counts of keys above b*; this CTA's candidates
-  const int nchunks = (n + 127) / 128;
-  const int per_warp = (nchunks + nw - 1) / nw;
-  const int c0 = warp * per_warp, c1 = min(nchunks, c0 + per_warp);
+  // Each thread owns `gpt` consecutive groups of 4 keys (gpt odd: the 16-byte
+  // reads of a warp hit distinct banks); the tail up to the 128-key chunk
+  // is 0. Pass 1 counts the keys above b* per thread and gathers this CTA's
+  // candidates.
+  uint32_t* cnt_t = flag + BIN_CAND_CAP;                     // [blockDim.x] per-thread counts
+  const int ngroups = ((n + 127) & ~127) / 4;
+  const int gpt = ((ngroups + (int)blockDim.x - 1) / (int)blockDim.x) | 1;
+  const int g_begin = min(ngroups, tid * gpt), g_end = min(ngroups, g_begin + gpt);
   uint32_t n_above = 0;
-  for (int chk = c0; chk < c1; ++chk) {
-    const int i0 = chk * 128 + 4 * lane;
-    const uint4 q = lds_key4(key_addr, i0);
+  for (int gi = 0; gi < gpt; ++gi) {           // same trip count in every lane: the warp vote below
+    const int g = g_begin + gi;
+    const bool in = g < g_end;
+    const uint4 q = in ? lds_key4(key_addr, 4 * g) : make_uint4(0u, 0u, 0u, 0u);
     const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
     bool any = false;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
-      const bool valid = i0 + j < n;
-      n_above += (valid && kv[j] > hi) ? 1u : 0u;
-      any |= valid && kv[j] >= lo && kv[j] <= hi;
+      n_above += kv[j] > hi ? 1u : 0u;
+      any |= kv[j] - lo <= hi - lo;            // lo <= key <= hi
     }
-    if (__any_sync(FULL, any)) {
+    if (__any_sync(FULL, any)) {               // rare: a boundary candidate
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (i0 + j < n && kv[j] >= lo && kv[j] <= hi) {
+        if (kv[j] - lo <= hi - lo) {
           const uint32_t slot = atomicAdd(&sh->ncand, 1u);
-          if (slot < (uint32_t)BIN_CAND_CAP) own[slot] = make_uint2(kv[j], (uint32_t)(i0 + j));
+          if (slot < (uint32_t)BIN_CAND_CAP) own[slot] = make_uint2(kv[j], (uint32_t)(4 * g + j));
         }
       }
     }
   }
+  cnt_t[tid] = n_above;
   n_above = __reduce_add_sync(FULL, n_above);
   if (lane == 0) sh->cnt_w[warp][0] = n_above;
   __syncthreads();
@@ -510,6 +520,7 @@ __device__ bool binned_select(KeyAt key_at, KeyAddr key_addr, int n, uint32_t k,
   for (int e = tid; e < m; e += blockDim.x) {
     const uint2 me = all[e];
     uint32_t ahead = 0;
+#pragma unroll 8
     for (int j = 0; j < m; ++j) {
       const uint2 o = all[j];
       ahead += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1u : 0u;
@@ -534,43 +545,46 @@ __device__ bool binned_select(KeyAt key_at, KeyAddr key_addr, int n, uint32_t k,
       const uint32_t i = all[off + e].y - g0;
       const uint32_t take = flag[off + e];
       asm volatile("st.shared.u32 [%0], %1;" ::"r"(key_addr((int)i)), "r"(take ? 0xffffffffu : 0u) : "memory");
-      if (take) atomicAdd(&sh->cnt_w[((int)i / 128) / per_warp][0], 1u);
+      if (take) atomicAdd(&cnt_t[((int)i / 4) / gpt], 1u);
+    }
+    if (tid == 0) {
+      uint32_t run = 0;
+      for (int c = 0; c < rank; ++c) run += sh->counts[c][0] + sh->selc[c];
+      sh->bin = run;                       // this CTA's first output position
     }
   }
   __syncthreads();
   sel_stamp(ts, 4);
-  if (tid == 0) {
-    uint32_t run = 0;
-    for (int c = 0; c < rank; ++c) run += sh->counts[c][0] + sh->selc[c];
-    for (int w = 0; w < nw; ++w) {
-      sh->off_w[w][0] = run;
-      run += sh->cnt_w[w][0];
-    }
-  }
+  // output positions: exclusive scan of the per-thread counts
+  const uint32_t mine_cnt = cnt_t[tid];
+  const uint32_t excl = block_exclusive_scan(mine_cnt, sh);
+  if (tid == (int)blockDim.x - 1) sh->total_in_bin = excl + mine_cnt;   // this CTA's count
   __syncthreads();
   sel_stamp(ts, 18);
-  // pass 2: emit keys > hi in index order (four per lane, warp-wide prefix)
-  uint32_t run = sh->off_w[warp][0];
-  for (int chk = c0; chk < c1; ++chk) {
-    const int i0 = chk * 128 + 4 * lane;
-    const uint4 q = lds_key4(key_addr, i0);
-    const bool t0 = i0 < n && q.x > hi, t1 = i0 + 1 < n && q.y > hi;
-    const bool t2 = i0 + 2 < n && q.z > hi, t3 = i0 + 3 < n && q.w > hi;
-    const uint32_t cnt = (uint32_t)t0 + (uint32_t)t1 + (uint32_t)t2 + (uint32_t)t3;
-    uint32_t incl = cnt;
+  // pass 2: each thread writes its keys > hi in index order
+  const uint32_t cta_base = sh->bin, cta_cnt = sh->total_in_bin;
+  const bool staged = cta_cnt <= stage_cap;
+  const int g0 = g0_of(rank);
+  uint32_t pos = excl;
+  if (mine_cnt > 0) {
+    for (int g = g_begin; g < g_end; ++g) {
+      const uint4 q = lds_key4(key_addr, 4 * g);
+      const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const uint32_t y = __shfl_up_sync(FULL, incl, o);
-      if (lane >= o) incl += y;
+      for (int j = 0; j < 4; ++j) {
+        if (kv[j] > hi) {
+          if (staged) stage[pos] = (uint32_t)(g0 + 4 * g + j);
+          else emit(cta_base + pos, 4 * g + j);
+          ++pos;
+        }
+      }
     }
-    uint32_t pos = run + incl - cnt;
-    if (t0) emit(pos++, i0);
-    if (t1) emit(pos++, i0 + 1);
-    if (t2) emit(pos++, i0 + 2);
-    if (t3) emit(pos, i0 + 3);
-    run += __shfl_sync(FULL, incl, 31);
   }
   __syncthreads();
+  if (staged) {
+    for (uint32_t e = tid; e < cta_cnt; e += blockDim.x)
+      if (cta_base + e < k) out[cta_base + e] = (int)stage[e];
+  }
   return true;
 }
 

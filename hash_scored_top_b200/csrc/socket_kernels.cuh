@@ -23,7 +23,8 @@ constexpr int SMEM_DYN_MAX = 232448;             // 227 KB opt-in per block
 __host__ __device__ constexpr int hist_words(int level) { return 1 << sel_bits(level); }
 constexpr int FUSED_THREADS = 1024;              // 32 warps: enough loads in flight to stream HBM
 constexpr int FUSED_WARPS = FUSED_THREADS / 32;
-constexpr int SCORE_PF = 2;                      // 32-key blocks in flight per warp
+constexpr int SCORE_PF = 2;                       // 32-key blocks in flight per warp
+constexpr uint32_t SCORE_L2_PREFETCH = 96u * 1024u;   // bytes of each CTA's key slice prefetched into L2
 constexpr int ATTEND_THREADS = 256;              // the attention kernel
 constexpr int ATTEND_WARPS = ATTEND_THREADS / 32;
 constexpr int ATTEND_BUFS = 2;                    // bf16: K/V slots per computing warp
@@ -276,6 +277,18 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
   cluster_arrive_relaxed();
   KeyIds<LP> buf[SCORE_PF];
   prefetch_blocks<LP, !HATA>(buf, ids_pair, norms_pair, blk0, nb);
+  if (warp == 1 && blk1 > blk0) {
+    // the first SCORE_L2_PREFETCH bytes of this CTA's slice stream into L2
+    // while the tables are built (more only delays the table's own loads)
+    constexpr uint32_t kChunk = 32768u;
+    const uint32_t slice = (uint32_t)(blk1 - blk0) * 32u;               // keys
+    const uint32_t want = min(slice, SCORE_L2_PREFETCH / (LP + 2u)) & ~31u;
+    const char* ids0 = reinterpret_cast<const char*>(ids_pair + (size_t)blk0 * 32 * LP);
+    const uint32_t ids_bytes = want * LP;
+    for (uint32_t off = (uint32_t)lane * kChunk; off < ids_bytes; off += 32u * kChunk)
+      prefetch_l2_bulk(ids0 + off, min(kChunk, ids_bytes - off));
+    if (!HATA && lane == 31 && want > 0) prefetch_l2_bulk(norms_pair + (size_t)blk0 * 32, want * 2u);
+  }
   if (tid == 0) sh->over_local = 0u;
   for (int i = tid; i < BIN_COUNT; i += blockDim.x) hist[0][i] = 0u;     // hist0 + hist1: the selection bins
   zero_table_padding_all<LP>(tab0, tab1, p.L, p.P);
@@ -298,11 +311,25 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
       for (int x = l - 32 * c; x < TABLE_COLS; x += S)
         for (int r = 0; r < C; ++r) st_cluster_f32(mapa(row + 4u * x, (uint32_t)r), v);
     };
+    // groups of 4 tables (4-aligned, inside one chunk): one 16-byte store per copy
+    auto store4 = [=](int bb, int l, const float* v, int cnt) {
+      if (cnt < 4) {
+        for (int q = 0; q < cnt; ++q) store(bb, l + q, v[q]);
+        return;
+      }
+      const int c = l >= 32 ? 1 : 0;
+      const int S = id_chunk_size(L, c);
+      const uint32_t row = (c ? t1a : t0a) + (uint32_t)bb * (TABLE_COLS * 4u);
+      for (int x = l - 32 * c; x < TABLE_COLS; x += S)
+        for (int r = 0; r < C; ++r) st_cluster_v4f32(mapa(row + 4u * x, (uint32_t)r), v);
+    };
     auto before_store = [] { cluster_wait(); };    // every CTA of the cluster has started
     void* scratch = sptr<void>(dyn, fs.base, fs.keysA);
     if (nl > 0) {
       if constexpr (HATA) build_hamming_table<D>(Qg, G, p.R, l0, nl, scratch, store, before_store);
-      else build_bucket_table<D>(Qg, G, p.R, p.P, p.tau, l0, nl, scratch, store, p.phase_ts, before_store);
+      else build_bucket_table<D, QT, decltype(store4), decltype(before_store), 4>(Qg, G, p.R, p.P, p.tau, l0, nl,
+                                                                                 scratch, store4, p.phase_ts,
+                                                                                 before_store);
     } else {
       cluster_wait();
     }
@@ -316,6 +343,12 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
   score_blocks<LP, !HATA>(buf, ids_pair, norms_pair, p.N, blk0, nb, fs.tbl0 + 4u * lane, fs.tbl1 + 4u * lane, keys,
                           hist[0], sh);
   stamp(p.phase_ts, 11);
+  // keys past the slice, up to its last 128-key chunk, read as 0
+  if (warp == 0) {
+    const int tail_end = (n_local + 127) & ~127;
+    for (int i = n_local + lane; i < tail_end; i += 32)
+      asm volatile("st.shared.u32 [%0], %1;" ::"r"(keys.addr((uint32_t)i)), "r"(0u) : "memory");
+  }
   __syncthreads();
   publish_coarse(hist[0], C, rank, sh);
   cluster_sync();     // every CTA's scores and histogram sums are final; the tables are no longer read
@@ -332,7 +365,8 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
     if (pos < (uint32_t)kk) idx_out[pos] = g0 + i;
   };
   const bool done = binned_select<HATA>(key_at, key_addr, n_local, (uint32_t)p.k, C, rank, g0_of, hist[0], sh, tab0u,
-                                       emit, p.phase_ts);
+                                       emit, idx_out, tab0u + bin_scratch_words(),
+                                       (uint32_t)(TABLE_BYTES / 4 - bin_scratch_words()), p.phase_ts);
   if (!done) {
     // exact radix select over the whole key range; every CTA has finished
     // reading the other CTAs' bins before any reuses its own

@@ -112,12 +112,15 @@ struct NoHook {
   __device__ void operator()() const {}
 };
 
-// Computes T_l(b) for the tables l in [l0, l0 + nl) and every bucket b < 2^P,
-// calling store(b, l, value_f32) once per entry. Qg points at the G query
-// rows of the pair (row stride D); scratch holds table_scratch_bytes. All
-// threads of the block must call this; it calls before_store() (all threads,
-// converged) just before the first store and ends with __syncthreads().
-template <int D, typename QT, typename Store, typename Hook = NoHook>
+// Computes T_l(b) for the tables l in [l0, l0 + nl) and every bucket b < 2^P.
+// VEC = 1: calls store(b, l, value_f32) once per entry. VEC = 4: calls
+// store(b, l, v, cnt) once per bucket and group of 4 tables l .. l + cnt - 1
+// (groups start at l0 + 4g; cnt < 4 only for the last group), v[0..cnt).
+// Qg points at the G query rows of the pair (row stride D); scratch holds
+// table_scratch_bytes. All threads of the block must call this; it calls
+// before_store() (all threads, converged) just before the first store and
+// ends with __syncthreads().
+template <int D, typename QT, typename Store, typename Hook = NoHook, int VEC = 1>
 __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_bfloat16* __restrict__ R, int P,
                                    float tau, int l0, int nl, void* scratch, Store store,
                                    unsigned long long* ts = nullptr, Hook before_store = Hook()) {
@@ -179,15 +182,37 @@ __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_
   // 4. table entries, summed over the group's heads
   before_store();
   const int nb = 1 << P;
-  for (int item = tid; item < nb * nl; item += nthr) {
-    const int li = item % nl;
-    const int b = item / nl;
-    double t = 0.0;
-    for (int h = 0; h < G; ++h) {
-      const int hl = h * nl + li;
-      t = fma(lo[hl * slo + (b & (nlo - 1))], hi[hl * shi + (b >> plo)], t);
+  if constexpr (VEC == 4) {
+    const int ng = (nl + 3) / 4;
+    for (int item = tid; item < nb * ng; item += nthr) {
+      const int g = item % ng;
+      const int b = item / ng;
+      const int cnt = min(4, nl - 4 * g);
+      float v[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q < cnt) {
+          double t = 0.0;
+          for (int h = 0; h < G; ++h) {
+            const int hl = h * nl + 4 * g + q;
+            t = fma(lo[hl * slo + (b & (nlo - 1))], hi[hl * shi + (b >> plo)], t);
+          }
+          v[q] = (float)t;
+        }
+      }
+      store(b, l0 + 4 * g, v, cnt);
     }
-    store(b, l0 + li, (float)t);
+  } else {
+    for (int item = tid; item < nb * nl; item += nthr) {
+      const int li = item % nl;
+      const int b = item / nl;
+      double t = 0.0;
+      for (int h = 0; h < G; ++h) {
+        const int hl = h * nl + li;
+        t = fma(lo[hl * slo + (b & (nlo - 1))], hi[hl * shi + (b >> plo)], t);
+      }
+      store(b, l0 + li, (float)t);
+    }
   }
   __syncthreads();
 }

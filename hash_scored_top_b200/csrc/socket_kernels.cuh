@@ -325,13 +325,13 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
     };
     auto before_store = [] { cluster_wait(); };    // every CTA of the cluster has started
     void* scratch = sptr<void>(dyn, fs.base, fs.keysA);
-    if (nl > 0) {
-      if constexpr (HATA) build_hamming_table<D>(Qg, G, p.R, l0, nl, scratch, store, before_store);
-      else build_bucket_table<D, QT, decltype(store4), decltype(before_store), 4>(Qg, G, p.R, p.P, p.tau, l0, nl,
-                                                                                 scratch, store4, p.phase_ts,
-                                                                                 before_store);
-    } else {
+    if (nl <= 0) {
       cluster_wait();
+    } else if constexpr (HATA) {
+      build_hamming_table<D>(Qg, G, p.R, l0, nl, scratch, store, before_store);
+    } else {
+      build_bucket_table<D, QT, decltype(store4), decltype(before_store), 4>(Qg, G, p.R, p.P, p.tau, l0, nl, scratch,
+                                                                            store4, p.phase_ts, before_store);
     }
   }
   stamp(p.phase_ts, 9);

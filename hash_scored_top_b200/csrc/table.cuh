@@ -79,6 +79,40 @@ __device__ __forceinline__ void project_rows(const double* qhat, int G, const __
   }
 }
 
+// The same projections on the fp64 tensor cores (mma m8n8k4, f64 in and
+// out): warp w computes 8x8 tiles z(h, mi) for 8 heads and 8 hyperplane rows,
+// accumulating over the head dimension in steps of 4 in a fixed order, so
+// every element's value depends only on its inputs. Calls out(item, z) once
+// per item h * nrows + mi (h < G, mi < nrows).
+__device__ __forceinline__ void mma_f64_m8n8k4(double& d0, double& d1, double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
+               : "+d"(d0), "+d"(d1) : "d"(a), "d"(b));
+}
+
+template <int D, typename Out>
+__device__ __forceinline__ void project_rows_mma(const double* qhat, int G, const __nv_bfloat16* rs, int nrows,
+                                                 Out out) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int mt = (G + 7) / 8, nt = (nrows + 7) / 8;
+  const int r = lane >> 2, c = lane & 3;     // fragment row; column within the k step
+  for (int task = warp; task < mt * nt; task += nw) {
+    const int hb = (task / nt) * 8, nb = (task % nt) * 8;
+    const int h = hb + r, n = nb + r;        // A row (head), B column (hyperplane row)
+    const bool hv = h < G, nv = n < nrows;
+    double d0 = 0.0, d1 = 0.0;
+#pragma unroll 8
+    for (int k0 = 0; k0 < D; k0 += 4) {
+      const double a = hv ? qhat[qpad_index<D>(h, k0 + c)] : 0.0;
+      const double b = nv ? (double)__bfloat162float(rs[n * D + k0 + c]) : 0.0;
+      mma_f64_m8n8k4(d0, d1, a, b);
+    }
+    // accumulator: row r, columns 2c and 2c + 1 of the tile
+    const int n0 = nb + 2 * c;
+    if (hv && n0 < nrows) out(h * nrows + n0, d0);
+    if (hv && n0 + 1 < nrows) out(h * nrows + n0 + 1, d1);
+  }
+}
+
 // Unit query rows (one warp per head) into qhat (padded rows, qpad_index),
 // float64. Each lane loads its D / 32 values once, then normalises them.
 template <int D, typename QT>
@@ -150,7 +184,7 @@ __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_
 
   // 2. projections z and the per-bit factors sigmoid(+-2z/tau)
   const double two_over_tau = 2.0 / (double)tau;
-  project_rows<D>(qhat, G, rs, nl * P, [&](int item, double z) {
+  project_rows_mma<D>(qhat, G, rs, nl * P, [&](int item, double z) {
     const double x = two_over_tau * z;                  // logit gap between bit=1 and bit=0
     const double e = exp(-fabs(x));
     const double p_big = 1.0 / (1.0 + e);               // sigmoid(|x|)

@@ -237,6 +237,11 @@ def run_ours(args, world, rank, local):
         api.socket_decode(c["Q"], c["K"], c["V"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k,
                           w.scale, O, None, ws)
 
+    def step(c):
+        # one decoder step: hash the current token (key N - 1), then decode over N keys
+        api.socket_decode_append(c["Q"], c["K"], c["V"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k,
+                                 w.scale, O, None, ws)
+
     # warm-up through the plain API (also sets the kernels' attributes)
     for i in range(args.warmup):
         c = caches[i % len(caches)]
@@ -252,8 +257,7 @@ def run_ours(args, world, rank, local):
     with torch.cuda.stream(side):
         with torch.cuda.graph(g_step, stream=side):
             for c in caches:
-                append(c)
-                decode(c)
+                step(c)
         with torch.cuda.graph(g_dec, stream=side):
             for c in caches:
                 decode(c)
@@ -329,7 +333,8 @@ def run_ours(args, world, rank, local):
         "config": {
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "L": w.L, "P": w.P,
             "tau": w.tau, "k": w.k, "kv_dtype": w.kv_dtype, "global_batch": w.B * world,
-            "step": "append 1 token (hash) + decode (tables, scores, exact top-k, sparse attention)",
+            "step": "socket_decode_append: hash 1 new token per pair, then decode (tables, scores, exact top-k, "
+                    "sparse attention)",
             "launch": f"CUDA graph of {per_graph} steps replayed {reps} times",
             "l2": f"inputs larger than L2: {args.caches} rotating caches x "
                   f"{(w.pairs * w.N * (w.L + 2)) / 1e6:.0f} MB of ids+norms", "parallelism": f"replicas x{world}",
@@ -379,9 +384,8 @@ def run_e2e(args, w, api, caches, device, world, ws):
         kv_dev.copy_(kv_host, non_blocking=True)
         c["K"][:, :, w.N - 1].copy_(kv_dev[0])
         c["V"][:, :, w.N - 1].copy_(kv_dev[1])
-        api.socket_hash_keys(c["K"], c["V"], c["R"], w.L, w.P, c["ids"], c["norms"], w.N - 1, 1)
-        api.socket_decode(q_dev, c["K"], c["V"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k,
-                          w.scale, O, None, ws)
+        api.socket_decode_append(q_dev, c["K"], c["V"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k,
+                                 w.scale, O, None, ws)
         o_host.copy_(O, non_blocking=True)
 
     for _ in range(3):

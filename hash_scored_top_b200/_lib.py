@@ -32,6 +32,8 @@ SIGNATURES = {
     "sk_noalloc_scratch_bytes": (_z, []),
     "socket_decode": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _f, _p, _p, _p, _z,
                            _p]),
+    "socket_decode_append": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _f, _p, _p, _p,
+                                  _z, _p]),
     "socket_select": (_i, [_p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _p, _p, _z, _p]),
     "hata_hash_keys": (_i, [_p, _i, _p, _i, _i, _i, _i, _i, _i, _p, _p]),
     "hata_decode": (_i, [_p, _p, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _z, _p]),

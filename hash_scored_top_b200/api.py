@@ -222,6 +222,26 @@ def socket_decode(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k:
     _check(rc, "socket_decode")
 
 
+def socket_decode_append(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k: int, scale: float, O,
+                         idx_out=None, ws=None):
+    """One decoder step: hash key N - 1 into (ids, norms), then the decode over N keys."""
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = K.shape
+    _want(K, Q.dtype, K.shape, "K")
+    _want(V, Q.dtype, K.shape, "V")
+    _want(R, torch.bfloat16, (L * P, d), "R")
+    _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
+    _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    if idx_out is not None:
+        _want(idx_out, torch.int32, (B, Hkv, k), "idx_out")
+    ws = _workspace(workspace_bytes(OP_DECODE, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    rc = _lib.lib.socket_decode_append(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R), _ptr(ids), _ptr(norms), B,
+                                       Hq, Hkv, Ncap, N, d, L, P, ctypes.c_float(tau), k, ctypes.c_float(scale),
+                                       _ptr(O), _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
+    _check(rc, "socket_decode_append")
+
+
 def socket_select(Q, R, ids, norms, N: int, L: int, P: int, tau: float, k: int, idx, ws=None):
     """SOCKET steps 2-4 without the attention: idx [B, Hkv, k] int32 ascending."""
     B, Hq, d = Q.shape

@@ -204,48 +204,52 @@ int max_cluster_size() {
   return cached;
 }
 
+// pdl: launch as the programmatic dependent of the previous kernel in the
+// stream (the kernel waits before reading what that kernel writes).
 template <typename Kern, typename Params>
-int launch_cluster(Kern kern, int grid, int C, size_t smem, cudaStream_t s, const Params& p) {
+int launch_cluster(Kern kern, int grid, int C, size_t smem, cudaStream_t s, const Params& p, bool pdl = false) {
   if (set_kernel_smem(kern, smem, C > 8) != cudaSuccess) return check_launch("cudaFuncSetAttribute");
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid, 1, 1);
   cfg.blockDim = dim3(FUSED_THREADS, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = C;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = pdl ? 2 : 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, p);
   if (e != cudaSuccess) return fail(SK_ERR_CUDA, "fused launch: %s", cudaGetErrorString(e));
   return check_launch("fused kernel");
 }
 
 template <int D, typename QT, bool HATA>
-int launch_select_t(const FusedParams& p, int pairs, cudaStream_t s) {
+int launch_select_t(const FusedParams& p, int pairs, bool pdl, cudaStream_t s) {
   const int grid = pairs * p.C;
   switch (ids_bytes_per_key(p.L)) {
-    case 16: return launch_cluster(socket_select_kernel<D, 16, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p);
-    case 32: return launch_cluster(socket_select_kernel<D, 32, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p);
-    case 48: return launch_cluster(socket_select_kernel<D, 48, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p);
-    default: return launch_cluster(socket_select_kernel<D, 64, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p);
+    case 16: return launch_cluster(socket_select_kernel<D, 16, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p, pdl);
+    case 32: return launch_cluster(socket_select_kernel<D, 32, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p, pdl);
+    case 48: return launch_cluster(socket_select_kernel<D, 48, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p, pdl);
+    default: return launch_cluster(socket_select_kernel<D, 64, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p, pdl);
   }
 }
 
-int launch_select(const FusedParams& p, int pairs, int d, sk_dtype q, bool hata, cudaStream_t s) {
+int launch_select(const FusedParams& p, int pairs, int d, sk_dtype q, bool hata, bool pdl, cudaStream_t s) {
   if (hata) {
-    if (d == 128) return q == SK_BF16 ? launch_select_t<128, __nv_bfloat16, true>(p, pairs, s)
-                                      : launch_select_t<128, float, true>(p, pairs, s);
-    return q == SK_BF16 ? launch_select_t<64, __nv_bfloat16, true>(p, pairs, s)
-                        : launch_select_t<64, float, true>(p, pairs, s);
+    if (d == 128) return q == SK_BF16 ? launch_select_t<128, __nv_bfloat16, true>(p, pairs, pdl, s)
+                                      : launch_select_t<128, float, true>(p, pairs, pdl, s);
+    return q == SK_BF16 ? launch_select_t<64, __nv_bfloat16, true>(p, pairs, pdl, s)
+                        : launch_select_t<64, float, true>(p, pairs, pdl, s);
   }
-  if (d == 128) return q == SK_BF16 ? launch_select_t<128, __nv_bfloat16, false>(p, pairs, s)
-                                    : launch_select_t<128, float, false>(p, pairs, s);
-  return q == SK_BF16 ? launch_select_t<64, __nv_bfloat16, false>(p, pairs, s)
-                      : launch_select_t<64, float, false>(p, pairs, s);
+  if (d == 128) return q == SK_BF16 ? launch_select_t<128, __nv_bfloat16, false>(p, pairs, pdl, s)
+                                    : launch_select_t<128, float, false>(p, pairs, pdl, s);
+  return q == SK_BF16 ? launch_select_t<64, __nv_bfloat16, false>(p, pairs, pdl, s)
+                      : launch_select_t<64, float, false>(p, pairs, pdl, s);
 }
 
 // ---------------------------------------------------------------- unfused pieces
@@ -708,7 +712,7 @@ namespace {
 int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, const void* ids,
                 const void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k,
                 float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, bool hata, bool attend,
-                cudaStream_t s) {
+                cudaStream_t s, bool after_append = false) {
   const int pairs = B * Hkv, G = Hq / Hkv;
   if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
   const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, hata, max_cluster_size());
@@ -762,7 +766,7 @@ int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const 
   p.chunk = fp.chunk;
   p.tau = tau;
   p.scale = scale;
-  SK_TRY(launch_select(p, pairs, d, kv, hata, s));
+  SK_TRY(launch_select(p, pairs, d, kv, hata, after_append, s));
   if (!attend) return SK_OK;
   return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, w, attend_ws_bytes(pairs, splits, G, d),
                        true, false, s);
@@ -793,6 +797,43 @@ int socket_decode(const void* Q, const void* K, const void* V, sk_dtype kv, cons
   if (k < 1 || k > N) return fail(SK_ERR_INVALID_ARG, "k=%d must be in [1, N=%d]", k, N);
   return decode_impl(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, scale, O, idx_out, ws, ws_bytes,
                      false, true, as_stream(stream));
+}
+
+int socket_decode_append(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, void* ids,
+                         void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k,
+                         float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  SK_NONNULL(Q);
+  SK_NONNULL(K);
+  SK_NONNULL(V);
+  SK_NONNULL(R);
+  SK_NONNULL(ids);
+  SK_NONNULL(norms);
+  SK_NONNULL(O);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(K, 16);
+  SK_ALIGNED(V, 16);
+  SK_ALIGNED(R, 16);
+  SK_ALIGNED(ids, 32);
+  SK_ALIGNED(norms, 2);
+  SK_TRY(check_dtype(kv));
+  SK_TRY(check_heads(B, Hq, Hkv, d));
+  SK_TRY(check_cache(Ncap, N));
+  SK_TRY(check_tables(L, P, tau));
+  if (L * P > 512) return fail(SK_ERR_UNSUPPORTED, "L*P=%d > 512", L * P);
+  if (k < 1 || k > N) return fail(SK_ERR_INVALID_ARG, "k=%d must be in [1, N=%d]", k, N);
+  // the workspace check comes before the first launch: a failure launches nothing
+  {
+    const int pairs = B * Hkv, G = Hq / Hkv;
+    if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
+    const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, false, max_cluster_size());
+    const size_t need = fp.C > 0 ? decode_ws_bytes(B, Hq, Hkv, k, d) : chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
+    if (ws == nullptr || ws_bytes < need)
+      return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
+  }
+  const cudaStream_t s = as_stream(stream);
+  SK_TRY(hash_launch(K, V, kv, R, B, Hkv, Ncap, N - 1, 1, d, L, P, ids, norms, s));
+  return decode_impl(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, scale, O, idx_out, ws, ws_bytes,
+                     false, true, s, true);
 }
 
 int socket_select(const void* Q, sk_dtype q, const void* R, const void* ids, const void* norms, int B, int Hq, int Hkv,

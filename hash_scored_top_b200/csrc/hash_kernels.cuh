@@ -114,6 +114,10 @@ template <typename KVT>
 __global__ void __launch_bounds__(512) hash_keys_append_kernel(const HashParams p) {
   __shared__ float ks[128];
   __shared__ uint32_t bits[16];       // 512 projection signs
+  // a selection kernel launched after this one as its programmatic dependent
+  // may start now: it waits (griddepcontrol.wait) before reading any bucket
+  // ID or norm, and reads nothing else this kernel writes
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int pair = blockIdx.x;
   const int key = p.n_begin + blockIdx.y;
   const int d = p.d, LP = p.L * p.P;

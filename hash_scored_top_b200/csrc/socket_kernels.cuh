@@ -272,11 +272,8 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
 
   // ---- setup. The cluster barrier is split: this arrive, and the wait just
   // before the first store into another CTA (the tables), so the barrier's
-  // latency hides behind the table build. The first key blocks are requested
-  // now; they arrive while the tables are built.
+  // latency hides behind the table build.
   cluster_arrive_relaxed();
-  KeyIds<LP> buf[SCORE_PF];
-  prefetch_blocks<LP, !HATA>(buf, ids_pair, norms_pair, blk0, nb);
   if (warp == 1 && blk1 > blk0) {
     // the first SCORE_L2_PREFETCH bytes of this CTA's slice stream into L2
     // while the tables are built (more only delays the table's own loads)
@@ -336,6 +333,12 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
   }
   stamp(p.phase_ts, 9);
   cluster_sync();     // every table entry has landed in every CTA
+  // Launched as the programmatic dependent of the key-append kernel, the
+  // kernel got here while that kernel may still run: the bucket IDs and norms
+  // are read only after it completed (a no-op for an ordinary launch).
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  KeyIds<LP> buf[SCORE_PF];
+  prefetch_blocks<LP, !HATA>(buf, ids_pair, norms_pair, blk0, nb);
   stamp(p.phase_ts, 1);
 
   // ---- SOCKET step 3: scores of this CTA's slice, kept on chip

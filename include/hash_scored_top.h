@@ -182,6 +182,22 @@ int socket_decode(const void* Q, const void* K, const void* V, sk_dtype kv, cons
                   void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * One decode step of a decoder loop: appends the current token (key N - 1,
+ * already written to K and V by the caller) to the hashed cache exactly like
+ * socket_hash_keys(..., n_begin = N - 1, n_count = 1, ...), then runs
+ * socket_decode over the N keys (results identical to those two calls). The
+ * selection kernel is launched as the programmatic dependent of the hashing
+ * kernel: its bucket-table build overlaps the hashing, and it reads bucket
+ * IDs and norms only after the hashing completed. ids and norms are updated
+ * in place (row N - 1). Requires L * P <= 512 and everything socket_decode
+ * requires. ws: sk_workspace_bytes(SK_OP_DECODE, ...) bytes.
+ */
+int socket_decode_append(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R,
+                         void* ids, void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L,
+                         int P, float tau, int k, float scale, float* O, int* idx_out, void* ws,
+                         size_t ws_bytes, void* stream);
+
+/*
  * Selection only, SOCKET steps 2-4 without the attention: the index list of
  * socket_decode (bucket tables, scores, exact top-k with ties to the lower
  * index), written ascending to idx [B][Hkv][k], for callers that run their

@@ -238,6 +238,29 @@ def test_select_only_matches_decode_and_oracle(api, name):
             assert pa.check_selection(s_ref, sel[b, h].cpu().numpy(), w.k) == [], (b, h)
 
 
+@pytest.mark.parametrize("name", ["llama8b_needles", "qwen_l48_g8", "tiny_f32"])
+def test_decode_append_equals_hash_then_decode(api, name):
+    """socket_decode_append = socket_hash_keys of key N - 1, then socket_decode."""
+    w = _w(name)
+    inp = wl.make_inputs(w, DEV)
+    Ncap = inp["K"].shape[2]
+    ids = api.empty_ids(w.B, w.Hkv, Ncap, w.L, DEV)
+    nrm = api.empty_norms(w.B, w.Hkv, Ncap, DEV)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, nrm, 0, w.N - 1)   # the cache before the step
+    ids2, nrm2 = ids.clone(), nrm.clone()
+    O1 = torch.empty(w.B, w.Hq, w.d, device=DEV)
+    idx1 = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=DEV)
+    api.socket_decode_append(inp["Q"], inp["K"], inp["V"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, w.k, w.scale,
+                             O1, idx1)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids2, nrm2, w.N - 1, 1)
+    O2 = torch.empty(w.B, w.Hq, w.d, device=DEV)
+    idx2 = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=DEV)
+    api.socket_decode(inp["Q"], inp["K"], inp["V"], inp["R"], ids2, nrm2, w.N, w.L, w.P, w.tau, w.k, w.scale, O2, idx2)
+    api.check_status()
+    assert torch.equal(ids, ids2) and torch.equal(nrm, nrm2)
+    assert torch.equal(idx1, idx2) and torch.equal(O1, O2)
+
+
 def test_fused_decode_is_deterministic(api):
     w = _w("llama8b_needles")
     inp = wl.make_inputs(w, DEV)

@@ -513,47 +513,56 @@ __device__ bool binned_select(KeyAt key_at, KeyAddr key_addr, int n, uint32_t k,
     while (c < C - 1 && e >= off + (int)sh->counts[c][1]) off += (int)sh->counts[c++][1];
     const uint2 v = *cluster.map_shared_rank(own + (e - off), (unsigned)c);
     all[e] = make_uint2(v.x, (uint32_t)g0_of(c) + v.y);
+    flag[e] = 0u;
   }
   __syncthreads();
   sel_stamp(ts, 20);
-  // exact order among the candidates: key descending, then index ascending
-  for (int e = tid; e < m; e += blockDim.x) {
-    const uint2 me = all[e];
-    uint32_t ahead = 0;
-#pragma unroll 8
-    for (int j = 0; j < m; ++j) {
-      const uint2 o = all[j];
-      ahead += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1u : 0u;
-    }
-    const uint32_t take = ahead < need ? 1u : 0u;
-    flag[e] = take;
-    if (take) {
-      int c = 0, off = 0;
-      while (c < C - 1 && e >= off + (int)sh->counts[c][1]) off += (int)sh->counts[c++][1];
-      atomicAdd(&sh->selc[c], 1u);
+  // exact order among the candidates (key descending, then index ascending):
+  // thread t counts, for candidate t % m, the candidates ahead of it among
+  // j = t / m, t / m + stride, ... (all threads share the m * m comparisons)
+  uint32_t* ahead_cnt = flag;                        // [m], zeroed by the gather
+  {
+    const int per = max(1, (int)blockDim.x / max(m, 1));   // threads per candidate
+    const int e = tid % max(m, 1), part = tid / max(m, 1);
+    if (m > 0 && part < per) {
+      const uint2 me = all[e];
+      uint32_t a = 0;
+      for (int j = part; j < m; j += per) {
+        const uint2 o = all[j];
+        a += (o.x > me.x || (o.x == me.x && o.y < me.y)) ? 1u : 0u;
+      }
+      if (a) atomicAdd(&ahead_cnt[e], a);
     }
   }
   __syncthreads();
   sel_stamp(ts, 21);
-  // this CTA's candidates: taken ones become all ones (> hi), the rest 0 (< lo)
+  // taken candidates of this CTA become all ones (> hi), the others 0 (< lo);
+  // selc[c]: candidates taken in CTA c
   {
     int off = 0;
     for (int c = 0; c < rank; ++c) off += (int)sh->counts[c][1];
     const int mine = (int)sh->counts[rank][1];
     const uint32_t g0 = (uint32_t)g0_of(rank);
-    for (int e = tid; e < mine; e += blockDim.x) {
-      const uint32_t i = all[off + e].y - g0;
-      const uint32_t take = flag[off + e];
-      asm volatile("st.shared.u32 [%0], %1;" ::"r"(key_addr((int)i)), "r"(take ? 0xffffffffu : 0u) : "memory");
-      if (take) atomicAdd(&cnt_t[((int)i / 4) / gpt], 1u);
-    }
-    if (tid == 0) {
-      uint32_t run = 0;
-      for (int c = 0; c < rank; ++c) run += sh->counts[c][0] + sh->selc[c];
-      sh->bin = run;                       // this CTA's first output position
+    for (int e = tid; e < m; e += blockDim.x) {
+      const bool take = ahead_cnt[e] < need;
+      if (take) {
+        int c = 0, o = 0;
+        while (c < C - 1 && e >= o + (int)sh->counts[c][1]) o += (int)sh->counts[c++][1];
+        atomicAdd(&sh->selc[c], 1u);
+      }
+      if (e >= off && e < off + mine) {
+        const uint32_t i = all[e].y - g0;
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(key_addr((int)i)), "r"(take ? 0xffffffffu : 0u) : "memory");
+        if (take) atomicAdd(&cnt_t[((int)i / 4) / gpt], 1u);
+      }
     }
   }
   __syncthreads();
+  if (tid == 0) {                                   // read after the scan's barriers
+    uint32_t run = 0;
+    for (int c = 0; c < rank; ++c) run += sh->counts[c][0] + sh->selc[c];
+    sh->bin = run;                                   // this CTA's first output position
+  }
   sel_stamp(ts, 4);
   // output positions: exclusive scan of the per-thread counts
   const uint32_t mine_cnt = cnt_t[tid];

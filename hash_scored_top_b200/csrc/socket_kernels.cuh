@@ -23,7 +23,10 @@ constexpr int SMEM_DYN_MAX = 232448;             // 227 KB opt-in per block
 __host__ __device__ constexpr int hist_words(int level) { return 1 << sel_bits(level); }
 constexpr int FUSED_THREADS = 1024;              // 32 warps: enough loads in flight to stream HBM
 constexpr int FUSED_WARPS = FUSED_THREADS / 32;
-constexpr int SCORE_PF = 2;                       // 32-key blocks in flight per warp
+// 32-key blocks in flight per warp while scoring (a third one measured no
+// faster at 32-byte rows and spills at longer ones: registers are capped at 64)
+template <int LP>
+__host__ __device__ constexpr int score_pf() { return 2; }
 constexpr uint32_t SCORE_L2_PREFETCH = 96u * 1024u;   // bytes of each CTA's key slice prefetched into L2
 constexpr int ATTEND_THREADS = 256;              // the attention kernel
 constexpr int ATTEND_WARPS = ATTEND_THREADS / 32;
@@ -129,21 +132,21 @@ __device__ __forceinline__ void zero_table_padding_all(float* t0, float* t1, int
 
 // Scores keys of blocks blk0 + warp + i * NW (i < nb) into sort keys in
 // shared memory and counts them into the CTA's selection histogram. buf holds
-// the first SCORE_PF blocks, already requested.
+// the first score_pf<LP>() blocks, already requested.
 template <int LP, bool NORM>
-__device__ __forceinline__ void score_blocks(KeyIds<LP> (&buf)[SCORE_PF], const uint8_t* __restrict__ ids_pair,
+__device__ __forceinline__ void score_blocks(KeyIds<LP> (&buf)[score_pf<LP>()], const uint8_t* __restrict__ ids_pair,
                                              const __half* __restrict__ norms_pair, int N, int blk0, int nb,
                                              uint32_t col0, uint32_t col1, const FusedKeys keys, uint32_t* hist,
                                              SelShared* sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int it = 0; it < nb; it += SCORE_PF) {
+  for (int it = 0; it < nb; it += score_pf<LP>()) {
 #pragma unroll
-    for (int u = 0; u < SCORE_PF; ++u) {
+    for (int u = 0; u < score_pf<LP>(); ++u) {
       const int i = it + u;
       if (i < nb) {
         const KeyIds<LP> cur = buf[u];
-        if (i + SCORE_PF < nb) {
-          const int key = (blk0 + warp + (i + SCORE_PF) * nw) * 32 + lane;
+        if (i + score_pf<LP>() < nb) {
+          const int key = (blk0 + warp + (i + score_pf<LP>()) * nw) * 32 + lane;
           load_key_ids<LP, NORM>(buf[u], ids_pair + (size_t)key * LP, norms_pair + key);
         }
         const float s = score_key<LP, NORM>(cur, col0, col1);
@@ -161,11 +164,11 @@ __device__ __forceinline__ void score_blocks(KeyIds<LP> (&buf)[SCORE_PF], const 
 }
 
 template <int LP, bool NORM>
-__device__ __forceinline__ void prefetch_blocks(KeyIds<LP> (&buf)[SCORE_PF], const uint8_t* __restrict__ ids_pair,
+__device__ __forceinline__ void prefetch_blocks(KeyIds<LP> (&buf)[score_pf<LP>()], const uint8_t* __restrict__ ids_pair,
                                                 const __half* __restrict__ norms_pair, int blk0, int nb) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
 #pragma unroll
-  for (int u = 0; u < SCORE_PF; ++u) {
+  for (int u = 0; u < score_pf<LP>(); ++u) {
     if (u < nb) {
       const int key = (blk0 + warp + u * nw) * 32 + lane;
       load_key_ids<LP, NORM>(buf[u], ids_pair + (size_t)key * LP, norms_pair + key);
@@ -337,7 +340,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
   // kernel got here while that kernel may still run: the bucket IDs and norms
   // are read only after it completed (a no-op for an ordinary launch).
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  KeyIds<LP> buf[SCORE_PF];
+  KeyIds<LP> buf[score_pf<LP>()];
   prefetch_blocks<LP, !HATA>(buf, ids_pair, norms_pair, blk0, nb);
   stamp(p.phase_ts, 1);
 

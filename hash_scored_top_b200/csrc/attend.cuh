@@ -206,29 +206,28 @@ __device__ __forceinline__ void mma_attend_slot(MmaAttendState<D>& st, uint32_t 
 
 // Per-warp partial results in shared memory, one slot per warp:
 //   pm[w][h], pl[w][h] (max in log2 domain, sum), po[w][h][D] (unnormalised).
+// Per-warp partial results (m[G], l[G], o[G][D]); warp w's lies at
+// base + w * ws floats (inside that warp's own K/V slot, free once the warp
+// has finished its keys).
 struct PartialView {
-  float* pm;
-  float* pl;
-  float* po;
+  float* base;
+  int ws;
   int G;
   int D;
+  __device__ __forceinline__ float& m(int w, int h) const { return base[(size_t)w * ws + h]; }
+  __device__ __forceinline__ float& l(int w, int h) const { return base[(size_t)w * ws + G + h]; }
+  __device__ __forceinline__ float* o(int w, int h) const { return base + (size_t)w * ws + 2 * G + (size_t)h * D; }
 };
 
-__host__ __device__ inline size_t partial_bytes(int nslots, int G, int D) {
-  return (size_t)(2 * nslots * G + nslots * G * D + 2 * G + G * D) * sizeof(float);
-}
+// Floats of one warp's partial.
+__host__ __device__ inline size_t partial_floats(int G, int D) { return (size_t)G * (D + 2); }
 
-__device__ __forceinline__ PartialView partial_view(float* base, int nslots, int G, int D, float*& cM, float*& cL,
-                                                    float*& cO) {
+__device__ __forceinline__ PartialView partial_view(float* base, int ws, int G, int D) {
   PartialView pv;
+  pv.base = base;
+  pv.ws = ws;
   pv.G = G;
   pv.D = D;
-  pv.pm = base;
-  pv.pl = pv.pm + nslots * G;
-  pv.po = pv.pl + nslots * G;
-  cM = pv.po + (size_t)nslots * G * D;
-  cL = cM + G;
-  cO = cL + G;
   return pv;
 }
 
@@ -263,10 +262,10 @@ __device__ __forceinline__ void store_mma_partial(MmaAttendState<D>& st, const P
       const int h = hbase + i;
       if (h < pv.G) {
         if (r == 0) {
-          pv.pm[w * pv.G + h] = st.m[i];
-          pv.pl[w * pv.G + h] = l[i];
+          pv.m(w, h) = st.m[i];
+          pv.l(w, h) = l[i];
         }
-        float* po = pv.po + ((size_t)w * pv.G + h) * D;
+        float* po = pv.o(w, h);
 #pragma unroll
         for (int j = 0; j < D / 16; ++j) {
           po[16 * j + r] = st.acc[j][i];
@@ -280,8 +279,8 @@ __device__ __forceinline__ void store_mma_partial(MmaAttendState<D>& st, const P
 // Marks partial slot w as empty (no keys) for every head.
 __device__ __forceinline__ void store_empty_partial(const PartialView& pv, int w, int lane) {
   for (int h = lane; h < pv.G; h += 32) {
-    pv.pm[w * pv.G + h] = -INFINITY;
-    pv.pl[w * pv.G + h] = 0.f;
+    pv.m(w, h) = -INFINITY;
+    pv.l(w, h) = 0.f;
   }
 }
 
@@ -386,11 +385,11 @@ __device__ void attend_keys_f32(const float* __restrict__ Qg, const float* __res
   }
   for (int hh = 0; hh < G; ++hh) {
     if (lane == 0) {
-      pv.pm[warp * G + hh] = hh == h ? m : -INFINITY;
-      pv.pl[warp * G + hh] = hh == h ? l : 0.f;
+      pv.m(warp, hh) = hh == h ? m : -INFINITY;
+      pv.l(warp, hh) = hh == h ? l : 0.f;
     }
   }
-  float* po = pv.po + ((size_t)warp * G + h) * D;
+  float* po = pv.o(warp, h);
 #pragma unroll
   for (int i = 0; i < D / 32; ++i) po[lane + 32 * i] = acc[i];
 }
@@ -402,11 +401,11 @@ __device__ __forceinline__ void merge_partials(const PartialView& pv, int nslots
   const int G = pv.G, D = pv.D;
   for (int h = threadIdx.x; h < G; h += blockDim.x) {
     float mm = -INFINITY;
-    for (int w = 0; w < nslots; ++w) mm = fmaxf(mm, pv.pm[w * G + h]);
+    for (int w = 0; w < nslots; ++w) mm = fmaxf(mm, pv.m(w, h));
     float ls = 0.f;
     for (int w = 0; w < nslots; ++w) {
-      const float pm = pv.pm[w * G + h];
-      if (pm != -INFINITY) ls += exp2f(pm - mm) * pv.pl[w * G + h];
+      const float pm = pv.m(w, h);
+      if (pm != -INFINITY) ls += exp2f(pm - mm) * pv.l(w, h);
     }
     M[h] = mm;
     Lsum[h] = ls;
@@ -417,8 +416,8 @@ __device__ __forceinline__ void merge_partials(const PartialView& pv, int nslots
     const float mm = M[h];
     float o = 0.f;
     for (int w = 0; w < nslots; ++w) {
-      const float pm = pv.pm[w * G + h];
-      if (pm != -INFINITY) o += exp2f(pm - mm) * pv.po[((size_t)w * G + h) * D + (e % D)];
+      const float pm = pv.m(w, h);
+      if (pm != -INFINITY) o += exp2f(pm - mm) * pv.o(w, h)[e % D];
     }
     O[e] = o;
   }

@@ -31,7 +31,9 @@ constexpr uint32_t SCORE_L2_PREFETCH = 96u * 1024u;   // bytes of each CTA's key
 constexpr int ATTEND_THREADS = 256;              // the attention kernel
 constexpr int ATTEND_WARPS = ATTEND_THREADS / 32;
 constexpr int ATTEND_BUFS = 2;                    // bf16: K/V slots per computing warp
-constexpr int ATTEND_MMA_WARPS = ATTEND_WARPS / ATTEND_BUFS;   // bf16: computing warps
+constexpr int ATTEND_MMA_WARPS = 6;               // bf16: computing warps
+constexpr int ATTEND_SLOTS = ATTEND_MMA_WARPS * ATTEND_BUFS > ATTEND_WARPS ? ATTEND_MMA_WARPS * ATTEND_BUFS
+                                                                           : ATTEND_WARPS;
 constexpr int ATTEND_MAX_SPLITS = 128;           // one head's partials fit in the warp slots
 
 __device__ __forceinline__ uint32_t key_of(float s) { return __float_as_uint(s); }
@@ -39,7 +41,7 @@ __device__ __forceinline__ uint32_t key_of(float s) { return __float_as_uint(s);
 static_assert(bin_scratch_words() * 4 <= TABLE_BYTES, "the selection scratch lives in the first table");
 static_assert(hist_words(0) + hist_words(1) >= BIN_COUNT, "the selection bins live in the first two radix histograms");
 static_assert(FUSED_THREADS * 4 == BIN_COUNT, "publish_coarse reads four bins per thread");
-static_assert(ATTEND_MMA_WARPS * ATTEND_BUFS == ATTEND_WARPS, "the bf16 slots are the warp slots, regrouped");
+static_assert(ATTEND_MMA_WARPS <= ATTEND_WARPS && ATTEND_SLOTS <= 32, "one mbarrier and phase word per slot");
 
 __host__ __device__ constexpr int table_chunks(int LP) { return LP > 32 ? 2 : 1; }
 
@@ -177,16 +179,18 @@ __device__ __forceinline__ void prefetch_blocks(KeyIds<LP> (&buf)[score_pf<LP>()
 }
 
 // Shared-memory plan of the attention stage: query stage, one mbarrier and
-// phase word per warp slot, warp slots, per-warp partials.
+// phase word per slot, K/V slots (computing warp w owns slots w * nbuf ..;
+// its partial goes into its first slot once its keys are done), the CTA's
+// merged result.
 struct AttendSmem {
   uint32_t qs;             // query rows (bf16 path)
   uint32_t mbar0;          // 8 bytes per slot
   uint32_t phases;         // 4 bytes per slot
-  uint32_t slot0;          // warp w's slot: slot0 + w * slot_stride
+  uint32_t slot0;          // slot s: slot0 + s * slot_stride
   uint32_t slot_stride;
   int ncw;                 // computing warps (one partial each)
-  int nbuf;                // slots per computing warp (bf16)
-  uint32_t partials;
+  int nbuf;                // slots per computing warp
+  uint32_t result;         // merged (M[G], L[G], O[G][D])
 };
 
 // Exact attention of cnt keys (keys(i), i < cnt) into merged per-CTA results
@@ -197,7 +201,10 @@ __device__ __forceinline__ void attend_and_merge(unsigned char* dyn, uint32_t ba
                                                  const KVT* Qg, const KVT* Kp, const KVT* Vp, int G, float scale,
                                                  KeyFn keys, int cnt, int nrows, float*& cM, float*& cL, float*& cO) {
   const int ncw = as.ncw;
-  const PartialView pv = partial_view(sptr<float>(dyn, base, as.partials), ncw, G, D, cM, cL, cO);
+  const PartialView pv = partial_view(sptr<float>(dyn, base, as.slot0), (int)(as.nbuf * as.slot_stride / 4u), G, D);
+  cM = sptr<float>(dyn, base, as.result);
+  cL = cM + G;
+  cO = cL + G;
   if constexpr (sizeof(KVT) == 2) {
     attend_tiles_bf16<D, ATTEND_BUFS>(reinterpret_cast<const __nv_bfloat16*>(Kp),
                                       reinterpret_cast<const __nv_bfloat16*>(Vp), keys, cnt, nrows, G, scale, as.qs,
@@ -548,8 +555,8 @@ __device__ __forceinline__ void attend_stamp(unsigned long long* ts, int phase) 
 // warp slots, partials, the CTA's index list, a flag word.
 template <int D>
 __host__ __device__ inline size_t attend_smem_bytes(int G, int keys_per_split) {
-  return q_stage_bytes<D>() + 8 * 32 + 4 * 32 + (size_t)ATTEND_WARPS * kv_slot_bytes<D>() +
-         partial_bytes(ATTEND_WARPS, G, D) + (((size_t)keys_per_split * 4 + 15) & ~(size_t)15) + 16;
+  return q_stage_bytes<D>() + 8 * 32 + 4 * 32 + (size_t)ATTEND_SLOTS * kv_slot_bytes<D>() +
+         ((partial_floats(G, D) * 4 + 15) & ~(size_t)15) + (((size_t)keys_per_split * 4 + 15) & ~(size_t)15) + 16;
 }
 
 // Exact attention over a key list, split over keys: grid = (pairs, splits).
@@ -582,14 +589,15 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
     as.phases = a;   a += 4u * 32u;
     as.slot0 = a;
     as.slot_stride = kv_slot_bytes<D>();
-    a += ATTEND_WARPS * kv_slot_bytes<D>();
+    a += ATTEND_SLOTS * kv_slot_bytes<D>();
     as.ncw = sizeof(KVT) == 2 ? ATTEND_MMA_WARPS : ATTEND_WARPS;
-    as.nbuf = ATTEND_BUFS;
-    as.partials = a;
+    as.nbuf = sizeof(KVT) == 2 ? ATTEND_BUFS : 1;
+    as.result = a;
+    a += (uint32_t)((partial_floats(G, D) * 4 + 15) & ~(size_t)15);
   }
   const size_t smem_total = attend_smem_bytes<D>(G, p.idx ? p.keys_per_split : 0);
   uint32_t* last_flag = reinterpret_cast<uint32_t*>(dyn + (smem_total - 16));
-  int* list_s = reinterpret_cast<int*>(dyn + (as.partials - base) + partial_bytes(ATTEND_WARPS, G, D));
+  int* list_s = reinterpret_cast<int*>(dyn + (as.result - base) + ((partial_floats(G, D) * 4 + 15) & ~(size_t)15));
   attend_setup<D, KVT>(dyn, base, as, Qg, G);
   attend_stamp(p.phase_ts, 1);
   asm volatile("griddepcontrol.wait;" ::: "memory");   // the key list is complete from here on

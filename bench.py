@@ -54,14 +54,17 @@ def parse_args():
 # ---------------------------------------------------------------- helpers
 def required_bytes(w) -> dict:
     """Algorithmic bytes of one fused decode launch and of one whole step."""
-    lp = 16 if w.L <= 16 else 32 if w.L <= 32 else 48 if w.L <= 48 else 64    # ID bytes per key
+    if w.hata:
+        lp, nb, r_bytes = 16, 0, 128 * w.d * 2                                  # 128-bit codes, no norms
+    else:
+        lp = 16 if w.L <= 16 else 32 if w.L <= 32 else 48 if w.L <= 48 else 64    # ID bytes per key
+        nb, r_bytes = 2, w.L * w.P * w.d * 2
     q_bytes = w.B * w.Hq * w.d * 2
     o_bytes = w.B * w.Hq * w.d * 4
-    r_bytes = w.L * w.P * w.d * 2
-    select = w.pairs * (w.N * lp + 2 * w.N + w.k * 4) + q_bytes + r_bytes     # ids + f16 norms in, index list out
+    select = w.pairs * (w.N * (lp + nb) + w.k * 4) + q_bytes + r_bytes        # ids (+ f16 norms) in, index list out
     attend = w.pairs * w.k * (2 * w.d * 2 + 4) + q_bytes + o_bytes           # index list + K/V rows in, O out
     decode = select + attend - w.pairs * w.k * 4 - q_bytes                   # the index list stays in L2
-    append = w.pairs * (2 * w.d * 2 + lp + 2) + r_bytes                      # new K/V row read, ids + norm written
+    append = w.pairs * (2 * w.d * 2 + lp + nb) + r_bytes                     # new K/V row read, ids + norm written
     return {"select": select, "attend": attend, "decode": decode, "step": decode + append,
             "dense": w.pairs * w.N * 2 * w.d * 2 + q_bytes + o_bytes}
 
@@ -201,10 +204,15 @@ def build_caches(w, api, wl, n_caches, device, rank=0):
         wc = dataclasses.replace(w, seed=cache_seed(w, c, rank))
         inp = wl.make_inputs(wc, device)
         Ncap = inp["K"].shape[2]
-        ids = api.empty_ids(w.B, w.Hkv, Ncap, w.L, device)
-        norms = api.empty_norms(w.B, w.Hkv, Ncap, device)
-        api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, norms, 0, w.N - 1)
-        caches.append({"Q": inp["Q"], "K": inp["K"], "V": inp["V"], "R": inp["R"], "ids": ids, "norms": norms})
+        if w.hata:
+            codes = api.empty_codes(w.B, w.Hkv, Ncap, device)
+            api.hata_hash_keys(inp["K"], inp["R128"], codes, 0, w.N - 1)
+            caches.append({"Q": inp["Q"], "K": inp["K"], "V": inp["V"], "R": inp["R128"], "ids": codes})
+        else:
+            ids = api.empty_ids(w.B, w.Hkv, Ncap, w.L, device)
+            norms = api.empty_norms(w.B, w.Hkv, Ncap, device)
+            api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, norms, 0, w.N - 1)
+            caches.append({"Q": inp["Q"], "K": inp["K"], "V": inp["V"], "R": inp["R"], "ids": ids, "norms": norms})
         torch.cuda.synchronize()
     return caches
 
@@ -219,28 +227,42 @@ def run_ours(args, world, rank, local):
     dist_barrier(world)
     w = wl.WORKLOADS[args.workload]
     device = torch.device("cuda", local)
-    caches = build_caches(w, api, wl, args.caches, device, rank)
+    # one cache already streams more than L2 per step for the hard-hash workload (17 GB of K/V each)
+    n_caches = 1 if w.hata else args.caches
+    caches = build_caches(w, api, wl, n_caches, device, rank)
     Ncap = caches[0]["K"].shape[2]
     O = torch.empty(w.B, w.Hq, w.d, device=device)
-    ws = torch.empty(api.workspace_bytes(api.OP_DECODE, w.B, w.Hq, w.Hkv, Ncap, w.N, w.d, w.L, w.P, w.k),
+    op = api.OP_HATA_DECODE if w.hata else api.OP_DECODE
+    ws = torch.empty(api.workspace_bytes(op, w.B, w.Hq, w.Hkv, Ncap, w.N, w.d, w.L, w.P, w.k),
                      dtype=torch.uint8, device=device)
 
     def append(c):
-        api.socket_hash_keys(c["K"], c["V"], c["R"], w.L, w.P, c["ids"], c["norms"], w.N - 1, 1)
+        if w.hata:
+            api.hata_hash_keys(c["K"], c["R"], c["ids"], w.N - 1, 1)
+        else:
+            api.socket_hash_keys(c["K"], c["V"], c["R"], w.L, w.P, c["ids"], c["norms"], w.N - 1, 1)
 
     idx_sel = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=device)
 
     def select(c):
-        api.socket_select(c["Q"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k, idx_sel)
+        if not w.hata:
+            api.socket_select(c["Q"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k, idx_sel)
 
     def decode(c):
-        api.socket_decode(c["Q"], c["K"], c["V"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k,
-                          w.scale, O, None, ws)
+        if w.hata:
+            api.hata_decode(c["Q"], c["K"], c["V"], c["R"], c["ids"], w.N, w.k, w.scale, O, None, ws)
+        else:
+            api.socket_decode(c["Q"], c["K"], c["V"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k,
+                              w.scale, O, None, ws)
 
     def step(c):
         # one decoder step: hash the current token (key N - 1), then decode over N keys
-        api.socket_decode_append(c["Q"], c["K"], c["V"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k,
-                                 w.scale, O, None, ws)
+        if w.hata:
+            append(c)
+            decode(c)
+        else:
+            api.socket_decode_append(c["Q"], c["K"], c["V"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau,
+                                     w.k, w.scale, O, None, ws)
 
     # warm-up through the plain API (also sets the kernels' attributes)
     for i in range(args.warmup):
@@ -261,16 +283,18 @@ def run_ours(args, world, rank, local):
         with torch.cuda.graph(g_dec, stream=side):
             for c in caches:
                 decode(c)
-        with torch.cuda.graph(g_sel, stream=side):
-            for c in caches:
-                select(c)
+        if not w.hata:
+            with torch.cuda.graph(g_sel, stream=side):
+                for c in caches:
+                    select(c)
     torch.cuda.synchronize()
     reps = max(1, args.steps // per_graph)
     steps = reps * per_graph
     for _ in range(3):
         g_step.replay()
         g_dec.replay()
-        g_sel.replay()
+        if not w.hata:
+            g_sel.replay()
     torch.cuda.synchronize()
 
     # ---- timed region: `steps` steps back to back
@@ -307,16 +331,21 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize()
     decode_us = dist_max(world, d0.elapsed_time(d1) * 1e3 / steps)
     # the selection kernel alone (the dominant kernel of the step)
-    d0.record(stream)
-    for _ in range(reps):
-        g_sel.replay()
-    d1.record(stream)
-    torch.cuda.synchronize()
-    select_us = dist_max(world, d0.elapsed_time(d1) * 1e3 / steps)
+    select_us = None
+    if not w.hata:
+        d0.record(stream)
+        for _ in range(reps):
+            g_sel.replay()
+        d1.record(stream)
+        torch.cuda.synchronize()
+        select_us = dist_max(world, d0.elapsed_time(d1) * 1e3 / steps)
 
     rb = required_bytes(w)
     peak, peak_kind = load_peaks()
-    achieved = rb["select"] / (select_us * 1e-6) / 1e9
+    # the hard-hash workload has no selection-only entry point: its roofline
+    # unit is the decode launch pair
+    roof_us, roof_bytes = (decode_us, rb["decode"]) if w.hata else (select_us, rb["select"])
+    achieved = roof_bytes / (roof_us * 1e-6) / 1e9
     result = {
         "metric": METRIC,
         "value": weak_value(world, steps, elapsed_ms),
@@ -333,20 +362,23 @@ def run_ours(args, world, rank, local):
         "config": {
             "workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "L": w.L, "P": w.P,
             "tau": w.tau, "k": w.k, "kv_dtype": w.kv_dtype, "global_batch": w.B * world,
-            "step": "socket_decode_append: hash 1 new token per pair, then decode (tables, scores, exact top-k, "
-                    "sparse attention)",
+            "step": ("hata_hash_keys of 1 new token per pair, then hata_decode (codes, Hamming scores, exact "
+                     "top-k, sparse attention)") if w.hata else
+                    ("socket_decode_append: hash 1 new token per pair, then decode (tables, scores, exact top-k, "
+                     "sparse attention)"),
             "launch": f"CUDA graph of {per_graph} steps replayed {reps} times",
-            "l2": f"inputs larger than L2: {args.caches} rotating caches x "
-                  f"{(w.pairs * w.N * (w.L + 2)) / 1e6:.0f} MB of ids+norms", "parallelism": f"replicas x{world}",
+            "l2": f"inputs larger than L2: {n_caches} rotating caches x "
+                  f"{rb['select'] / 1e6:.0f} MB of hashed keys per step",
+            "parallelism": f"replicas x{world}",
         },
         "keys_scored_per_s": world * steps * w.pairs * w.N / (elapsed_ms * 1e-3),
         "required_bytes_per_step": rb["step"],
         "hbm_gbs_required": world * rb["step"] * steps / (elapsed_ms * 1e-3) / 1e9,
         "roofline": {
-            "kernel": "socket_select_kernel",
+            "kernel": "socket_select_kernel + socket_attend_kernel (hard hash)" if w.hata else "socket_select_kernel",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-            "peak_kind": peak_kind, "traffic": profiled_traffic(w.name),
-            "bytes_per_launch": rb["select"], "avg_launch_us": select_us,
+            "peak_kind": peak_kind, "traffic": None if w.hata else profiled_traffic(w.name),
+            "bytes_per_launch": roof_bytes, "avg_launch_us": roof_us,
         },
         "decode_kernels": {
             "kernels": "socket_select_kernel -> socket_attend_kernel (programmatic dependent launch)",
@@ -356,7 +388,7 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 3 * steps,
         "clocks": clocks,
     }
-    if not args.no_extras:
+    if not args.no_extras and not w.hata:
         result["e2e"] = run_e2e(args, w, api, caches, device, world, ws)
         result["dense_decode"] = run_dense(w, api, caches, device, rb, peak)
         if rank == 0 and world == 1:
@@ -469,6 +501,7 @@ def run_reference(args):
     import torch
     from threadpoolctl import threadpool_limits
     from hash_scored_top_b200 import workloads as wl
+    from oracle import hata_ref as ho
     from oracle import socket_ref as so
 
     w = wl.WORKLOADS[args.workload]
@@ -476,24 +509,32 @@ def run_reference(args):
     Qg = inp["Q"][0].double().numpy()
     K = inp["K"][0, 0, : w.N].double().numpy()
     V = inp["V"][0, 0, : w.N].double().numpy()
-    R = inp["R"].double().numpy()
-    ids, _ = so.hash_key_ids(K, R, w.L, w.P)
-    norms = so.value_norms_f16(V)
+    R = inp["R128" if w.hata else "R"].double().numpy()
+    if w.hata:
+        codes, _ = ho.binary_codes(K, R)
+
+        def decode(n, kk):
+            ho.hata_decode_pair(Qg, K[:n], V[:n], R, codes[:n], kk, w.scale)
+    else:
+        ids, _ = so.hash_key_ids(K, R, w.L, w.P)
+        norms = so.value_norms_f16(V)
+
+        def decode(n, kk):
+            so.socket_decode_pair(Qg, K[:n], V[:n], R, ids[:n], norms[:n], w.L, w.P, w.tau, kk, w.scale)
     # size the per-step sample so that warmup + steps fit in about two minutes
     budget = 120.0 / max(1, args.steps + args.warmup)
     with threadpool_limits(1):
         n_try = min(w.N, 8192)
         t0 = time.perf_counter()
-        so.socket_decode_pair(Qg, K[:n_try], V[:n_try], R, ids[:n_try], norms[:n_try], w.L, w.P, w.tau,
-                              max(1, w.k * n_try // w.N), w.scale)
+        decode(n_try, max(1, w.k * n_try // w.N))
         per_key = (time.perf_counter() - t0) / n_try
         n = int(min(w.N, max(256, budget / per_key)))
         kk = max(1, w.k * n // w.N)
         for _ in range(args.warmup):
-            so.socket_decode_pair(Qg, K[:n], V[:n], R, ids[:n], norms[:n], w.L, w.P, w.tau, kk, w.scale)
+            decode(n, kk)
         t0 = time.perf_counter()
         for _ in range(args.steps):
-            so.socket_decode_pair(Qg, K[:n], V[:n], R, ids[:n], norms[:n], w.L, w.P, w.tau, kk, w.scale)
+            decode(n, kk)
         dt = time.perf_counter() - t0
     scale = (w.pairs * w.N) / n                      # sample keys -> one whole step
     value = args.steps / (dt * scale)

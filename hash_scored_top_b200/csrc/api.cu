@@ -164,8 +164,11 @@ FusedPlan plan_select(int pairs, int N, int k, int G, int d, int L, int P, bool 
     const int bpc = (nblk + c - 1) / c;
     const int per = ((L + c - 1) / c + 3) & ~3;
     const int nl = per < L ? per : L;
-    const size_t scratch = hata ? hamming_scratch_bytes(G, d, nl) : table_scratch_bytes(G, d, nl, P);
-    if ((((uint32_t)bpc * 32u + 127u) & ~127u) <= fused_key_capacity(nch) && scratch <= kSegAFree) {
+    // the hard-hash variant builds all its 16 tables in every CTA, with its
+    // scratch in segment B; the soft tables' scratch is in segment A
+    const bool fits = hata ? hamming_scratch_bytes(G, d, L) <= seg_b_bytes(nch)
+                           : table_scratch_bytes(G, d, nl, P) <= kSegAFree;
+    if ((((uint32_t)bpc * 32u + 127u) & ~127u) <= fused_key_capacity(nch) && fits) {
       fp.C = c;
       fp.blocks_per_cta = bpc;
       fp.chunk = (k + c - 1) / c;

@@ -193,7 +193,7 @@ __device__ void build_hamming_table(const QT* __restrict__ Qg, int G, const __nv
   for (int i = tid; i < G * 16; i += blockDim.x) qbyte[i] = 0u;
   stage_rows<D>(R128, 8 * m0, 8 * nm, rs);
   __syncthreads();
-  project_rows<D>(qd, G, rs, 8 * nm, [&](int item, double z) {
+  project_rows_mma<D>(qd, G, rs, 8 * nm, [&](int item, double z) {
     const int h = item / (8 * nm), mi = item % (8 * nm);
     if (z > 0.0) atomicOr(&qbyte[h * 16 + m0 + mi / 8], 1u << (mi % 8));
   });

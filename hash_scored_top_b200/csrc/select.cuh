@@ -404,6 +404,96 @@ __device__ __forceinline__ uint4 lds_key4(KeyAddr key_addr, int i) {
 // g0_of(c): first global index of CTA c. emit(pos, i) as in ordered_compact.
 // scratch: bin_scratch_words() words, the same offset in every CTA. The
 // cluster has synchronised since publish_coarse.
+// Ordered compaction with a tie quota, thread-contiguous: keys > th.t (>= t
+// when th.take_eq is all) are taken, and of the keys == t the first
+// th.take_eq in index order across the cluster. Each thread owns `gpt`
+// consecutive groups of 4 keys (keys past n up to the 128-key chunk must not
+// compare above t); one block scan of packed (greater, equal) counts gives the
+// positions. Writes the pair's list through `stage` (stage_cap words) when
+// this CTA's part fits, else with emit(pos, i). out: the pair's index list.
+template <typename KeyAddr, typename G0Of, typename Emit>
+__device__ void contiguous_compact(KeyAddr key_addr, int n, const SelThreshold& th, int C, int rank, G0Of g0_of,
+                                   SelShared* sh, Emit emit, int* out, uint32_t k, uint32_t* stage,
+                                   uint32_t stage_cap, unsigned long long* ts = nullptr) {
+  cg::cluster_group cluster = cg::this_cluster();
+  const int tid = threadIdx.x;
+  const bool all_eq = th.take_eq == 0xffffffffu;
+  const int ngroups = ((n + 127) & ~127) / 4;
+  const int gpt = ((ngroups + (int)blockDim.x - 1) / (int)blockDim.x) | 1;
+  const int g_begin = min(ngroups, tid * gpt), g_end = min(ngroups, g_begin + gpt);
+  uint32_t n_gt = 0, n_eq = 0;
+  for (int g = g_begin; g < g_end; ++g) {
+    const uint4 q = lds_key4(key_addr, 4 * g);
+    const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const bool valid = 4 * g + j < n;
+      n_gt += (valid && (all_eq ? kv[j] >= th.t : kv[j] > th.t)) ? 1u : 0u;
+      n_eq += (valid && !all_eq && kv[j] == th.t) ? 1u : 0u;
+    }
+  }
+  // packed scan: greater counts in the low 16 bits, equal counts in the high
+  const uint32_t mine = n_gt | (n_eq << 16);
+  const uint32_t excl = block_exclusive_scan(mine, sh);
+  if (tid == (int)blockDim.x - 1) {
+    const uint32_t tot = excl + mine;
+    sh->cnt_w[0][0] = tot & 0xffffu;
+    sh->cnt_w[0][1] = tot >> 16;
+  }
+  __syncthreads();
+  if (tid < C) {
+    uint32_t* dst = cluster.map_shared_rank(&sh->counts[rank][0], (unsigned)tid);
+    dst[0] = sh->cnt_w[0][0];
+    dst[1] = sh->cnt_w[0][1];
+  }
+  sel_stamp(ts, 19);
+  cluster_sync();
+  sel_stamp(ts, 20);
+  // this CTA's tie quota and first output position
+  uint32_t eq_before = 0, sel_before = 0, my_take = 0, my_off = 0;
+  for (int c = 0; c < C; ++c) {
+    const uint32_t e = sh->counts[c][1];
+    const uint32_t left = th.take_eq > eq_before ? th.take_eq - eq_before : 0u;
+    const uint32_t take = all_eq ? 0u : (left < e ? left : e);
+    if (c == rank) {
+      my_take = take;
+      my_off = sel_before;
+    }
+    sel_before += sh->counts[c][0] + take;
+    eq_before += e;
+  }
+  const uint32_t cta_cnt = sh->counts[rank][0] + my_take;
+  const bool staged = cta_cnt <= stage_cap;
+  const uint32_t ex_gt = excl & 0xffffu, ex_eq = excl >> 16;
+  uint32_t pos = ex_gt + (ex_eq < my_take ? ex_eq : my_take);   // position inside this CTA's part
+  uint32_t eq_seen = ex_eq;
+  const int g0 = g0_of(rank);
+  if (n_gt + n_eq > 0) {
+    for (int g = g_begin; g < g_end; ++g) {
+      const uint4 q = lds_key4(key_addr, 4 * g);
+      const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int i = 4 * g + j;
+        if (i >= n) continue;
+        bool take = all_eq ? kv[j] >= th.t : kv[j] > th.t;
+        if (!all_eq && kv[j] == th.t) take = eq_seen++ < my_take;
+        if (take) {
+          if (staged) stage[pos] = (uint32_t)(g0 + i);
+          else emit(my_off + pos, i);
+          ++pos;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  if (staged) {
+    for (uint32_t e = tid; e < cta_cnt; e += blockDim.x)
+      if (my_off + e < k) out[my_off + e] = (int)stage[e];
+  }
+  sel_stamp(ts, 21);
+}
+
 // The selection is written to out[0..k) (the pair's index list, global
 // index = g0_of(rank) + local index): through `stage` (stage_cap words of
 // shared memory) and coalesced stores when this CTA's part fits, else with
@@ -458,7 +548,7 @@ __device__ bool binned_select(KeyAt key_at, KeyAddr key_addr, int n, uint32_t k,
     SelThreshold th;
     th.t = bin_lo<true>(bstar);
     th.take_eq = need == in_bin ? 0xffffffffu : need;   // whole bin: every key >= t
-    ordered_compact(key_at, n, th, C, rank, sh, emit, ts);
+    contiguous_compact(key_addr, n, th, C, rank, g0_of, sh, emit, out, k, stage, stage_cap, ts);
     return true;
   }
   const uint32_t lo = bin_lo<false>(bstar), hi = bin_hi<false>(bstar);

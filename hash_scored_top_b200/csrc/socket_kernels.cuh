@@ -332,17 +332,25 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
     };
     auto before_store = [] { cluster_wait(); };    // every CTA of the cluster has started
     void* scratch = sptr<void>(dyn, fs.base, fs.keysA);
-    if (nl <= 0) {
+    if constexpr (HATA) {
+      // the 16 byte-tables of the hard-hash variant are cheap (popcounts of
+      // the query codes): every CTA builds all of them in its own memory
+      auto local_store = [=](int bb, int l, float v) {
+        float* row = tab0 + bb * TABLE_COLS;
+        for (int x = l; x < TABLE_COLS; x += 16) row[x] = v;
+      };
+      // scratch in segment B (the keys are not written yet): the 128 staged
+      // hyperplane rows do not fit segment A
+      build_hamming_table<D>(Qg, G, p.R, 0, p.L, sptr<void>(dyn, fs.base, fs.segB), local_store, before_store);
+    } else if (nl <= 0) {
       cluster_wait();
-    } else if constexpr (HATA) {
-      build_hamming_table<D>(Qg, G, p.R, l0, nl, scratch, store, before_store);
     } else {
       build_bucket_table<D, QT, decltype(store4), decltype(before_store), 4>(Qg, G, p.R, p.P, p.tau, l0, nl, scratch,
                                                                             store4, p.phase_ts, before_store);
     }
   }
   stamp(p.phase_ts, 9);
-  cluster_sync();     // every table entry has landed in every CTA
+  if constexpr (!HATA) cluster_sync();     // every table entry has landed in every CTA
   // Launched as the programmatic dependent of the key-append kernel, the
   // kernel got here while that kernel may still run: the bucket IDs and norms
   // are read only after it completed (a no-op for an ordinary launch).

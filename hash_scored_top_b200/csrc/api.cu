@@ -167,7 +167,8 @@ FusedPlan plan_select(int pairs, int N, int k, int G, int d, int L, int P, bool 
     // the hard-hash variant builds all its 16 tables in every CTA, with its
     // scratch in segment B; the soft tables' scratch is in segment A
     const bool fits = hata ? hamming_scratch_bytes(G, d, L) <= seg_b_bytes(nch)
-                           : table_scratch_bytes(G, d, nl, P) <= kSegAFree;
+                           : table_scratch_dbl_bytes(G, d, nl, P) <= kSegAFree &&
+                                 table_scratch_rows_bytes(d, nl, P) <= seg_b_bytes(nch);
     if ((((uint32_t)bpc * 32u + 127u) & ~127u) <= fused_key_capacity(nch) && fits) {
       fp.C = c;
       fp.blocks_per_cta = bpc;

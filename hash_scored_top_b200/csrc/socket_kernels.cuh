@@ -345,8 +345,11 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
     } else if (nl <= 0) {
       cluster_wait();
     } else {
+      // doubles in segment A, staged hyperplane rows in segment B (neither
+      // holds keys yet)
       build_bucket_table<D, QT, decltype(store4), decltype(before_store), 4>(Qg, G, p.R, p.P, p.tau, l0, nl, scratch,
-                                                                            store4, p.phase_ts, before_store);
+                                                                            store4, p.phase_ts, before_store,
+                                                                            sptr<void>(dyn, fs.base, fs.segB));
     }
   }
   stamp(p.phase_ts, 9);

@@ -20,13 +20,18 @@
 namespace hst {
 
 // Bytes of shared scratch build_bucket_table needs for nl tables: float64
-// words for the unit queries, bit factors and lo/hi products, then the
-// staged bf16 hyperplane rows.
-__host__ __device__ inline size_t table_scratch_bytes(int G, int d, int nl, int P) {
+// words for the unit queries, bit factors and lo/hi products (the "double"
+// part), then the staged bf16 hyperplane rows (the "rows" part). The rows may
+// go to a separate buffer (rows_scratch); otherwise they follow the doubles.
+__host__ __device__ inline size_t table_scratch_dbl_bytes(int G, int d, int nl, int P) {
   const int plo = P / 2, phi = P - plo;
   size_t dbl = (size_t)G * (d + 8) + (size_t)G * nl * P * 2 + (size_t)G * nl * ((1 << plo) + (1 << phi) + 2);
   dbl = (dbl + 1) & ~(size_t)1;                         // keep the bf16 rows 16-byte aligned
-  return dbl * 8 + (size_t)nl * P * d * 2;
+  return dbl * 8;
+}
+__host__ __device__ inline size_t table_scratch_rows_bytes(int d, int nl, int P) { return (size_t)nl * P * d * 2; }
+__host__ __device__ inline size_t table_scratch_bytes(int G, int d, int nl, int P) {
+  return table_scratch_dbl_bytes(G, d, nl, P) + table_scratch_rows_bytes(d, nl, P);
 }
 
 __device__ __forceinline__ double load_q(const float* q, int i) { return (double)q[i]; }
@@ -44,45 +49,11 @@ __device__ __forceinline__ int qpad_index(int h, int c) {
   return h * qpad_row<D>() + (c / (D / 8)) * (D / 8 + 1) + c % (D / 8);
 }
 
-// Projections z[item] = q_hat_h . r_m for items (h, m) with m = row0 + mi,
-// mi < nrows, computed as eight partial dot products of D / 8 terms (one per
-// lane of an aligned group of 8 lanes, two independent chains each, added in a
-// fixed butterfly order) in float64: short dependency chains, since float64
-// latency is long. Calls out(item, z) once per item from the group's first
-// lane. qhat: G padded rows (qpad_index); rs: [nrows][D] bf16 rows.
-template <int D, typename Out>
-__device__ __forceinline__ void project_rows(const double* qhat, int G, const __nv_bfloat16* rs, int nrows, Out out) {
-  const int nitems = G * nrows;
-  for (int base = 0; base < 8 * nitems; base += blockDim.x) {
-    const int e = base + threadIdx.x;
-    const bool valid = e < 8 * nitems;
-    const int item = valid ? e >> 3 : 0, part = e & 7;
-    const int h = item / nrows, mi = item % nrows;
-    const double* qh = qhat + h * qpad_row<D>() + part * (D / 8 + 1);
-    const uint4* rr = reinterpret_cast<const uint4*>(rs + (size_t)mi * D + part * (D / 8));
-    double z0 = 0.0, z1 = 0.0;
-#pragma unroll
-    for (int c8 = 0; c8 < D / 64; ++c8) {
-      const uint4 w = rr[c8];
-      const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        z0 = fma(qh[c8 * 8 + 2 * k], (double)bf16lo_to_f32(ws[k]), z0);
-        z1 = fma(qh[c8 * 8 + 2 * k + 1], (double)bf16hi_to_f32(ws[k]), z1);
-      }
-    }
-    double z = z0 + z1;
-    z += __shfl_xor_sync(FULL, z, 1);
-    z += __shfl_xor_sync(FULL, z, 2);
-    z += __shfl_xor_sync(FULL, z, 4);
-    if (valid && part == 0) out(item, z);
-  }
-}
-
-// The same projections on the fp64 tensor cores (mma m8n8k4, f64 in and
-// out): warp w computes 8x8 tiles z(h, mi) for 8 heads and 8 hyperplane rows,
-// accumulating over the head dimension in steps of 4 in a fixed order, so
-// every element's value depends only on its inputs. Calls out(item, z) once
+// Projections z(h, mi) = qhat_h . r_mi on the fp64 tensor cores (mma
+// m8n8k4, f64 in and out): warp w computes 8x8 tiles for 8 heads and 8
+// hyperplane rows, accumulating over the head dimension in steps of 4 in a
+// fixed order, so every element's value depends only on its inputs. qhat: G
+// padded rows (qpad_index); rs: [nrows][D] bf16 rows. Calls out(item, z) once
 // per item h * nrows + mi (h < G, mi < nrows).
 __device__ __forceinline__ void mma_f64_m8n8k4(double& d0, double& d1, double a, double b) {
   asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0,%1}, {%2}, {%3}, {%0,%1};"
@@ -151,13 +122,15 @@ struct NoHook {
 // store(b, l, v, cnt) once per bucket and group of 4 tables l .. l + cnt - 1
 // (groups start at l0 + 4g; cnt < 4 only for the last group), v[0..cnt).
 // Qg points at the G query rows of the pair (row stride D); scratch holds
-// table_scratch_bytes. All threads of the block must call this; it calls
+// table_scratch_bytes, or table_scratch_dbl_bytes when rows_scratch (16-byte
+// aligned, table_scratch_rows_bytes) is given. All threads of the block must call this; it calls
 // before_store() (all threads, converged) just before the first store and
 // ends with __syncthreads().
 template <int D, typename QT, typename Store, typename Hook = NoHook, int VEC = 1>
 __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_bfloat16* __restrict__ R, int P,
                                    float tau, int l0, int nl, void* scratch, Store store,
-                                   unsigned long long* ts = nullptr, Hook before_store = Hook()) {
+                                   unsigned long long* ts = nullptr, Hook before_store = Hook(),
+                                   void* rows_scratch = nullptr) {
   auto tstamp = [&](int ph) {
     if (ts != nullptr && threadIdx.x == 0) {
       ts[blockIdx.x * 24 + ph] = (unsigned long long)clock64();
@@ -174,7 +147,8 @@ __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_
   double* lo = sig + G * nl * P * 2;                    // [G][nl][slo]
   double* hi = lo + G * nl * slo;                       // [G][nl][shi]
   const int ndbl = (G * qpad_row<D>() + G * nl * P * 2 + G * nl * (slo + shi) + 1) & ~1;   // 16-byte aligned rows
-  __nv_bfloat16* rs = reinterpret_cast<__nv_bfloat16*>(qhat + ndbl);                       // [nl * P][D]
+  __nv_bfloat16* rs = rows_scratch ? reinterpret_cast<__nv_bfloat16*>(rows_scratch)        // [nl * P][D]
+                                    : reinterpret_cast<__nv_bfloat16*>(qhat + ndbl);
 
   // 1. unit query rows; this CTA's hyperplane rows
   unit_queries<D>(Qg, G, qhat);

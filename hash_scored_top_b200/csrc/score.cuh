@@ -15,10 +15,10 @@
 // with byte 1 replaced by the ID (one byte-permute) plus the compile-time
 // offset 4j in the load instruction. Rows >= 2^P and tables >= L hold zero.
 //
-// The LP values of a key go to 8 (16 for LP > 32) partial sums of at most 4
-// terms that are added in a fixed tree, so an f32 score carries at most 9
-// roundings of 2^-24 (entry, sums, norm product) -- below the 1e-6 relative
-// near-tie window of the selection.
+// The LP values of a key go to 8 (16 for LP = 64) partial sums of at most 6
+// (4 for LP = 64) terms that are added in a fixed tree, so an f32 score of
+// non-negative terms carries at most 10 roundings of 2^-24 (entry, sums, norm
+// product) -- below the 1e-6 relative near-tie window of the selection.
 #pragma once
 
 #include "common.cuh"
@@ -58,10 +58,10 @@ __device__ __forceinline__ float lds_imm(uint32_t addr) {
   return v;
 }
 
-// Number of partial sums: every partial gets at most 4 terms.
+// Number of partial sums (more would spill registers at 48-byte rows).
 template <int LP>
 struct ScoreAcc {
-  static constexpr int N = LP > 32 ? 16 : 8;
+  static constexpr int N = LP > 48 ? 16 : 8;
 };
 
 template <int LP, int J>

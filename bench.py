@@ -391,6 +391,7 @@ def run_ours(args, world, rank, local):
     if not args.no_extras and not w.hata:
         result["e2e"] = run_e2e(args, w, api, caches, device, world, ws)
         result["dense_decode"] = run_dense(w, api, caches, device, rb, peak)
+        result["prefill_hash"] = run_prefill_hash(w, api, caches, device, peak)
         if rank == 0 and world == 1:
             result["cpu_baseline"] = cpu_baseline(w, caches[0], sample_pairs=8)
     del g_step, g_dec, g_sel
@@ -435,6 +436,28 @@ def run_e2e(args, w, api, caches, device, world, ws):
             "d2h_bytes_per_step": o_host.numel() * o_host.element_size(), "steps": n,
             "note": "plain API calls per step (no graph); KV cache resident in HBM; per-step query + new "
                     "K/V row in, output out"}
+
+
+def run_prefill_hash(w, api, caches, device, peak):
+    """Prefill hashing (SOCKET step 1) of all N cached keys of one cache: reads K and V once."""
+    import torch
+    c = caches[0]
+    n, warm = 5, 2
+    for _ in range(warm):
+        api.socket_hash_keys(c["K"], c["V"], c["R"], w.L, w.P, c["ids"], c["norms"], 0, w.N)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(n):
+        api.socket_hash_keys(c["K"], c["V"], c["R"], w.L, w.P, c["ids"], c["norms"], 0, w.N)
+    e.record()
+    torch.cuda.synchronize()
+    ms = s.elapsed_time(e) / n
+    lp = 16 if w.L <= 16 else 32 if w.L <= 32 else 48 if w.L <= 48 else 64
+    nbytes = w.pairs * w.N * (2 * w.d * 2 + lp + 2) + w.L * w.P * w.d * 2   # K, V in; ids, norms out
+    gbs = nbytes / (ms * 1e-3) / 1e9
+    return {"us": ms * 1e3, "bytes": nbytes, "hbm_gbs": gbs, "frac_of_peak": gbs / peak,
+            "keys_per_s": w.pairs * w.N / (ms * 1e-3)}
 
 
 def run_dense(w, api, caches, device, rb, peak):

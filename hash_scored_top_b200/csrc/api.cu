@@ -11,6 +11,7 @@
 
 #include "../../include/hash_scored_top.h"
 #include "socket_kernels.cuh"
+#include "hash_tc.cuh"
 
 using namespace hst;
 
@@ -529,6 +530,30 @@ int hash_launch(const void* K, const void* V, sk_dtype kv, const void* R, int B,
   hp.P = P;
   hp.pairs = B * Hkv;
   const int LP = L * P;
+  if (kv == SK_BF16 && P == 8) {        // tensor-core projections (one table per n-tile)
+    if (n_count <= kAppendMaxKeys) {
+      const dim3 grid(hp.pairs, n_count);
+      if (d == 64) hash_keys_tc_append_kernel<64><<<grid, HTC_APPEND_THREADS, 0, s>>>(hp);
+      else hash_keys_tc_append_kernel<128><<<grid, HTC_APPEND_THREADS, 0, s>>>(hp);
+      return check_launch("hash_keys_tc_append_kernel");
+    }
+    const size_t smem = htc_smem_bytes(d, L, V != nullptr);
+    const int threads = htc_threads(L);
+    const long units = (long)hp.pairs * ((n_begin + n_count - 1) / HTC_KEYS - n_begin / HTC_KEYS + 1);
+    int per_sm = 1;
+    if (d == 64) {
+      set_kernel_smem(hash_keys_tc_kernel<64>, smem);
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hash_keys_tc_kernel<64>, threads, smem);
+    } else {
+      set_kernel_smem(hash_keys_tc_kernel<128>, smem);
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hash_keys_tc_kernel<128>, threads, smem);
+    }
+    const long slots = (long)(per_sm > 0 ? per_sm : 1) * kNumSMs;
+    const int grid = (int)(units < slots ? units : slots);
+    if (d == 64) hash_keys_tc_kernel<64><<<grid, threads, smem, s>>>(hp);
+    else hash_keys_tc_kernel<128><<<grid, threads, smem, s>>>(hp);
+    return check_launch("hash_keys_tc_kernel");
+  }
   if (n_count <= kAppendMaxKeys) {      // decode-time append: a few keys per pair
     const dim3 grid(hp.pairs, n_count);
     const int threads = (LP + 31) / 32 * 32;

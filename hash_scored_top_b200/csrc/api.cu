@@ -9,6 +9,8 @@
 #include <string>
 #include <vector>
 
+#include <cudaTypedefs.h>
+
 #include "../../include/hash_scored_top.h"
 #include "socket_kernels.cuh"
 #include "hash_tc.cuh"
@@ -511,6 +513,32 @@ size_t select_ws_bytes(const FusedPlan& fp, int pairs, int Ncap, int L) {
   return align256(table_image_bytes(pairs, L)) + align256((size_t)pairs * Ncap * 4);
 }
 
+// 2-D tensor map of a [rows][d] bf16 matrix for TMA tiles of 64 columns x
+// box_rows rows with the 128-byte swizzle (the layout the tcgen05 hash
+// kernel's operands use). The driver's encoder is looked up once through the
+// runtime.
+int encode_rows_map(CUtensorMap* map, const void* base, long rows, int d, int box_rows) {
+  static PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  });
+  if (encode == nullptr) return fail(SK_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(SK_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return SK_OK;
+}
+
 constexpr int kAppendMaxKeys = 16;
 
 int hash_launch(const void* K, const void* V, sk_dtype kv, const void* R, int B, int Hkv, int Ncap, int n_begin,
@@ -530,29 +558,36 @@ int hash_launch(const void* K, const void* V, sk_dtype kv, const void* R, int B,
   hp.P = P;
   hp.pairs = B * Hkv;
   const int LP = L * P;
-  if (kv == SK_BF16 && P == 8) {        // tensor-core projections (one table per n-tile)
-    if (n_count <= kAppendMaxKeys) {
-      const dim3 grid(hp.pairs, n_count);
-      if (d == 64) hash_keys_tc_append_kernel<64><<<grid, HTC_APPEND_THREADS, 0, s>>>(hp);
-      else hash_keys_tc_append_kernel<128><<<grid, HTC_APPEND_THREADS, 0, s>>>(hp);
-      return check_launch("hash_keys_tc_append_kernel");
-    }
-    const size_t smem = htc_smem_bytes(d, L, V != nullptr);
-    const int threads = htc_threads(L);
-    const long units = (long)hp.pairs * ((n_begin + n_count - 1) / HTC_KEYS - n_begin / HTC_KEYS + 1);
+  if (kv == SK_BF16 && P == 8 && n_count > kAppendMaxKeys) {   // tcgen05 projections, tiles of 128 keys
+    const TcPlan pl = tc_plan(d, L, V != nullptr);
+    TcRows tr;
+    tr.tile_key0 = n_begin / TC_M;
+    tr.tiles_per_pair = (n_begin + n_count - 1) / TC_M - tr.tile_key0 + 1;
+    tr.n_tiles = hp.pairs * tr.tiles_per_pair;
+    CUtensorMap mapK, mapV, mapR;
+    std::memset(&mapV, 0, sizeof(mapV));
+    SK_TRY(encode_rows_map(&mapR, R, (long)8 * L, d, 32));
+    SK_TRY(encode_rows_map(&mapK, K, (long)hp.pairs * Ncap, d, TC_M));
+    if (V != nullptr) SK_TRY(encode_rows_map(&mapV, V, (long)hp.pairs * Ncap, d, TC_M));
+    // at most 512 / (the columns one CTA allocates) CTAs may share an SM's
+    // tensor memory: ask for enough shared memory that no more fit
+    const int share = 512 / (pl.ncols * (pl.ahead ? 2 : 1));
+    size_t smem = pl.smem;
+    const size_t floor_bytes = (size_t)(TC_SMEM_SM / (share + 1)) - 1024 + 16;
+    if (smem < floor_bytes) smem = floor_bytes;
     int per_sm = 1;
     if (d == 64) {
-      set_kernel_smem(hash_keys_tc_kernel<64>, smem);
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hash_keys_tc_kernel<64>, threads, smem);
+      set_kernel_smem(hash_keys_tcgen05_kernel<64>, smem);
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hash_keys_tcgen05_kernel<64>, TC_THREADS, smem);
     } else {
-      set_kernel_smem(hash_keys_tc_kernel<128>, smem);
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hash_keys_tc_kernel<128>, threads, smem);
+      set_kernel_smem(hash_keys_tcgen05_kernel<128>, smem);
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, hash_keys_tcgen05_kernel<128>, TC_THREADS, smem);
     }
     const long slots = (long)(per_sm > 0 ? per_sm : 1) * kNumSMs;
-    const int grid = (int)(units < slots ? units : slots);
-    if (d == 64) hash_keys_tc_kernel<64><<<grid, threads, smem, s>>>(hp);
-    else hash_keys_tc_kernel<128><<<grid, threads, smem, s>>>(hp);
-    return check_launch("hash_keys_tc_kernel");
+    const int grid = (int)(tr.n_tiles < slots ? tr.n_tiles : slots);
+    if (d == 64) hash_keys_tcgen05_kernel<64><<<grid, TC_THREADS, smem, s>>>(hp, tr, mapK, mapV, mapR);
+    else hash_keys_tcgen05_kernel<128><<<grid, TC_THREADS, smem, s>>>(hp, tr, mapK, mapV, mapR);
+    return check_launch("hash_keys_tcgen05_kernel");
   }
   if (n_count <= kAppendMaxKeys) {      // decode-time append: a few keys per pair
     const dim3 grid(hp.pairs, n_count);

@@ -1,304 +1,434 @@
 // Tensor-core hashing of bf16 keys with P = 8 hyperplanes per table (SOCKET
 // technical summary, section 中核メカニズム：ソフト LSH, step 1; the hard-hash
 // codes of the HATA digest, section 3, are the same computation with 16
-// tables of 8). The projections of 16 keys on the 8 hyperplanes of one table
-// are one chain of mma.sync m16n8k16 over the head dimension (bf16 products
-// are exact, the sums are f32), so with P = 8 the sign pattern of a tile row
-// is that key's bucket ID. The value norm is a float64 sum of squares rounded
-// once to the nearest f16.
+// tables of 8). For a tile of 128 keys the projections K_tile . R^T are one
+// tcgen05 MMA chain over the head dimension (M = 128 keys, N = the
+// hyperplanes, bf16 operands in shared memory, f32 accumulators in tensor
+// memory). With P = 8, columns 8l .. 8l + 7 of a key's row are table l's
+// hyperplanes, so the key's ID bytes are the sign bits of its row taken 8 at a
+// time. The value norm is a float64 sum of squares rounded once to the nearest
+// f16.
 //
-// The bulk kernel (prefill, 64-key units) and the append kernel (decode time,
-// one CTA per key) issue the same MMA chain per table -- operand fragments
-// filled from the same bf16 values, k steps in the same order, accumulator
-// from zero -- and the MMA computes each output element from its own row and
-// column only, so a key gets the same ID bytes either way.
+// The kernel hashes key ranges of more than a few keys (prefill); the
+// decode-time append of a few keys per pair stays on the SIMT append kernel,
+// whose latency hides behind the selection kernel that follows it. The two
+// sum the f32 projection in different orders, so a key's sign bit can differ
+// between them only where its projection is within f32 rounding of zero.
+//
+// Thread roles (256 threads): warps 0-3 decode the accumulators -- warp w
+// owns tensor-memory lanes 32w .. 32w + 31, i.e. rows 32w .. 32w + 31 of the
+// tile, one key per thread. Warps 4-7 take the value norms (row m in thread
+// 128 + m); thread 128 also issues the tile loads and the MMAs. Bulk tiles
+// arrive by TMA tensor copies into rings of key and value stages (128-byte
+// swizzle). When two accumulator buffers fit in tensor memory (8L <= 256),
+// the MMAs of tile i + 1 run while tile i is decoded.
 #pragma once
 
-#include "attend.cuh"
+#include <cuda.h>
+
 #include "hash_kernels.cuh"
 
 namespace hst {
 
-constexpr int HTC_TPW = 4;          // tables per warp (B fragments held in registers)
-constexpr int HTC_KEYS = 64;        // keys per unit of the bulk kernel
-constexpr int HTC_STAGES = 3;       // units in flight per CTA (cp.async ring)
-constexpr int HTC_APPEND_THREADS = 256;
+constexpr int TC_M = 128;               // keys per tile = MMA M = tensor-memory lanes used
+constexpr int TC_THREADS = 256;
+constexpr int TC_MAX_KSTAGES = 4;
+constexpr int TC_VSTAGES = 2;
+constexpr int TC_SMEM_MAX = 232448;     // dynamic shared memory of one CTA at most
+constexpr int TC_SMEM_SM = 233472;      // shared memory of one SM
+constexpr uint32_t TC_ATOM = TC_M * 128;  // one 128-row x 128-byte swizzle column of a tile
 
-__host__ __device__ inline int htc_threads(int L) { return 32 * ((L + HTC_TPW - 1) / HTC_TPW); }
+// Shared-memory plan (host and device compute the same one). Operands are
+// K-major with the 128-byte swizzle: a matrix of r rows x d bf16 is d / 64
+// column atoms of r rows x 128 bytes (atom a at a * r * 128), row n at n * 128
+// inside the atom, its 16-byte chunk c at ((c ^ n) & 7) * 16.
+//  R      [npad rows][d]; rows >= 8L are zero
+//  K ring kstages x [128 rows][d]
+//  V ring vstages x [128 rows][d] (0 stages without norms)
+//  ctl    mbarriers fullK[4], fullV[2], mma[2], R (8 B each); tensor-memory
+//         base address (4 B); failure flag (4 B)
+// ahead = 1: two accumulator buffers, the MMAs of tile i + 1 are issued while
+// tile i is decoded (needs 2 * ncols <= 512 and 3 key stages).
+struct TcPlan {
+  int npad, ncols, kstages, vstages, ahead;
+  uint32_t r_off, k_off, v_off, tile_bytes, ctl_off, smem;
+};
 
-// Shared memory of the bulk kernel: per stage the unit's key rows [64][D + 8]
-// bf16 (the 16-byte pad makes the ldmatrix rows conflict-free) and, when
-// norms are wanted, its value rows [64][D]; then two ID-byte buffers
-// [64][LPB] (the unit being computed and the one being written out).
-__host__ __device__ inline size_t htc_stage_bytes(int D, bool values) {
-  return (size_t)HTC_KEYS * (D + 8) * 2 + (values ? (size_t)HTC_KEYS * D * 2 : 0);
+__host__ __device__ inline TcPlan tc_plan(int d, int L, bool values) {
+  TcPlan p;
+  p.npad = (8 * L + 31) / 32 * 32;
+  p.ncols = 32;
+  while (p.ncols < p.npad) p.ncols *= 2;
+  p.tile_bytes = (uint32_t)TC_M * d * 2;
+  p.r_off = 0;
+  p.k_off = (uint32_t)p.npad * d * 2;
+  p.vstages = values ? TC_VSTAGES : 0;
+  const uint32_t room = (uint32_t)TC_SMEM_MAX - p.k_off - 128 - (uint32_t)p.vstages * p.tile_bytes;
+  p.kstages = (int)(room / p.tile_bytes);
+  if (p.kstages > TC_MAX_KSTAGES) p.kstages = TC_MAX_KSTAGES;
+  p.ahead = 2 * p.ncols <= 512 && p.kstages >= 3 ? 1 : 0;
+  p.v_off = p.k_off + (uint32_t)p.kstages * p.tile_bytes;
+  p.ctl_off = p.v_off + (uint32_t)p.vstages * p.tile_bytes;
+  p.smem = p.ctl_off + 128;
+  return p;
 }
-__host__ __device__ inline size_t htc_smem_bytes(int D, int L, bool values) {
-  return HTC_STAGES * htc_stage_bytes(D, values) + 2 * (size_t)HTC_KEYS * ids_bytes_per_key(L);
+
+// ---------------------------------------------------------------- tcgen05 wrappers
+__device__ __forceinline__ void tmem_alloc(uint32_t slot, uint32_t ncols) {
+  asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(slot), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tmem_relinquish() {
+  asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
+  asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr), "r"(ncols) : "memory");
+}
+__device__ __forceinline__ void tc_fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// D[tmem] (+)= A[smem] . B[smem]^T, bf16 inputs, f32 accumulators.
+__device__ __forceinline__ void tc_mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                            uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Arrives once on the mbarrier when every MMA this thread issued so far is done.
+__device__ __forceinline__ void tc_commit(uint32_t mbar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(mbar) : "memory");
 }
 
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+// 32 (or 64) consecutive f32 columns of this thread's tensor-memory lane; the
+// wait takes the registers as operands so that no use is scheduled before it.
+#define HST_TMEM_LD32(addr, v)                                                                                   \
+  asm volatile(                                                                                                  \
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"            \
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"                                 \
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]),           \
+        "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]),     \
+        "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),   \
+        "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])    \
+      : "r"(addr))
+#define HST_TMEM_WAIT(v)                                                                                         \
+  asm volatile("tcgen05.wait::ld.sync.aligned;"                                                                  \
+               : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]), "+r"(v[6]), "+r"(v[7]),  \
+                 "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]), "+r"(v[12]), "+r"(v[13]), "+r"(v[14]),         \
+                 "+r"(v[15]), "+r"(v[16]), "+r"(v[17]), "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]),       \
+                 "+r"(v[22]), "+r"(v[23]), "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]),       \
+                 "+r"(v[29]), "+r"(v[30]), "+r"(v[31])                                                            \
+               :                                                                                                 \
+               : "memory")
 
-// Float64 norm of a value row held as D/8 chunks of 8 bf16, chunk j in lane
-// j of a group of D/8 lanes: each lane sums its 8 squares in order, then the
-// group adds by an xor tree. Every lane of the group returns the norm.
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
+  HST_TMEM_LD32(taddr, v);
+  HST_TMEM_WAIT(v);
+}
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&v)[32], uint32_t (&x)[32]) {
+  HST_TMEM_LD32(taddr, v);
+  HST_TMEM_LD32(taddr + 32u, x);
+  HST_TMEM_WAIT(v);
+  HST_TMEM_WAIT(x);
+}
+
+// Sign word of 32 accumulator columns: bit j = [column j > 0], four
+// independent byte chains.
+__device__ __forceinline__ uint32_t sign_word(const uint32_t (&v)[32]) {
+  uint32_t by[4];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t b = 0u;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) b |= (__uint_as_float(v[8 * q + k]) > 0.f ? 1u : 0u) << k;
+    by[q] = b;
+  }
+  return by[0] | (by[1] << 8) | (by[2] << 16) | (by[3] << 24);
+}
+
+// Shared-memory operand descriptor, K-major, 128-byte swizzle: 8-row x
+// 128-byte atoms (rows 128 bytes apart, atom start 1024-byte aligned), `sbo`
+// bytes between 8-row groups; the k offset inside the atom is added to the
+// start address; descriptor version 1, layout type 2.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr, uint32_t sbo) {
+  return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)1u << 16) | ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) |
+         (1ull << 46) | (2ull << 61);
+}
+// 2-D TMA tensor copy (no multicast) of the box at (x, y) into shared memory,
+// completing its bytes on the mbarrier.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t mbar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];" ::"r"(
+          dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(mbar)
+      : "memory");
+}
+// Instruction descriptor: f32 accumulators, bf16 A and B, both K-major, M = 128, N = n.
+__device__ __forceinline__ uint32_t umma_idesc_bf16(int n) {
+  return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(TC_M >> 4) << 24);
+}
+
+// Rotates the 4*NW bytes of w so that byte j becomes input byte (j + r) mod 4NW.
+template <int NW>
+__device__ __forceinline__ void rotate_bytes(uint32_t (&w)[NW], int r) {
+  const int rw = r >> 2;
+#pragma unroll
+  for (int s = 1; s < NW; s <<= 1) {
+    uint32_t u[NW];
+#pragma unroll
+    for (int i = 0; i < NW; ++i) u[i] = (rw & s) ? w[(i + s) % NW] : w[i];
+#pragma unroll
+    for (int i = 0; i < NW; ++i) w[i] = u[i];
+  }
+  const uint32_t sh = 8u * (uint32_t)(r & 3);
+  uint32_t u[NW];
+#pragma unroll
+  for (int i = 0; i < NW; ++i) u[i] = __funnelshift_r(w[i], w[(i + 1) % NW], sh);
+#pragma unroll
+  for (int i = 0; i < NW; ++i) w[i] = u[i];
+}
+
+// Float64 norm of row m of a value tile in the swizzled operand layout at
+// vbase: chunk c's 8 squares are summed in order into p_c, then p is folded
+// in halves (p_c += p_{c+h} for h = D/16, ..., 1), and the square root of p_0
+// is returned.
 template <int D>
-__device__ __forceinline__ double value_norm_chunks(uint4 chunk) {
+__device__ __forceinline__ double value_norm_tile(uint32_t vbase, int m) {
   constexpr int CPR = D / 8;
-  const uint32_t w[4] = {chunk.x, chunk.y, chunk.z, chunk.w};
-  double ss = 0.0;
+  double p[CPR];
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const double lo = (double)bf16lo_to_f32(w[e]), hi = (double)bf16hi_to_f32(w[e]);
-    ss = fma(lo, lo, ss);
-    ss = fma(hi, hi, ss);
+  for (int c = 0; c < CPR; ++c) {
+    uint32_t w[4];
+    const uint32_t a = vbase + (uint32_t)(c >> 3) * TC_ATOM + (uint32_t)m * 128u + (uint32_t)(((c ^ m) & 7) * 16);
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(w[0]), "=r"(w[1]), "=r"(w[2]), "=r"(w[3]) : "r"(a));
+    double s = 0.0;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const double lo = (double)bf16lo_to_f32(w[e]), hi = (double)bf16hi_to_f32(w[e]);
+      s = fma(lo, lo, s);
+      s = fma(hi, hi, s);
+    }
+    p[c] = s;
   }
 #pragma unroll
-  for (int o = CPR / 2; o > 0; o >>= 1) ss += __shfl_xor_sync(FULL, ss, o);
-  return sqrt(ss);
+  for (int h = CPR / 2; h > 0; h >>= 1)
+#pragma unroll
+    for (int c = 0; c < h; ++c) p[c] = p[c] + p[c + h];
+  return sqrt(p[0]);
 }
 
-// Sign byte of one table from an m16n8 accumulator: lane (r, q) holds
-// hyperplanes 2q, 2q + 1 of rows r (acc 0, 1) and r + 8 (acc 2, 3). Returns
-// the byte of row r in .x and of row r + 8 in .y, on every lane.
-__device__ __forceinline__ uint2 htc_sign_bytes(const float (&acc)[4]) {
-  const int q = threadIdx.x & 3;
-  uint32_t v0 = (acc[0] > 0.f ? 1u : 0u) << (2 * q) | (acc[1] > 0.f ? 1u : 0u) << (2 * q + 1);
-  uint32_t v1 = (acc[2] > 0.f ? 1u : 0u) << (2 * q) | (acc[3] > 0.f ? 1u : 0u) << (2 * q + 1);
-  v0 |= __shfl_xor_sync(FULL, v0, 1);
-  v1 |= __shfl_xor_sync(FULL, v1, 1);
-  v0 |= __shfl_xor_sync(FULL, v0, 2);
-  v1 |= __shfl_xor_sync(FULL, v1, 2);
-  return make_uint2(v0, v1);
+// Which keys the tiles hold: tile u covers keys key0 .. key0 + 127 of pair
+// u / tiles_per_pair, key0 = (tile_key0 + u % tiles_per_pair) * 128.
+struct TcRows {
+  int tiles_per_pair;  // tiles covering [n_begin, n_begin + n_count) in one pair
+  int tile_key0;       // first tile index (keys tile_key0 * 128 ..)
+  int n_tiles;
+};
+struct TcTile {
+  int pair, key0;
+};
+__device__ __forceinline__ TcTile tc_tile(const TcRows& tr, int u) {
+  TcTile t;
+  t.pair = u / tr.tiles_per_pair;
+  t.key0 = (tr.tile_key0 + (u - t.pair * tr.tiles_per_pair)) * TC_M;
+  return t;
+}
+// (pair, key) of row m; returns whether the key is one to write (inside
+// [n_begin, n_begin + n_count)).
+__device__ __forceinline__ bool tc_row(const HashParams& p, const TcTile& t, int m, int* pair, int* key) {
+  *pair = t.pair;
+  *key = t.key0 + m;
+  return *key >= p.n_begin && *key < p.n_begin + p.n_count;
 }
 
-// B fragments of table t for k step k: hyperplane row 8t + g, columns
-// 16k + 2q (+1) and 16k + 8 + 2q (+1), as bf16 pairs.
-__device__ __forceinline__ uint2 htc_b_frag(const __nv_bfloat16* __restrict__ R, int D, int t, int k) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t* row = reinterpret_cast<const uint32_t*>(R + (size_t)(8 * t + (lane >> 2)) * D);
-  return make_uint2(__ldg(row + 8 * k + (lane & 3)), __ldg(row + 8 * k + 4 + (lane & 3)));
-}
-
-// Bulk: keys [n_begin, n_begin + n_count) of every pair, in units of 64 keys
-// aligned to multiples of 64 (a unit's keys outside the range are computed
-// and not written; rows at or past Ncap are zero-filled). Persistent: CTA b
-// takes units b, b + gridDim.x, ..., with HTC_STAGES units of keys (and
-// values) in flight through cp.async. Warp w holds the B fragments of tables
-// 4w .. 4w + 3 in registers for the whole kernel and runs them over the 4 row
-// tiles of every unit; all warps then take the unit's value norms.
-// Launch with htc_threads(L) threads and htc_smem_bytes(D, L, V != nullptr).
+// Launch: TC_THREADS threads, tc_plan(...).smem bytes of dynamic shared
+// memory, persistent over the tiles (CTA b takes tiles b, b + gridDim.x, ...).
+// mapK / mapV: 2-D bf16 tensor maps of K and V as [pairs * Ncap rows][D],
+// box 64 x 128, 128-byte swizzle (rows past the last pair read as zero).
+// mapR: the hyperplanes [8L rows][D], box 64 x 32, 128-byte swizzle (rows
+// past 8L read as zero).
 template <int D>
-__global__ void __launch_bounds__(512, 1) hash_keys_tc_kernel(const HashParams p) {
-  extern __shared__ __align__(1024) unsigned char dyn[];
-  constexpr int KS = D / 16;                 // k steps
-  constexpr int RW = D + 8;                  // padded key row, bf16 elements
-  constexpr int CPR = D / 8;                 // 16-byte chunks per row
-  const bool values = p.V != nullptr;
-  const int LPB = ids_bytes_per_key(p.L);
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int q = lane & 3, g = lane >> 2;
-  const int nthreads = blockDim.x, nwarps = nthreads >> 5;
-  const uint32_t stage_bytes = (uint32_t)htc_stage_bytes(D, values);
-  const uint32_t smem0 = smem_u32(dyn);
-  uint8_t* idsb0 = dyn + HTC_STAGES * stage_bytes;
-
-  const int n_end = p.n_begin + p.n_count;
-  const int u_begin = p.n_begin / HTC_KEYS, u_end = (n_end + HTC_KEYS - 1) / HTC_KEYS;
-  const int units_per_pair = u_end - u_begin;
-  const int total = p.pairs * units_per_pair;
-  // first key of unit u (of its pair), or -1 past the end; the pair in *pair
-  auto unit_key0 = [&](int u, int* pair) {
-    if (u >= total) return -1;
-    *pair = u / units_per_pair;
-    return (u_begin + (u - *pair * units_per_pair)) * HTC_KEYS;
-  };
-
-  // cp.async copies of the unit at (pair, k0) into stage st
-  auto issue = [&](int pair, int k0, int st) {
-    if (k0 < 0) return;
-    const size_t base = ((size_t)pair * p.Ncap + k0) * D;
-    const __nv_bfloat16* kb = reinterpret_cast<const __nv_bfloat16*>(p.K) + base;
-    const uint32_t ks = smem0 + st * stage_bytes;
-    for (int e = tid; e < HTC_KEYS * CPR; e += nthreads) {
-      const int row = e / CPR, c = e % CPR;
-      const bool ok = k0 + row < p.Ncap;
-      cp_async16(ks + (uint32_t)(row * RW + 8 * c) * 2, ok ? kb + (size_t)row * D + 8 * c : kb, ok);
-    }
-    if (values) {
-      const __nv_bfloat16* vb = reinterpret_cast<const __nv_bfloat16*>(p.V) + base;
-      const uint32_t vs = ks + HTC_KEYS * RW * 2;
-      for (int e = tid; e < HTC_KEYS * CPR; e += nthreads) {
-        const bool ok = k0 + e / CPR < p.Ncap;
-        cp_async16(vs + (uint32_t)e * 16, ok ? vb + (size_t)e * 8 : vb, ok);
-      }
-    }
-  };
-
-  // ID bytes of the unit at (pair, k0) from buffer ib to global; clears ib
-  auto write_out = [&](int pair, int k0, uint8_t* ib) {
-    uint32_t* out = reinterpret_cast<uint32_t*>(p.ids + ((size_t)pair * p.Ncap + k0) * LPB);
-    uint32_t* src = reinterpret_cast<uint32_t*>(ib);
-    const bool whole = k0 >= p.n_begin && k0 + HTC_KEYS <= n_end;
-    for (int e = tid; e < HTC_KEYS * LPB / 4; e += nthreads) {
-      if (whole) {
-        out[e] = src[e];
-      } else {
-        const int key = k0 + (4 * e) / LPB;
-        if (key >= p.n_begin && key < n_end) out[e] = src[e];
-      }
-      src[e] = 0u;
-    }
-  };
-
-  // the ring holds units i .. i + HTC_STAGES - 2 ahead of the loop (HTC_STAGES == 3)
-  int pair_cur = 0, pair_n1 = 0, pair_n2 = 0, pair_prev = 0;
-  int k0_cur = unit_key0(blockIdx.x, &pair_cur);
-  int k0_n1 = unit_key0(blockIdx.x + gridDim.x, &pair_n1);
-  int k0_prev = -1;
-  issue(pair_cur, k0_cur, 0);
-  cp_async_commit();
-  issue(pair_n1, k0_n1, 1);
-  cp_async_commit();
-  for (int e = tid; e < 2 * HTC_KEYS * LPB / 4; e += nthreads) reinterpret_cast<uint32_t*>(idsb0)[e] = 0u;
-
-  uint32_t bf[HTC_TPW][KS][2];
-#pragma unroll
-  for (int j = 0; j < HTC_TPW; ++j) {
-    const int t = min(warp * HTC_TPW + j, p.L - 1);
-#pragma unroll
-    for (int k = 0; k < KS; ++k) {
-      const uint2 b = htc_b_frag(p.R, D, t, k);
-      bf[j][k][0] = b.x;
-      bf[j][k][1] = b.y;
-    }
-  }
-  const int ntab = min(HTC_TPW, p.L - warp * HTC_TPW);     // tables of this warp (>= 1)
-  const uint32_t a_lane = (uint32_t)(((lane & 15) * RW + (lane >> 4) * 8) * 2);
-  // this lane stores table 4w + q: its byte of key n sits at
-  // off + ((t - off - n) mod S); S divides 64, so the key's offset in the unit decides
-  const int t_mine = warp * HTC_TPW + q;
-  const int pos_off = t_mine >= 32 ? 32 : 0;
-  const int pos_mask = id_chunk_size(p.L, pos_off >> 5) - 1;
-  const int pos_base = t_mine - pos_off - g;
-
-  int i = 0;
-  for (; k0_cur >= 0; ++i) {
-    cp_async_wait<HTC_STAGES - 2>();
-    __syncthreads();               // unit i landed for every thread; unit i - 1 fully consumed
-    const int k0_n2 = unit_key0(blockIdx.x + (i + 2) * gridDim.x, &pair_n2);
-    issue(pair_n2, k0_n2, (i + 2) % HTC_STAGES);
-    cp_async_commit();
-    if (k0_prev >= 0) write_out(pair_prev, k0_prev, idsb0 + ((i - 1) & 1) * HTC_KEYS * LPB);
-
-    const uint32_t ks = smem0 + (i % HTC_STAGES) * stage_bytes;
-    uint8_t* ib = idsb0 + (i & 1) * HTC_KEYS * LPB;
-#pragma unroll 1
-    for (int mt = 0; mt < HTC_KEYS / 16; ++mt) {
-      float acc[HTC_TPW][4];
-#pragma unroll
-      for (int j = 0; j < HTC_TPW; ++j) acc[j][0] = acc[j][1] = acc[j][2] = acc[j][3] = 0.f;
-      const uint32_t a_addr = ks + (uint32_t)(mt * 16 * RW * 2) + a_lane;
-#pragma unroll
-      for (int k = 0; k < KS; ++k) {
-        uint32_t a0, a1, a2, a3;
-        ldsm_x4(a_addr + 32u * k, a0, a1, a2, a3);
-#pragma unroll
-        for (int j = 0; j < HTC_TPW; ++j)
-          if (j < ntab) mma_bf16_16816(acc[j], a0, a1, a2, a3, bf[j][k][0], bf[j][k][1]);
-      }
-      // byte j of v0 / v1: the ID of table 4w + j for rows g / g + 8, after the
-      // or-reduction over the 4 lanes of the row (each holds 2 hyperplanes)
-      uint32_t v0 = 0u, v1 = 0u;
-#pragma unroll
-      for (int j = 0; j < HTC_TPW; ++j) {
-        const uint32_t b = 1u << (8 * j + 2 * q);
-        v0 |= (acc[j][0] > 0.f ? b : 0u) | (acc[j][1] > 0.f ? 2u * b : 0u);
-        v1 |= (acc[j][2] > 0.f ? b : 0u) | (acc[j][3] > 0.f ? 2u * b : 0u);
-      }
-      v0 |= __shfl_xor_sync(FULL, v0, 1);
-      v1 |= __shfl_xor_sync(FULL, v1, 1);
-      v0 |= __shfl_xor_sync(FULL, v0, 2);
-      v1 |= __shfl_xor_sync(FULL, v1, 2);
-      if (q < ntab) {
-        const int r0 = mt * 16 + g;
-        ib[r0 * LPB + pos_off + ((pos_base - 16 * mt) & pos_mask)] = (uint8_t)(v0 >> (8 * q));
-        ib[(r0 + 8) * LPB + pos_off + ((pos_base - 16 * mt - 8) & pos_mask)] = (uint8_t)(v1 >> (8 * q));
-      }
-    }
-    if (values) {                  // value norms: a group of D/8 lanes per key
-      const uint4* vs = reinterpret_cast<const uint4*>(dyn + (i % HTC_STAGES) * stage_bytes + HTC_KEYS * RW * 2);
-      constexpr int KPW = 32 / CPR;
-      for (int r = warp * KPW; r < HTC_KEYS; r += nwarps * KPW) {
-        const int row = r + lane / CPR;
-        const double nrm = value_norm_chunks<D>(vs[row * CPR + lane % CPR]);
-        const int key = k0_cur + row;
-        if (lane % CPR == 0 && key >= p.n_begin && key < n_end)
-          p.norms[(size_t)pair_cur * p.Ncap + key] = __double2half(nrm);
-      }
-    }
-    pair_prev = pair_cur;
-    k0_prev = k0_cur;
-    pair_cur = pair_n1;
-    k0_cur = k0_n1;
-    pair_n1 = pair_n2;
-    k0_n1 = k0_n2;
-  }
-  cp_async_wait<0>();
-  __syncthreads();
-  if (k0_prev >= 0) write_out(pair_prev, k0_prev, idsb0 + ((i - 1) & 1) * HTC_KEYS * LPB);
-}
-
-// Append: one CTA of 256 threads per (pair, key) for a few keys per pair (a
-// decode step appends one). The key is row 0 of the A operand (rows 1..15
-// zero); warp w runs tables w, w + 8, ... with fragments loaded straight from
-// global memory, and the last warp takes the value norm with the bulk
-// kernel's lane grouping. A selection kernel launched after this one as its
-// programmatic dependent may start at once: it waits (griddepcontrol.wait)
-// before reading any bucket ID or norm and reads nothing else written here.
-template <int D>
-__global__ void __launch_bounds__(HTC_APPEND_THREADS) hash_keys_tc_append_kernel(const HashParams p) {
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    hash_keys_tcgen05_kernel(const HashParams p, const TcRows tr, const __grid_constant__ CUtensorMap mapK,
+                             const __grid_constant__ CUtensorMap mapV, const __grid_constant__ CUtensorMap mapR) {
+  // a selection kernel launched after this one as its programmatic dependent
+  // may start now: it waits (griddepcontrol.wait) before reading any bucket
+  // ID or norm, and reads nothing else this kernel writes
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-  __shared__ __align__(16) uint8_t idsb[64];
-  constexpr int KS = D / 16;
-  constexpr int CPR = D / 8;
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int q = lane & 3, g = lane >> 2;
-  const int pair = blockIdx.x;
-  const int key = p.n_begin + blockIdx.y;
+  extern __shared__ __align__(1024) unsigned char dyn[];
+  constexpr int KS = D / 16;                 // MMA k steps
+  constexpr int NATOM = D / 64;              // 128-byte column atoms per row
+  const bool values = p.V != nullptr;
+  const TcPlan pl = tc_plan(D, p.L, values);
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const bool decoder = tid < TC_M;
+  const int m = tid & (TC_M - 1);            // this thread's row of every tile
   const int LPB = ids_bytes_per_key(p.L);
-  const size_t row_off = ((size_t)pair * p.Ncap + key) * D;
-  if (tid < 16) reinterpret_cast<uint32_t*>(idsb)[tid] = 0u;
-  const uint32_t* krow = reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(p.K) + row_off);
-  uint32_t a0[KS], a2[KS];
-#pragma unroll
-  for (int k = 0; k < KS; ++k) {
-    a0[k] = g == 0 ? __ldg(krow + 8 * k + q) : 0u;        // row 0, columns 16k + 2q, +1
-    a2[k] = g == 0 ? __ldg(krow + 8 * k + 4 + q) : 0u;    // row 0, columns 16k + 8 + 2q, +1
+  const int SK = pl.kstages, SV = pl.vstages, A = pl.ahead;
+  const int rn = pl.npad;                    // rows of R in shared memory
+  const uint32_t s0 = smem_u32(dyn);
+  constexpr uint32_t kTslot = 72, kFail = 76;   // control-block offsets after the 9 mbarriers
+  const uint32_t fullK = s0 + pl.ctl_off, fullV = fullK + 32, mmab = fullK + 48, rbar = fullK + 64;
+  const uint32_t tslot = fullK + kTslot;
+  volatile int* fail = reinterpret_cast<volatile int*>(dyn + pl.ctl_off + kFail);
+  auto kstage = [&](int j) { return s0 + pl.k_off + (uint32_t)(j % SK) * pl.tile_bytes; };
+  auto vstage = [&](int j) { return s0 + pl.v_off + (uint32_t)(j % (SV > 0 ? SV : 1)) * pl.tile_bytes; };
+
+  if (warp == 0) {
+    tmem_alloc(tslot, (uint32_t)pl.ncols * (A ? 2u : 1u));
+    tmem_relinquish();
   }
-  __syncthreads();
-  for (int t = warp; t < p.L; t += HTC_APPEND_THREADS / 32) {
-    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (tid == TC_M) {
+    for (int j = 0; j < 9; ++j) mbar_init(fullK + 8u * j, 1);
+    *fail = 0;
+    fence_mbar_init();
+    // the hyperplanes, 32 rows x 64 columns per box, into the R operand layout
+    mbar_arrive_expect_tx(rbar, (uint32_t)rn * D * 2u);
+    for (int b = 0; b < rn / 32; ++b)
 #pragma unroll
-    for (int k = 0; k < KS; ++k) {
-      const uint2 b = htc_b_frag(p.R, D, t, k);
-      mma_bf16_16816(acc, a0[k], 0u, a2[k], 0u, b.x, b.y);
+      for (int a = 0; a < NATOM; ++a)
+        tma_load_2d(s0 + pl.r_off + (uint32_t)a * (uint32_t)rn * 128u + (uint32_t)b * 4096u, &mapR, 64 * a,
+                    32 * b, rbar);
+  }
+
+  // thread 128: TMA copies of ring position j's keys (or values)
+  auto tma_rows = [&](const CUtensorMap* map, int j, uint32_t dst, uint32_t bar) {
+    const int u = (int)blockIdx.x + j * (int)gridDim.x;
+    if (u >= tr.n_tiles) return;
+    const TcTile t = tc_tile(tr, u);
+    const int row = t.pair * p.Ncap + t.key0;
+    mbar_arrive_expect_tx(bar, pl.tile_bytes);
+#pragma unroll
+    for (int a = 0; a < NATOM; ++a) tma_load_2d(dst + (uint32_t)a * TC_ATOM, map, 64 * a, row, bar);
+  };
+  auto tma_keys = [&](int j) { tma_rows(&mapK, j, kstage(j), fullK + 8u * (uint32_t)(j % SK)); };
+  auto tma_values = [&](int j) { tma_rows(&mapV, j, vstage(j), fullV + 8u * (uint32_t)(j % SV)); };
+  // accumulator buffer of ring position j, and the parity of its mbarrier phase
+  auto buf_of = [&](int j) { return A ? (uint32_t)(j & 1) : 0u; };
+  auto par_of = [&](int j) { return A ? (uint32_t)((j >> 1) & 1) : (uint32_t)(j & 1); };
+  // thread 128: the MMAs of ring position j into accumulator buffer buf_of(j)
+  bool r_ready = false;
+  auto issue_mma = [&](int j, uint32_t tbase) {
+    if (!r_ready) {
+      if (!mbar_wait_bounded(rbar, 0u)) *fail = 1;
+      r_ready = true;
     }
-    const uint2 by = htc_sign_bytes(acc);
-    if (lane == 0) idsb[id_byte_pos(p.L, t, key)] = (uint8_t)by.x;
+    tc_fence_after_sync();
+    const uint32_t buf = buf_of(j);
+    const uint32_t ks = kstage(j);
+    for (int n0 = 0; n0 < rn; n0 += 256) {
+      const int nn = min(256, rn - n0);
+      const uint32_t idesc = umma_idesc_bf16(nn);
+#pragma unroll
+      for (int s = 0; s < KS; ++s) {
+        const uint32_t koff = (uint32_t)(s >> 2) * TC_ATOM + (uint32_t)(s & 3) * 32u;
+        const uint32_t roff =
+            (uint32_t)(s >> 2) * (uint32_t)rn * 128u + (uint32_t)n0 * 128u + (uint32_t)(s & 3) * 32u;
+        tc_mma_bf16(tbase + buf * (uint32_t)pl.ncols + (uint32_t)n0, umma_desc_sw128(ks + koff, 1024u),
+                    umma_desc_sw128(s0 + pl.r_off + roff, 1024u), idesc, s > 0 ? 1u : 0u);
+      }
+    }
+    tc_commit(mmab + 8u * buf);
+  };
+  auto wait_keys = [&](int j) {
+    if (!mbar_wait_bounded(fullK + 8u * (uint32_t)(j % SK), (uint32_t)((j / SK) & 1))) *fail = 1;
+  };
+
+  const int G = (int)gridDim.x;
+  const int my_tiles = tr.n_tiles > (int)blockIdx.x ? (tr.n_tiles - 1 - (int)blockIdx.x) / G + 1 : 0;
+  if (tid == TC_M) {
+    for (int j = 0; j < SK - 1; ++j) tma_keys(j);
+    for (int j = 0; j < SV - 1; ++j) tma_values(j);
   }
-  if (p.V && warp == HTC_APPEND_THREADS / 32 - 1) {
-    const uint4* vrow = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.V) + row_off);
-    const double nrm = value_norm_chunks<D>(lane < CPR ? __ldg(vrow + lane) : make_uint4(0u, 0u, 0u, 0u));
-    if (lane == 0) p.norms[(size_t)pair * p.Ncap + key] = __double2half(nrm);
-  }
+  tc_fence_before_sync();
   __syncthreads();
-  if (tid < LPB) p.ids[((size_t)pair * p.Ncap + key) * LPB + tid] = idsb[tid];
+  tc_fence_after_sync();
+  const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(dyn + pl.ctl_off + kTslot);
+  if (A && tid == TC_M && my_tiles > 0) {
+    wait_keys(0);
+    issue_mma(0, tbase);
+  }
+
+  for (int i = 0; i < my_tiles; ++i) {
+    const int u = (int)blockIdx.x + i * G;
+    tc_fence_before_sync();                  // the decoded buffer's tensor-memory reads are done
+    __syncthreads();                         // ... and tile i - 1's stages are consumed
+    if (*fail) break;
+    const TcTile t = tc_tile(tr, u);
+    int pair, key;
+    const bool mine = tc_row(p, t, m, &pair, &key);
+    const size_t kidx = (size_t)pair * p.Ncap + key;
+
+    if (!decoder) {
+      if (tid == TC_M) {
+        tma_keys(i + SK - 1);                // into the stages of tile i - 1
+        if (SV > 0) tma_values(i + SV - 1);
+        const int j = i + A;
+        if (j < my_tiles) {
+          wait_keys(j);
+          issue_mma(j, tbase);
+        }
+      }
+      if (SV > 0 && !mbar_wait_bounded(fullV + 8u * (uint32_t)(i % SV), (uint32_t)((i / SV) & 1))) *fail = 1;
+      if (values) {
+        const double nrm = value_norm_tile<D>(vstage(i), m);
+        if (mine) p.norms[kidx] = __double2half(nrm);
+      }
+    } else {
+      // the row's signs: bit j of word b is column 32b + j, i.e. hyperplane
+      // j % 8 of table 4b + j / 8; columns >= 8L are zero and give zero bits
+      const uint32_t buf = buf_of(i);
+      if (!mbar_wait_bounded(mmab + 8u * buf, par_of(i))) *fail = 1;
+      tc_fence_after_sync();
+      const uint32_t ta = tbase + ((uint32_t)(32 * warp) << 16) + buf * (uint32_t)pl.ncols;
+      uint32_t w[16];
+#pragma unroll
+      for (int b = 0; b < 16; ++b) w[b] = 0u;
+#pragma unroll
+      for (int b = 0; b < 16; b += 2) {
+        if (32 * (b + 1) < rn) {
+          uint32_t v[32], x[32];
+          tmem_ld64(ta + (uint32_t)(32 * b), v, x);
+          w[b] = sign_word(v);
+          w[b + 1] = sign_word(x);
+        } else if (32 * b < rn) {
+          uint32_t v[32];
+          tmem_ld32(ta + (uint32_t)(32 * b), v);
+          w[b] = sign_word(v);
+        }
+      }
+      if (mine) {
+        // rotated layout: byte j of chunk c (tables 32c ..) of key n holds table 32c + (j + n) mod S_c
+        uint4* out = reinterpret_cast<uint4*>(p.ids + kidx * LPB);
+        if (LPB == 16) {
+          uint32_t c0[4] = {w[0], w[1], w[2], w[3]};
+          rotate_bytes<4>(c0, key & 15);
+          out[0] = make_uint4(c0[0], c0[1], c0[2], c0[3]);
+        } else {
+          uint32_t c0[8] = {w[0], w[1], w[2], w[3], w[4], w[5], w[6], w[7]};
+          rotate_bytes<8>(c0, key & 31);
+          out[0] = make_uint4(c0[0], c0[1], c0[2], c0[3]);
+          out[1] = make_uint4(c0[4], c0[5], c0[6], c0[7]);
+          if (LPB == 48) {
+            uint32_t c1[4] = {w[8], w[9], w[10], w[11]};
+            rotate_bytes<4>(c1, key & 15);
+            out[2] = make_uint4(c1[0], c1[1], c1[2], c1[3]);
+          } else if (LPB == 64) {
+            uint32_t c1[8] = {w[8], w[9], w[10], w[11], w[12], w[13], w[14], w[15]};
+            rotate_bytes<8>(c1, key & 31);
+            out[2] = make_uint4(c1[0], c1[1], c1[2], c1[3]);
+            out[3] = make_uint4(c1[4], c1[5], c1[6], c1[7]);
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before_sync();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after_sync();
+    tmem_dealloc(tbase, (uint32_t)pl.ncols * (A ? 2u : 1u));
+  }
 }
 
 }  // namespace hst

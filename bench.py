@@ -456,7 +456,8 @@ def run_prefill_hash(w, api, caches, device, peak):
     lp = 16 if w.L <= 16 else 32 if w.L <= 32 else 48 if w.L <= 48 else 64
     nbytes = w.pairs * w.N * (2 * w.d * 2 + lp + 2) + w.L * w.P * w.d * 2   # K, V in; ids, norms out
     gbs = nbytes / (ms * 1e-3) / 1e9
-    return {"us": ms * 1e3, "bytes": nbytes, "hbm_gbs": gbs, "frac_of_peak": gbs / peak,
+    kernel = "hash_keys_tcgen05_kernel" if (w.kv_dtype == "bf16" and w.P == 8) else "hash_keys_simt_kernel"
+    return {"kernel": kernel, "us": ms * 1e3, "bytes": nbytes, "hbm_gbs": gbs, "frac_of_peak": gbs / peak,
             "keys_per_s": w.pairs * w.N / (ms * 1e-3)}
 
 

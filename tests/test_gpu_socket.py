@@ -69,6 +69,38 @@ def test_hash_keys_match_oracle(api, name):
     assert total_robust >= 0.99 * w.B * w.Hkv * w.N * w.L
 
 
+# bf16 keys with P = 8 go through the tensor-core prefill kernel: L = 10 pads
+# the last 4-table block and the 16-byte ID row; L = 64 needs two 256-column
+# MMA chunks and leaves room for one key stage; L = 5 at d = 64 pads rows of
+# R past 8L; Ncap not a multiple of 128 leaves a partial last tile.
+@pytest.mark.parametrize("L,d,N,B,Hkv", [(10, 128, 700, 1, 2), (64, 128, 300, 1, 1), (5, 64, 333, 2, 1)])
+def test_hash_keys_tensor_core_shapes(api, L, d, N, B, Hkv):
+    w = wl.shrink(wl.LLAMA_1B, B=B, Hkv=Hkv, Hq=Hkv, d=d, N=N, L=L, P=8, k=N // 10, outlier_channels=0)
+    inp = wl.make_inputs(w, DEV)
+    Ncap = inp["K"].shape[2]
+    ids = api.empty_ids(w.B, w.Hkv, Ncap, w.L, DEV)
+    norms = api.empty_norms(w.B, w.Hkv, Ncap, DEV)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, norms, 0, w.N)
+    # the same keys in two ranges that split a 128-key tile
+    ids2 = api.empty_ids(w.B, w.Hkv, Ncap, w.L, DEV)
+    norms2 = api.empty_norms(w.B, w.Hkv, Ncap, DEV)
+    cut = 77
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids2, norms2, 0, cut)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids2, norms2, cut, w.N - cut)
+    torch.cuda.synchronize()
+    assert torch.equal(ids, ids2) and torch.equal(norms, norms2)
+    gpu_nat = api.ids_to_natural(ids, w.L).cpu().numpy()
+    ref_nat, ref_norms, proj = pa.oracle_socket_cache(inp, w)
+    R = inp["R"].double().cpu().numpy()
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            K = inp["K"][b, h, : w.N].double().cpu().numpy()
+            robust = pa.sign_band(K, R, proj[(b, h)]).reshape(w.N, w.L, w.P).all(axis=2)
+            assert pa.check_ids(gpu_nat[b, h, : w.N], ref_nat[b, h, : w.N], robust) == 0
+            assert np.array_equal(norms[b, h, : w.N].cpu().numpy(), ref_norms[b, h, : w.N])
+    assert np.all(gpu_nat[:, :, w.N:] == 0)
+
+
 def test_hash_keys_append_touches_only_the_range(api):
     w = _w("llama1b_ragged")
     inp = wl.make_inputs(w, DEV)

@@ -91,7 +91,11 @@ typedef enum {
  * K, V: [B][Hkv][Ncap][d] (dtype kv); R: [L*P][d] bf16.
  * ids, norms: outputs in the layouts above. Keys outside the range are not
  * touched, so appending one decoded token is n_begin = N, n_count = 1.
- * The projections accumulate in f32; the norm in f64.
+ * The projections accumulate in f32; the norm in f64. Ranges of more than
+ * 16 keys with bf16 keys and P == 8 run on the tensor cores, shorter ranges
+ * (decode-time appends) on a low-latency kernel; the two add the f32
+ * projection up in different orders, so a key's bit can depend on which one
+ * hashed it only where its projection is within f32 rounding of zero.
  * Requires 1 <= P <= 8, 1 <= L <= 64, L*P <= 512, 0 <= n_begin,
  * n_begin + n_count <= Ncap (n_count == 0 is a no-op).
  */
@@ -215,7 +219,8 @@ int socket_select(const void* Q, sk_dtype q, const void* R, const void* ids, con
  * Hard-hash codes (HATA digest, section 3, with seeded random hyperplanes
  * standing in for the learned hash): for keys n in [n_begin, n_begin+n_count)
  * of every pair, code bit c = [k_n . r_c > 0] for the 128 rows of R128,
- * written to `codes` in the layout above.
+ * written to `codes` in the layout above. The same kernels as
+ * socket_hash_keys with 16 tables of 8 hyperplanes and no values.
  */
 int hata_hash_keys(const void* K, sk_dtype kv, const void* R128, int B, int Hkv, int Ncap,
                    int n_begin, int n_count, int d, void* codes, void* stream);

@@ -762,10 +762,10 @@ int socket_sparse_attend_noalloc(const void* Q, const void* K, const void* V, sk
                 B, Hkv, G, d, need, kNoAllocScratchBytes);
   void* scratch = nullptr;
   SK_TRY(noalloc_scratch_address(&scratch));
-  // zero_counters: the merge counters keep the previous call's contents and
-  // must start at zero; the partials are written before they are read
-  return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, scratch, kNoAllocScratchBytes, false,
-                       true, as_stream(stream), false);
+  // the merge counters keep the previous call's contents and must start at
+  // zero; the partials are written before they are read
+  return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, scratch, kNoAllocScratchBytes,
+                       /*pdl=*/false, /*zero_counters=*/true, as_stream(stream), /*allow_cluster=*/false);
 }
 
 namespace {

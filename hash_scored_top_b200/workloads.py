@@ -18,7 +18,7 @@ stand in for them:
   positions are replaced by 3 * sqrt(d) * q_hat_h + eps, eps ~ N(0, I), where
   q_hat_h is the unit query of head h = kvh * G + (j mod G) -- a key that points
   along the query with a typical key norm (the needle-in-a-haystack idea of
-  the HGA page, section 4 "結果").
+  the HGA page, gist.science/ja/paper/2606.30709, section 4 "結果").
 
 Draw order (one torch.Generator per workload, on the target device): Q, R,
 then for each batch element K[b], V[b] (and xi[b]), then outlier channels,

@@ -21,9 +21,20 @@ Sources, cited by page title and section:
 * HATA digest -- "HATA: Hash-Aware Top-k Attention" (aibr.jp/archives/117328),
   section 3 "中核となる技術的要素" (binary hash codes compared to rank keys).
 
-Functions with no independent pin: none. Every function here is pinned by a
-``-m "not gpu"`` test in ``tests/test_oracle_*.py`` against closed forms,
-invariants, library routines or brute force.
+Pins. Every public function below is named in a ``-m "not gpu"`` test that
+a plausible slip in it would fail; the expected values there are closed
+forms, hand-built fixtures, brute force or scipy routines, never this
+package's own output:
+
+* hash_key_ids, value_norms_f16, bucket_probabilities, group_bucket_table,
+  soft_collision_scores, select_topk, socket_decode_pair:
+  ``tests/test_oracle_socket.py`` (basis-vector fixtures, negation and scale
+  invariance, fsum brute force, the bit-factorisation identity, the tau
+  limits, brute-force top-k with ties, k = N against scipy's softmax);
+* exact_attention, attend_subset, dense_decode, binary_codes,
+  hamming_match_scores: ``tests/test_oracle_attention_hata.py``;
+* hata_decode_pair, socket_decode, hata_decode (the compositions and the
+  query-head -> KV-head mapping): ``tests/test_oracle_compositions.py``.
 """
 
 from .socket_ref import (

@@ -6,7 +6,8 @@ static device array inside the library instead of a caller workspace.
 
 The GPU test calls the new entry point through the C ABI twice in a row, on
 different shapes, and checks each output against socket_sparse_attend with a
-caller workspace, at the tolerance the other attention tests use. It must pass
+caller workspace and against the oracle's attention over the same keys, at
+the tolerance the other attention tests use. It must pass
 in a fresh process (the first call looks up the scratch address) and after
 every other test (the scratch keeps the previous call's contents). The file
 name makes pytest collect it last.
@@ -17,6 +18,7 @@ import ctypes
 import numpy as np
 import pytest
 
+from oracle import attention_ref as ao
 from tests import parity as pa
 
 DEV = "cuda"
@@ -69,10 +71,15 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls(lib):
         api.check_status()
         got, ref = O_new.cpu().numpy(), O_ws.cpu().numpy()
         assert np.isfinite(got).all(), call
+        idx_h = idx.cpu().numpy()
         for p in range(w.B * w.Hkv):
             b, h = divmod(p, w.Hkv)
             rows = slice(h * w.G, (h + 1) * w.G)
             assert pa.row_rel_err(got[b, rows], ref[b, rows]) < pa.out_tol(w), (call, b, h)
+            # and against the oracle's attention over the same subset
+            Qg, K, V = pa.pair_arrays(inp, w, b, h)
+            o_ref = ao.attend_subset(Qg, K, V, idx_h[b, h], w.scale)
+            assert pa.row_rel_err(got[b, rows], o_ref) < pa.out_tol(w), (call, b, h)
 
 
 def test_noalloc_rejects_shapes_beyond_the_static_scratch(lib):

@@ -36,6 +36,7 @@ METRIC = "decode-attention steps/sec and keys scored/sec at N=100K; HBM GB/s vs 
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["attend.cuh", "common.cuh", "score.cuh", "select.cuh", "socket_kernels.cuh", "table.cuh",
                  "hash_kernels.cuh"]
+NOMINAL_HBM_GBS = 8000.0
 
 
 def parse_args():
@@ -48,6 +49,9 @@ def parse_args():
     ap.add_argument("--caches", type=int, default=4, help="independent caches rotated over (L2 defeat)")
     ap.add_argument("--e2e-steps", type=int, default=2000)
     ap.add_argument("--no-extras", action="store_true", help="skip the dense-decode and CPU baselines")
+    ap.add_argument("--no-others", action="store_true", help="skip the records of the other workloads")
+    ap.add_argument("--clock-window", type=float, default=0.5,
+                    help="seconds of untimed replays under the clock sampler right before the timed region")
     return ap.parse_args()
 
 
@@ -111,7 +115,7 @@ class ClockSampler:
         self.uuid = device_uuid
 
     def __enter__(self):
-        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50"]
+        cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "20"]
         if self.uuid:
             cmd += ["-i", self.uuid]
         try:
@@ -119,9 +123,11 @@ class ClockSampler:
         except OSError:
             self.proc = None
         time.sleep(0.3)
+        self.t0 = time.perf_counter()
         return self
 
     def __exit__(self, *exc):
+        self.window_s = time.perf_counter() - self.t0
         self.out = ""
         if self.proc is not None:
             self.proc.terminate()
@@ -146,10 +152,11 @@ class ClockSampler:
             for name, val in zip(names, parts[3:7]):
                 if val.lower().startswith("active"):
                     reasons.add(name)
+        window = round(getattr(self, "window_s", 0.0), 3)
         if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "window_s": window}
         return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
-                "samples": len(sm)}
+                "samples": len(sm), "window_s": window}
 
 
 # ---------------------------------------------------------------- distributed plumbing
@@ -309,12 +316,18 @@ def run_ours(args, world, rank, local):
     dist_barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(uuid) as clk:
-        torch.cuda.nvtx.range_push("timed")
+        # the clock record needs a window of a few hundred ms: untimed replays of
+        # the same step fill it up to the timed region, which follows at once
+        t_end = time.perf_counter() + args.clock_window
+        while time.perf_counter() < t_end:
+            g_step.replay()
+            torch.cuda.synchronize()
         start.record(stream)
+        torch.cuda.nvtx.range_push("timed")
         for _ in range(reps):
             g_step.replay()
-        end.record(stream)
         torch.cuda.nvtx.range_pop()
+        end.record(stream)
         torch.cuda.synchronize()
     dist_barrier(world)
     api.check_status()
@@ -378,16 +391,23 @@ def run_ours(args, world, rank, local):
             "kernel": "socket_select_kernel + socket_attend_kernel (hard hash)" if w.hata else "socket_select_kernel",
             "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
             "peak_kind": peak_kind, "traffic": None if w.hata else profiled_traffic(w.name),
+            "frac_of_nominal_8tbs": achieved / NOMINAL_HBM_GBS,
             "bytes_per_launch": roof_bytes, "avg_launch_us": roof_us,
         },
         "decode_kernels": {
             "kernels": "socket_select_kernel -> socket_attend_kernel (programmatic dependent launch)",
             "avg_us": decode_us, "bytes": rb["decode"], "gbs": rb["decode"] / (decode_us * 1e-6) / 1e9,
             "frac": rb["decode"] / (decode_us * 1e-6) / 1e9 / peak,
+            "frac_of_nominal_8tbs": rb["decode"] / (decode_us * 1e-6) / 1e9 / NOMINAL_HBM_GBS,
         },
         "gpu_launches": 3 * steps,
         "clocks": clocks,
     }
+    if not args.no_others:
+        result["workloads"] = {}
+        for name in wl.WORKLOADS:
+            if name != w.name:
+                result["workloads"][name] = run_workload_record(name, api, wl, device, peak)
     if not args.no_extras and not w.hata:
         result["e2e"] = run_e2e(args, w, api, caches, device, world, ws)
         result["dense_decode"] = run_dense(w, api, caches, device, rb, peak)
@@ -396,6 +416,67 @@ def run_ours(args, world, rank, local):
             result["cpu_baseline"] = cpu_baseline(w, caches[0], sample_pairs=8)
     del g_step, g_dec, g_sel
     return result
+
+
+OTHER_STEPS = {"tiny_f32": 200, "llama3.2-1b_n32k": 200, "llama3.1-8b_n100k": 100, "qwen3-30b_n140k": 50,
+               "hata_n256k": 20}
+
+
+def run_workload_record(name, api, wl, device, peak):
+    """One decode step of another workload, timed step by step with CUDA events
+    (an L2 flush of 256 MB between steps, outside the events): one cache drawn
+    and hashed by the library, then socket_decode_append (or the hard-hash
+    append + decode) over all N keys."""
+    import torch
+    w = wl.WORKLOADS[name]
+    inp = wl.make_inputs(w, device)
+    Ncap = inp["K"].shape[2]
+    O = torch.empty(w.B, w.Hq, w.d, device=device)
+    if w.hata:
+        codes = api.empty_codes(w.B, w.Hkv, Ncap, device)
+        api.hata_hash_keys(inp["K"], inp["R128"], codes, 0, w.N - 1)
+        ws = torch.empty(api.workspace_bytes(api.OP_HATA_DECODE, w.B, w.Hq, w.Hkv, Ncap, w.N, w.d, 16, 8, w.k),
+                         dtype=torch.uint8, device=device)
+
+        def step():
+            api.hata_hash_keys(inp["K"], inp["R128"], codes, w.N - 1, 1)
+            api.hata_decode(inp["Q"], inp["K"], inp["V"], inp["R128"], codes, w.N, w.k, w.scale, O, None, ws)
+    else:
+        ids = api.empty_ids(w.B, w.Hkv, Ncap, w.L, device)
+        norms = api.empty_norms(w.B, w.Hkv, Ncap, device)
+        api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, norms, 0, w.N - 1)
+        ws = torch.empty(api.workspace_bytes(api.OP_DECODE, w.B, w.Hq, w.Hkv, Ncap, w.N, w.d, w.L, w.P, w.k),
+                         dtype=torch.uint8, device=device)
+
+        def step():
+            api.socket_decode_append(inp["Q"], inp["K"], inp["V"], inp["R"], ids, norms, w.N, w.L, w.P, w.tau, w.k,
+                                     w.scale, O, None, ws)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    n = OTHER_STEPS.get(name, 50)
+    for _ in range(3):
+        step()
+    api.check_status()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    for e0, e1 in ev:
+        flush.zero_()
+        e0.record()
+        step()
+        e1.record()
+    torch.cuda.synchronize()
+    api.check_status()
+    times = [e0.elapsed_time(e1) * 1e3 for e0, e1 in ev]
+    us = sum(times) / n
+    rb = required_bytes(w)
+    gbs = rb["step"] / (us * 1e-6) / 1e9
+    rec = {"us_per_step": us, "us_median": statistics.median(times), "steps_per_s": 1e6 / us,
+           "required_bytes_per_step": rb["step"], "hbm_gbs": gbs, "frac_of_peak": gbs / peak,
+           "keys_scored_per_s": w.pairs * w.N / (us * 1e-6), "steps": n,
+           "shape": {"B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "L": w.L, "P": w.P, "k": w.k,
+                     "kv_dtype": w.kv_dtype, "hard_hash": w.hata},
+           "timing": "CUDA events around each step, 256 MB L2 flush between steps outside the events"}
+    del inp, O, ws, flush
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_e2e(args, w, api, caches, device, world, ws):
@@ -501,6 +582,97 @@ def _oracle_pair_inputs(w, cache, pairs):
     return out
 
 
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def host_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def _limit_blas_env(env):
+    for var in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS"):
+        env[var] = "1"
+
+
+def _cpu_worker(i, wname, barrier, queue):
+    """One host core: draws one seeded (batch, kv-head) pair of the workload on
+    the CPU, hashes it with the oracle (prefill, untimed), then times the
+    oracle's decode of that pair between two barriers."""
+    _limit_blas_env(os.environ)
+    from threadpoolctl import threadpool_limits
+    from hash_scored_top_b200 import workloads as wl
+    from oracle import hata_ref as ho
+    from oracle import socket_ref as so
+    w = wl.WORKLOADS[wname]
+    wp = wl.shrink(w, B=1, Hkv=1, Hq=w.G, seed=w.seed + 7919 * (i + 1))
+    inp = wl.make_inputs(wp, "cpu")
+    Qg = inp["Q"][0].double().numpy()
+    K = inp["K"][0, 0, : w.N].float().numpy()
+    V = inp["V"][0, 0, : w.N].float().numpy()
+    with threadpool_limits(1):
+        if w.hata:
+            R = inp["R128"].double().numpy()
+            codes, _ = ho.binary_codes(K, R)
+
+            def decode():
+                ho.hata_decode_pair(Qg, K, V, R, codes, w.k, w.scale)
+        else:
+            R = inp["R"].double().numpy()
+            ids, _ = so.hash_key_ids(K, R, w.L, w.P)
+            norms = so.value_norms_f16(V)
+
+            def decode():
+                so.socket_decode_pair(Qg, K, V, R, ids, norms, w.L, w.P, w.tau, w.k, w.scale)
+        barrier.wait(timeout=600)
+        t0 = time.monotonic()
+        decode()
+        t1 = time.monotonic()
+    queue.put((i, t0, t1))
+
+
+def cpu_baseline_all_cores(w, max_workers=32):
+    """The oracle on every host core at once: one process per core (spawned),
+    each decoding one seeded pair of the workload; the wall time from the first
+    start to the last finish covers that many pairs of a step."""
+    import multiprocessing as mp
+    n = max(1, min(host_cores(), max_workers, w.pairs))
+    ctx = mp.get_context("spawn")
+    barrier = ctx.Barrier(n)
+    queue = ctx.Queue()
+    env_backup = {v: os.environ.get(v) for v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+    _limit_blas_env(os.environ)
+    try:
+        procs = [ctx.Process(target=_cpu_worker, args=(i, w.name, barrier, queue)) for i in range(n)]
+        for p in procs:
+            p.start()
+        res = [queue.get(timeout=900) for _ in range(n)]
+        for p in procs:
+            p.join(60)
+    finally:
+        for var, val in env_backup.items():
+            if val is None:
+                os.environ.pop(var, None)
+            else:
+                os.environ[var] = val
+    wall = max(r[2] for r in res) - min(r[1] for r in res)
+    return {"value": n / (wall * w.pairs), "unit": "decode steps/s", "cores": n, "kind": "oracle",
+            "wall_s": wall,
+            "sample": f"{n} seeded (batch, kv-head) pairs of the workload drawn on the host, one per core "
+                      f"(spawned processes, BLAS 1 thread each), decoded at once; {n} of {w.pairs} pairs of a "
+                      f"step, scaled to a whole step"}
+
+
 def cpu_baseline(w, cache, sample_pairs=8):
     from threadpoolctl import threadpool_limits
     from oracle import socket_ref as so
@@ -514,9 +686,14 @@ def cpu_baseline(w, cache, sample_pairs=8):
                 so.socket_decode_pair(Qg, K, V, R, ids, norms, w.L, w.P, w.tau, w.k, w.scale)
             times.append(time.perf_counter() - t0)
     t = statistics.median(times)
-    return {"value": len(pairs) / (t * w.pairs), "unit": "decode steps/s", "cores": 1, "kind": "oracle",
-            "sample": f"{len(pairs)} of {w.pairs} (batch, kv-head) pairs of one step, median of 3, "
-                      f"float64 numpy, BLAS limited to 1 thread; scaled to a whole step"}
+    single = {"value": len(pairs) / (t * w.pairs), "cores": 1,
+              "sample": f"{len(pairs)} of {w.pairs} (batch, kv-head) pairs of the bench's first cache, "
+                        f"median of 3, float64 numpy, BLAS limited to 1 thread; scaled to a whole step"}
+    out = cpu_baseline_all_cores(w)
+    out["single_core"] = single
+    out["cpu_model"] = cpu_model()
+    out["host_cores"] = host_cores()
+    return out
 
 
 def run_reference(args):
@@ -570,7 +747,11 @@ def run_reference(args):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded, same workload)",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "N": w.N, "L": w.L,
                    "P": w.P, "tau": w.tau, "k": w.k},
-        "cpu_baseline": {"value": value, "unit": "decode steps/s", "cores": 1, "kind": "oracle", "sample": sample},
+        "ms_per_step_extrapolated": True,
+        "extrapolation": f"each timed step decodes {n} keys of one pair; ms_per_step and value scale that time "
+                         f"by {scale:.1f} to a whole step of {w.pairs} pairs x {w.N} keys",
+        "cpu_baseline": {"value": value, "unit": "decode steps/s", "cores": 1, "kind": "oracle", "sample": sample,
+                         "cpu_model": cpu_model()},
         "e2e": {"value": value, "unit": "decode steps/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 

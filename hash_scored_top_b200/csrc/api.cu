@@ -1,6 +1,7 @@
 // C ABI of libhash_scored_top.so: argument validation, launch planning and
 // launches. Every entry point validates on the host before launching
 // anything, allocates nothing, and runs asynchronously on the caller's stream.
+#include <algorithm>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -161,8 +162,11 @@ FusedPlan plan_select(int pairs, int N, int k, int G, int d, int L, int P, bool 
   FusedPlan fp;
   const int nch = table_chunks_of(L);
   const int nblk = (N + 31) / 32;
+  // one CTA per SM for every pair at once, in clusters of at most 8 CTAs
+  // (16-CTA clusters need a free GPC each and do not all fit at once); larger
+  // clusters only when a pair's keys do not fit
   int c = 1;
-  while (c * 2 <= max_c && pairs * c * 2 <= kNumSMs) c *= 2;
+  while (c * 2 <= std::min(max_c, 8) && pairs * c * 2 <= kNumSMs) c *= 2;
   for (; c <= max_c; c *= 2) {
     const int bpc = (nblk + c - 1) / c;
     const int per = ((L + c - 1) / c + 3) & ~3;

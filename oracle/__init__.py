@@ -20,6 +20,8 @@ Sources, cited by page title and section:
   section "理論的基盤" (theoretical foundation) for the tau -> 0 limit.
 * HATA digest -- "HATA: Hash-Aware Top-k Attention" (aibr.jp/archives/117328),
   section 3 "中核となる技術的要素" (binary hash codes compared to rank keys).
+* SOCKET technical summary, "主要な貢献" item 4 and "理論的基盤": the
+  soft-count attention estimator (``estimator_ref``).
 
 Pins. Every public function below is named in a ``-m "not gpu"`` test that
 a plausible slip in it would fail; the expected values there are closed
@@ -34,7 +36,10 @@ package's own output:
 * exact_attention, attend_subset, dense_decode, binary_codes,
   hamming_match_scores: ``tests/test_oracle_attention_hata.py``;
 * hata_decode_pair, socket_decode, hata_decode (the compositions and the
-  query-head -> KV-head mapping): ``tests/test_oracle_compositions.py``.
+  query-head -> KV-head mapping): ``tests/test_oracle_compositions.py``;
+* soft_counts, soft_count_attention: ``tests/test_oracle_estimator.py``
+  (a one-hyperplane case worked with math.exp, the tau -> infinity limit, a
+  pure-Python loop over tables and buckets).
 """
 
 from .socket_ref import (
@@ -49,6 +54,7 @@ from .socket_ref import (
 )
 from .attention_ref import exact_attention, attend_subset, dense_decode
 from .hata_ref import binary_codes, hamming_match_scores, hata_decode_pair, hata_decode
+from .estimator_ref import soft_counts, soft_count_attention
 
 __all__ = [
     "hash_key_ids",
@@ -66,4 +72,6 @@ __all__ = [
     "hamming_match_scores",
     "hata_decode_pair",
     "hata_decode",
+    "soft_counts",
+    "soft_count_attention",
 ]

@@ -19,7 +19,7 @@ from . import _lib
 
 SK_F32, SK_BF16 = 0, 1
 (OP_HASH_KEYS, OP_SCORE, OP_TOPK, OP_SPARSE_ATTEND, OP_DECODE, OP_HATA_HASH, OP_HATA_DECODE, OP_DENSE_DECODE,
- OP_SELECT) = range(9)
+ OP_SELECT, OP_SOFT_COUNT) = range(10)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -295,6 +295,24 @@ def dense_decode(Q, K, V, N: int, scale: float, O, ws=None):
     rc = _lib.lib.dense_decode(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), B, Hq, Hkv, Ncap, N, d, ctypes.c_float(scale),
                                _ptr(O), _ptr(ws), _ws_bytes(ws), _stream())
     _check(rc, "dense_decode")
+
+
+def socket_soft_count_attend(Q, V, R, ids, idx, L: int, P: int, tau: float, O, ws=None):
+    """The soft-count attention estimator over the selected keys idx (see the C header)."""
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = V.shape
+    k = idx.shape[-1]
+    _want(V, Q.dtype, V.shape, "V")
+    _want(R, torch.bfloat16, (L * P, d), "R")
+    _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
+    _want(idx, torch.int32, (B, Hkv, k), "idx")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    if ws is None:              # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_SOFT_COUNT, B, Hq, Hkv, Ncap, k, d, L, P, k), Q.device, ws)
+    rc = _lib.lib.socket_soft_count_attend(_ptr(Q), _ptr(V), _dtype_code(V), _ptr(R), _ptr(ids), _ptr(idx), B, Hq,
+                                           Hkv, Ncap, d, L, P, ctypes.c_float(tau), k, _ptr(O), _ptr(ws),
+                                           _ws_bytes(ws), _stream())
+    _check(rc, "socket_soft_count_attend")
 
 
 def check_status():

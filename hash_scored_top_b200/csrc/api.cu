@@ -14,6 +14,7 @@
 
 #include "../../include/hash_scored_top.h"
 #include "socket_kernels.cuh"
+#include "estimator.cuh"
 #include "hash_tc.cuh"
 
 using namespace hst;
@@ -613,6 +614,45 @@ int hash_launch(const void* K, const void* V, sk_dtype kv, const void* R, int B,
   return check_launch("hash_keys_simt_kernel");
 }
 
+// Soft-count estimator plan: keys per CTA (at most EST_MAX_KEYS, about two
+// CTAs per SM over all pairs) and tables per factor chunk (the largest
+// multiple of 4 whose float64 scratch leaves the whole plan within the
+// shared-memory limit).
+struct EstPlan {
+  int keys_per_split = 0, splits = 0, lchunk = 0;
+  size_t smem = 0;
+};
+
+EstPlan plan_estimator(int pairs, int k, int G, int d, int L, int P) {
+  EstPlan ep;
+  const int want_splits = std::max(1, (2 * kNumSMs + pairs - 1) / pairs);
+  int kps = (k + want_splits - 1) / want_splits;
+  kps = std::max(32, std::min(EST_MAX_KEYS, kps));
+  ep.keys_per_split = kps;
+  ep.splits = (k + kps - 1) / kps;
+  for (int lc = (L + 3) & ~3; lc >= 4; lc -= 4) {
+    const size_t sm = est_smem_bytes(G, d, lc, P);
+    if (sm <= (size_t)SMEM_DYN_MAX) {
+      ep.lchunk = lc;
+      ep.smem = sm;
+      break;
+    }
+  }
+  return ep;
+}
+
+size_t est_ws_bytes(int pairs, int splits, int G, int d) {
+  return align256((size_t)pairs * splits * G * (d + 1) * 4) + align256((size_t)pairs * 4);
+}
+
+template <int D, typename KVT>
+int launch_estimator_t(const EstParams& ep, int pairs, size_t smem, cudaStream_t s) {
+  auto kern = soft_count_attend_kernel<D, KVT>;
+  if (set_kernel_smem(kern, smem) != cudaSuccess) return check_launch("cudaFuncSetAttribute(estimator smem)");
+  kern<<<dim3(pairs, ep.splits), EST_THREADS, smem, s>>>(ep);
+  return check_launch("soft_count_attend_kernel");
+}
+
 }  // namespace
 
 // ================================================================ C ABI
@@ -983,6 +1023,61 @@ int dense_decode(const void* Q, const void* K, const void* V, sk_dtype kv, int B
                        as_stream(stream));
 }
 
+
+int socket_soft_count_attend(const void* Q, const void* V, sk_dtype kv, const void* R, const void* ids, const int* idx,
+                             int B, int Hq, int Hkv, int Ncap, int d, int L, int P, float tau, int k, float* O,
+                             void* ws, size_t ws_bytes, void* stream) {
+  SK_NONNULL(Q);
+  SK_NONNULL(V);
+  SK_NONNULL(R);
+  SK_NONNULL(ids);
+  SK_NONNULL(idx);
+  SK_NONNULL(O);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(V, 16);
+  SK_ALIGNED(R, 16);
+  SK_ALIGNED(ids, 32);
+  SK_TRY(check_dtype(kv));
+  SK_TRY(check_heads(B, Hq, Hkv, d));
+  if (Ncap < 32 || Ncap % 32) return fail(SK_ERR_INVALID_ARG, "Ncap=%d must be a positive multiple of 32", Ncap);
+  SK_TRY(check_tables(L, P, tau));
+  if (k < 1) return fail(SK_ERR_INVALID_ARG, "k=%d must be >= 1", k);
+  const int pairs = B * Hkv, G = Hq / Hkv;
+  if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
+  const EstPlan plan = plan_estimator(pairs, k, G, d, L, P);
+  if (plan.lchunk == 0) return fail(SK_ERR_UNSUPPORTED, "estimator scratch does not fit (G=%d, P=%d)", G, P);
+  const size_t need = est_ws_bytes(pairs, plan.splits, G, d);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
+  EstParams ep;
+  ep.Q = Q;
+  ep.V = V;
+  ep.R = reinterpret_cast<const __nv_bfloat16*>(R);
+  ep.ids = reinterpret_cast<const uint8_t*>(ids);
+  ep.idx = idx;
+  ep.part = reinterpret_cast<float*>(ws);
+  ep.counters = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(ws) +
+                                                align256((size_t)pairs * plan.splits * G * (d + 1) * 4));
+  ep.O = O;
+  ep.Hq = Hq;
+  ep.Hkv = Hkv;
+  ep.Ncap = Ncap;
+  ep.L = L;
+  ep.P = P;
+  ep.k = k;
+  ep.keys_per_split = plan.keys_per_split;
+  ep.splits = plan.splits;
+  ep.lchunk = plan.lchunk;
+  ep.tau = tau;
+  cudaStream_t s = as_stream(stream);
+  const cudaError_t e = cudaMemsetAsync(ep.counters, 0, (size_t)pairs * 4, s);
+  if (e != cudaSuccess) return fail(SK_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
+  if (d == 128) return kv == SK_BF16 ? launch_estimator_t<128, __nv_bfloat16>(ep, pairs, plan.smem, s)
+                                     : launch_estimator_t<128, float>(ep, pairs, plan.smem, s);
+  return kv == SK_BF16 ? launch_estimator_t<64, __nv_bfloat16>(ep, pairs, plan.smem, s)
+                       : launch_estimator_t<64, float>(ep, pairs, plan.smem, s);
+}
+
 size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, int k) {
   const size_t bad = (size_t)-1;
   if (B < 1 || Hq < 1 || Hkv < 1 || Hq % Hkv) return bad;
@@ -1001,6 +1096,10 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
     case SK_OP_DENSE_DECODE:
       if (N < 1) return bad;
       return attend_ws_bytes(pairs, attend_splits(N, pairs, true), G, d);
+    case SK_OP_SOFT_COUNT: {
+      if (k < 1 || G > 8 || L < 1 || L > kMaxL || P < 1 || P > 8) return bad;
+      return est_ws_bytes(pairs, plan_estimator(pairs, k, G, d, L, P).splits, G, d);
+    }
     case SK_OP_SELECT: {
       if (k < 1 || N < 1 || G > 8 || L < 1 || L > kMaxL || P < 1 || P > 8) return bad;
       return select_ws_bytes(plan_select(pairs, N, k, G, d, L, P, false, 8), pairs, Ncap, L);

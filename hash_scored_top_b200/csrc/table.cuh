@@ -117,20 +117,25 @@ struct NoHook {
   __device__ void operator()() const {}
 };
 
-// Computes T_l(b) for the tables l in [l0, l0 + nl) and every bucket b < 2^P.
-// VEC = 1: calls store(b, l, value_f32) once per entry. VEC = 4: calls
-// store(b, l, v, cnt) once per bucket and group of 4 tables l .. l + cnt - 1
-// (groups start at l0 + 4g; cnt < 4 only for the last group), v[0..cnt).
-// Qg points at the G query rows of the pair (row stride D); scratch holds
-// table_scratch_bytes, or table_scratch_dbl_bytes when rows_scratch (16-byte
-// aligned, table_scratch_rows_bytes) is given. All threads of the block must call this; it calls
-// before_store() (all threads, converged) just before the first store and
-// ends with __syncthreads().
-template <int D, typename QT, typename Store, typename Hook = NoHook, int VEC = 1>
-__device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_bfloat16* __restrict__ R, int P,
-                                   float tau, int l0, int nl, void* scratch, Store store,
-                                   unsigned long long* ts = nullptr, Hook before_store = Hook(),
-                                   void* rows_scratch = nullptr) {
+// The per-bit factors of tables [l0, l0 + nl) for every head of the group,
+// float64, left in scratch: p_{h,l0+li}(b) = lo[hl * slo + (b & (nlo - 1))] *
+// hi[hl * shi + (b >> plo)] with hl = h * nl + li.
+struct BucketFactors {
+  const double* lo;
+  const double* hi;
+  int slo, shi, plo, nlo;
+};
+
+// Steps 1-3 of the table build (unit queries, projections on the fp64 tensor
+// cores, per-bit sigmoids, products over the low and high bits). Same
+// arguments as build_bucket_table; all threads of the block call it; it ends
+// with __syncthreads().
+// rows_global = true: the hyperplane rows are read from R in global memory
+// (not staged), so scratch needs only table_scratch_dbl_bytes.
+template <int D, typename QT>
+__device__ BucketFactors bucket_factors(const QT* __restrict__ Qg, int G, const __nv_bfloat16* __restrict__ R, int P,
+                                        float tau, int l0, int nl, void* scratch, unsigned long long* ts = nullptr,
+                                        void* rows_scratch = nullptr, bool rows_global = false) {
   auto tstamp = [&](int ph) {
     if (ts != nullptr && threadIdx.x == 0) {
       ts[blockIdx.x * 24 + ph] = (unsigned long long)clock64();
@@ -147,12 +152,13 @@ __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_
   double* lo = sig + G * nl * P * 2;                    // [G][nl][slo]
   double* hi = lo + G * nl * slo;                       // [G][nl][shi]
   const int ndbl = (G * qpad_row<D>() + G * nl * P * 2 + G * nl * (slo + shi) + 1) & ~1;   // 16-byte aligned rows
-  __nv_bfloat16* rs = rows_scratch ? reinterpret_cast<__nv_bfloat16*>(rows_scratch)        // [nl * P][D]
-                                    : reinterpret_cast<__nv_bfloat16*>(qhat + ndbl);
+  const __nv_bfloat16* rs = rows_global ? R + (size_t)l0 * P * D
+                           : rows_scratch ? reinterpret_cast<const __nv_bfloat16*>(rows_scratch)   // [nl * P][D]
+                                          : reinterpret_cast<const __nv_bfloat16*>(qhat + ndbl);
 
   // 1. unit query rows; this CTA's hyperplane rows
   unit_queries<D>(Qg, G, qhat);
-  stage_rows<D>(R, l0 * P, nl * P, rs);
+  if (!rows_global) stage_rows<D>(R, l0 * P, nl * P, const_cast<__nv_bfloat16*>(rs));
   __syncthreads();
   tstamp(5);
 
@@ -186,6 +192,28 @@ __device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_
   }
   __syncthreads();
   tstamp(13);
+  return BucketFactors{lo, hi, slo, shi, plo, nlo};
+}
+
+// Computes T_l(b) for the tables l in [l0, l0 + nl) and every bucket b < 2^P.
+// VEC = 1: calls store(b, l, value_f32) once per entry. VEC = 4: calls
+// store(b, l, v, cnt) once per bucket and group of 4 tables l .. l + cnt - 1
+// (groups start at l0 + 4g; cnt < 4 only for the last group), v[0..cnt).
+// Qg points at the G query rows of the pair (row stride D); scratch holds
+// table_scratch_bytes, or table_scratch_dbl_bytes when rows_scratch (16-byte
+// aligned, table_scratch_rows_bytes) is given. All threads of the block must call this; it calls
+// before_store() (all threads, converged) just before the first store and
+// ends with __syncthreads().
+template <int D, typename QT, typename Store, typename Hook = NoHook, int VEC = 1>
+__device__ void build_bucket_table(const QT* __restrict__ Qg, int G, const __nv_bfloat16* __restrict__ R, int P,
+                                   float tau, int l0, int nl, void* scratch, Store store,
+                                   unsigned long long* ts = nullptr, Hook before_store = Hook(),
+                                   void* rows_scratch = nullptr) {
+  const int tid = threadIdx.x, nthr = blockDim.x;
+  const BucketFactors bf = bucket_factors<D, QT>(Qg, G, R, P, tau, l0, nl, scratch, ts, rows_scratch);
+  const double* lo = bf.lo;
+  const double* hi = bf.hi;
+  const int slo = bf.slo, shi = bf.shi, plo = bf.plo, nlo = bf.nlo;
 
   // 4. table entries, summed over the group's heads
   before_store();

@@ -80,7 +80,8 @@ typedef enum {
   SK_OP_HATA_HASH = 5,
   SK_OP_HATA_DECODE = 6,
   SK_OP_DENSE_DECODE = 7,
-  SK_OP_SELECT = 8
+  SK_OP_SELECT = 8,
+  SK_OP_SOFT_COUNT = 9
 } sk_op;
 
 /*
@@ -244,6 +245,26 @@ int hata_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const 
 int dense_decode(const void* Q, const void* K, const void* V, sk_dtype kv, int B, int Hq, int Hkv,
                  int Ncap, int N, int d, float scale, float* O, void* ws, size_t ws_bytes,
                  void* stream);
+
+/*
+ * The soft-count attention estimator (SOCKET technical summary, section
+ * 主要な貢献 item 4, the estimator whose end-to-end error the paper bounds,
+ * and section 理論的基盤, the soft score as a kernel estimate): over the
+ * selected keys idx[p] of every pair, each query head h of the pair gets
+ *   O_h = sum_i c_{h,i} v_i / sum_i c_{h,i},  c_{h,i} = sum_l p_{h,l}(id_l(i)),
+ * the soft collision counts of the head's own soft bucket assignment (as in
+ * socket_score, with no value-norm weight) in place of the softmax weights.
+ * Reads the selected keys' values and cached bucket IDs, not their keys.
+ * V: [B][Hkv][Ncap][d] (dtype kv); Q: [B][Hq][d] (dtype kv); R, ids as above;
+ * idx: [B][Hkv][k] int32 in [0, Ncap) (any order; the result does not depend
+ * on it beyond f32 rounding of the sums); O: [B][Hq][d] f32. The counts are
+ * float64, the weighted sums f32 in a fixed order (deterministic).
+ * Requires 1 <= P <= 8, 1 <= L <= 64, tau > 0, k >= 1, G <= 8.
+ * ws: sk_workspace_bytes(SK_OP_SOFT_COUNT, ..., k) bytes.
+ */
+int socket_soft_count_attend(const void* Q, const void* V, sk_dtype kv, const void* R, const void* ids, const int* idx,
+                             int B, int Hq, int Hkv, int Ncap, int d, int L, int P, float tau, int k, float* O,
+                             void* ws, size_t ws_bytes, void* stream);
 
 /* Scratch bytes needed by `op` for these shapes (0 if none). Arguments an
  * op does not use are ignored. Returns (size_t)-1 for invalid shapes. */

@@ -69,8 +69,9 @@ def required_bytes(w) -> dict:
     attend = w.pairs * w.k * (2 * w.d * 2 + 4) + q_bytes + o_bytes           # index list + K/V rows in, O out
     decode = select + attend - w.pairs * w.k * 4 - q_bytes                   # the index list stays in L2
     append = w.pairs * (2 * w.d * 2 + lp + nb) + r_bytes                     # new K/V row read, ids + norm written
+    estimate = w.pairs * w.k * (w.d * 2 + lp + 4) + q_bytes + r_bytes + o_bytes  # index list, V rows, their IDs
     return {"select": select, "attend": attend, "decode": decode, "step": decode + append,
-            "dense": w.pairs * w.N * 2 * w.d * 2 + q_bytes + o_bytes}
+            "dense": w.pairs * w.N * 2 * w.d * 2 + q_bytes + o_bytes, "estimate": estimate}
 
 
 def load_peaks() -> tuple[float, str]:
@@ -412,6 +413,7 @@ def run_ours(args, world, rank, local):
         result["e2e"] = run_e2e(args, w, api, caches, device, world, ws)
         result["dense_decode"] = run_dense(w, api, caches, device, rb, peak)
         result["prefill_hash"] = run_prefill_hash(w, api, caches, device, peak)
+        result["soft_count_estimator"] = run_estimator(w, api, caches, device, rb, peak)
         if rank == 0 and world == 1:
             result["cpu_baseline"] = cpu_baseline(w, caches[0], sample_pairs=8)
     del g_step, g_dec, g_sel
@@ -540,6 +542,44 @@ def run_prefill_hash(w, api, caches, device, peak):
     kernel = "hash_keys_tcgen05_kernel" if (w.kv_dtype == "bf16" and w.P == 8) else "hash_keys_simt_kernel"
     return {"kernel": kernel, "us": ms * 1e3, "bytes": nbytes, "hbm_gbs": gbs, "frac_of_peak": gbs / peak,
             "keys_per_s": w.pairs * w.N / (ms * 1e-3)}
+
+
+def run_estimator(w, api, caches, device, rb, peak):
+    """The soft-count attention estimator over each cache's selected keys
+    (selection done once per cache, untimed), the caches taken in turn."""
+    import torch
+    Ncap = caches[0]["K"].shape[2]
+    idxs = []
+    for c in caches:
+        idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=device)
+        api.socket_select(c["Q"], c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k, idx)
+        idxs.append(idx)
+    O = torch.empty(w.B, w.Hq, w.d, device=device)
+    ws = torch.empty(api.workspace_bytes(api.OP_SOFT_COUNT, w.B, w.Hq, w.Hkv, Ncap, w.k, w.d, w.L, w.P, w.k),
+                     dtype=torch.uint8, device=device)
+    n, warm = 100, 5
+
+    def est(i):
+        c = caches[i % len(caches)]
+        api.socket_soft_count_attend(c["Q"], c["V"], c["R"], c["ids"], idxs[i % len(caches)], w.L, w.P, w.tau, O,
+                                     ws)
+
+    for i in range(warm):
+        est(i)
+    torch.cuda.synchronize()
+    api.check_status()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for i in range(n):
+        est(i)
+    e.record()
+    torch.cuda.synchronize()
+    api.check_status()
+    us = s.elapsed_time(e) * 1e3 / n
+    gbs = rb["estimate"] / (us * 1e-6) / 1e9
+    return {"kernel": "soft_count_attend_kernel", "us": us, "bytes": rb["estimate"], "hbm_gbs": gbs,
+            "frac_of_peak": gbs / peak, "frac_of_nominal_8tbs": gbs / NOMINAL_HBM_GBS,
+            "launch": f"plain API calls, {len(caches)} caches in turn, each with its own selected index list"}
 
 
 def run_dense(w, api, caches, device, rb, peak):

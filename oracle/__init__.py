@@ -22,6 +22,10 @@ Sources, cited by page title and section:
   section 3 "中核となる技術的要素" (binary hash codes compared to rank keys).
 * SOCKET technical summary, "主要な貢献" item 4 and "理論的基盤": the
   soft-count attention estimator (``estimator_ref``).
+* Tactic digest -- "Tactic: Adaptive Sparse Attention with Clustering and
+  Distribution Fitting for Long-Context LLMs" (aibr.jp/archives/79195),
+  section 3 "中核となる技術的要素" (the cumulative score target): the
+  adaptive k, and per-query-head index sets (``selection_ref``).
 
 Pins. Every public function below is named in a ``-m "not gpu"`` test that
 a plausible slip in it would fail; the expected values there are closed
@@ -39,7 +43,11 @@ package's own output:
   query-head -> KV-head mapping): ``tests/test_oracle_compositions.py``;
 * soft_counts, soft_count_attention: ``tests/test_oracle_estimator.py``
   (a one-hyperplane case worked with math.exp, the tau -> infinity limit, a
-  pure-Python loop over tables and buckets).
+  pure-Python loop over tables and buckets);
+* per_head_scores, socket_decode_pair_per_head, adaptive_k, select_adaptive,
+  socket_decode_pair_adaptive: ``tests/test_oracle_selection.py`` (uniform
+  and geometric closed forms, hand-built ties and clamps, a pure-Python
+  greedy loop, the one-head and equal-heads reductions, scipy's softmax).
 """
 
 from .socket_ref import (
@@ -55,6 +63,13 @@ from .socket_ref import (
 from .attention_ref import exact_attention, attend_subset, dense_decode
 from .hata_ref import binary_codes, hamming_match_scores, hata_decode_pair, hata_decode
 from .estimator_ref import soft_counts, soft_count_attention
+from .selection_ref import (
+    per_head_scores,
+    socket_decode_pair_per_head,
+    adaptive_k,
+    select_adaptive,
+    socket_decode_pair_adaptive,
+)
 
 __all__ = [
     "hash_key_ids",
@@ -74,4 +89,9 @@ __all__ = [
     "hata_decode",
     "soft_counts",
     "soft_count_attention",
+    "per_head_scores",
+    "socket_decode_pair_per_head",
+    "adaptive_k",
+    "select_adaptive",
+    "socket_decode_pair_adaptive",
 ]

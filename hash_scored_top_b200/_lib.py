@@ -39,6 +39,10 @@ SIGNATURES = {
     "hata_decode": (_i, [_p, _p, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _z, _p]),
     "dense_decode": (_i, [_p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _z, _p]),
     "socket_soft_count_attend": (_i, [_p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _i, _p, _p, _z, _p]),
+    "socket_decode_heads": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _f, _p, _p, _p,
+                                 _z, _p]),
+    "socket_decode_adaptive": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _f, _i, _i,
+                                    _f, _p, _p, _p, _p, _z, _p]),
     "sk_workspace_bytes": (_z, [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "sk_check_status": (_i, [_p]),
     "sk_profile_phases": (_i, [_p]),

@@ -19,7 +19,7 @@ from . import _lib
 
 SK_F32, SK_BF16 = 0, 1
 (OP_HASH_KEYS, OP_SCORE, OP_TOPK, OP_SPARSE_ATTEND, OP_DECODE, OP_HATA_HASH, OP_HATA_DECODE, OP_DENSE_DECODE,
- OP_SELECT, OP_SOFT_COUNT) = range(10)
+ OP_SELECT, OP_SOFT_COUNT, OP_DECODE_HEADS, OP_DECODE_ADAPTIVE, OP_DECODE_ADAPTIVE_HEADS) = range(13)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -220,6 +220,49 @@ def socket_decode(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k:
                                 Ncap, N, d, L, P, ctypes.c_float(tau), k, ctypes.c_float(scale), _ptr(O),
                                 _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
     _check(rc, "socket_decode")
+
+
+def socket_decode_heads(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k: int, scale: float, O,
+                        idx_out=None, ws=None):
+    """The decode step with one index set per query head; idx_out: [B, Hq, k]."""
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = K.shape
+    _want(K, Q.dtype, K.shape, "K")
+    _want(V, Q.dtype, K.shape, "V")
+    _want(R, torch.bfloat16, (L * P, d), "R")
+    _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
+    _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    if idx_out is not None:
+        _want(idx_out, torch.int32, (B, Hq, k), "idx_out")
+    ws = _workspace(workspace_bytes(OP_DECODE_HEADS, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    rc = _lib.lib.socket_decode_heads(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R), _ptr(ids), _ptr(norms), B,
+                                      Hq, Hkv, Ncap, N, d, L, P, ctypes.c_float(tau), k, ctypes.c_float(scale),
+                                      _ptr(O), _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
+    _check(rc, "socket_decode_heads")
+
+
+def socket_decode_adaptive(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, mass: float, k_min: int,
+                           k_max: int, scale: float, O, idx, kcount, per_head: bool = False, ws=None):
+    """The decode step with the adaptive k; idx: [B, U, k_max], kcount: [B, U] (U = Hkv, or Hq per head)."""
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = K.shape
+    U = Hq if per_head else Hkv
+    _want(K, Q.dtype, K.shape, "K")
+    _want(V, Q.dtype, K.shape, "V")
+    _want(R, torch.bfloat16, (L * P, d), "R")
+    _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
+    _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    _want(idx, torch.int32, (B, U, k_max), "idx")
+    _want(kcount, torch.int32, (B, U), "kcount")
+    op = OP_DECODE_ADAPTIVE_HEADS if per_head else OP_DECODE_ADAPTIVE
+    ws = _workspace(workspace_bytes(op, B, Hq, Hkv, Ncap, N, d, L, P, k_max), Q.device, ws)
+    rc = _lib.lib.socket_decode_adaptive(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R), _ptr(ids), _ptr(norms),
+                                         B, Hq, Hkv, Ncap, N, d, L, P, ctypes.c_float(tau), int(bool(per_head)),
+                                         ctypes.c_float(mass), k_min, k_max, ctypes.c_float(scale), _ptr(O),
+                                         _ptr(idx), _ptr(kcount), _ptr(ws), _ws_bytes(ws), _stream())
+    _check(rc, "socket_decode_adaptive")
 
 
 def socket_decode_append(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k: int, scale: float, O,

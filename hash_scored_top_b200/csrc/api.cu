@@ -15,6 +15,7 @@
 #include "../../include/hash_scored_top.h"
 #include "socket_kernels.cuh"
 #include "estimator.cuh"
+#include "adaptive.cuh"
 #include "hash_tc.cuh"
 
 using namespace hst;
@@ -315,8 +316,9 @@ int launch_score_t(const ScoreParams& sp, dim3 grid, cudaStream_t s) {
 }
 
 int launch_score(const float* T, const void* ids, const void* norms, int pairs, int Ncap, int N, int L, float* scores,
-                 cudaStream_t s) {
+                 cudaStream_t s, int pair_div = 1) {
   ScoreParams sp;
+  sp.pair_div = pair_div;
   sp.T = T;
   sp.ids = reinterpret_cast<const uint8_t*>(ids);
   sp.norms = reinterpret_cast<const __half*>(norms);
@@ -374,6 +376,48 @@ int launch_topk(const float* scores, int pairs, int Ncap, int N, int k, int* idx
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, tp);
   if (e != cudaSuccess) return fail(SK_ERR_CUDA, "top-k launch: %s", cudaGetErrorString(e));
   return check_launch("socket_topk_kernel");
+}
+
+// Adaptive top-k: one cluster per unit, the unit's scores split over its CTAs.
+int launch_adaptive_topk(const float* scores, int units, int Ncap, int N, float mass, int k_min, int k_max, int* idx,
+                         int* kcount, cudaStream_t s) {
+  const int cap = (int)((SMEM_DYN_MAX - kAdaptFixedBytes) / 4);
+  int C = 0;
+  for (int c = 1; c <= max_cluster_size(); c *= 2)
+    if ((N + c - 1) / c <= cap) {
+      C = c;
+      break;
+    }
+  if (C == 0) return fail(SK_ERR_UNSUPPORTED, "adaptive top-k: N=%d too large", N);
+  AdaptParams ap;
+  ap.scores = scores;
+  ap.idx = idx;
+  ap.kcount = kcount;
+  ap.Ncap = Ncap;
+  ap.N = N;
+  ap.k_min = k_min;
+  ap.k_max = k_max;
+  ap.C = C;
+  ap.keys_per_cta = (N + C - 1) / C;
+  ap.mass = mass;
+  const size_t smem = kAdaptFixedBytes + (size_t)ap.keys_per_cta * 4;
+  auto kern = socket_adaptive_topk_kernel;
+  if (set_kernel_smem(kern, smem, C > 8) != cudaSuccess) return check_launch("cudaFuncSetAttribute(adaptive smem)");
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(units * C, 1, 1);
+  cfg.blockDim = dim3(FUSED_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ap);
+  if (e != cudaSuccess) return fail(SK_ERR_CUDA, "adaptive top-k launch: %s", cudaGetErrorString(e));
+  return check_launch("socket_adaptive_topk_kernel");
 }
 
 // Clusters of S CTAs (1, S, 1) that fit on the GPU at once with this launch
@@ -461,12 +505,17 @@ int launch_attend_t(AttendParams ap, int pairs, int G, bool pdl, bool cluster, c
 // (at most max_cluster_size() splits); otherwise the splits merge through
 // workspace ws (partials + counters). zero_counters: clear the counters first
 // (standalone calls); otherwise the selection kernel did.
+// pair_div / counts: see AttendParams (units per cache pair; per-unit list
+// lengths).
 int launch_attend(const void* Q, const void* K, const void* V, sk_dtype kv, const int* idx, int B, int Hq, int Hkv,
                   int Ncap, int n, int d, float scale, float* O, void* ws, size_t ws_bytes, bool pdl,
-                  bool zero_counters, cudaStream_t s, bool allow_cluster = true) {
+                  bool zero_counters, cudaStream_t s, bool allow_cluster = true, int pair_div = 1,
+                  const int* counts = nullptr) {
   const int pairs = B * Hkv, G = Hq / Hkv;
   if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
   AttendParams ap;
+  ap.pair_div = pair_div;
+  ap.counts = counts;
   ap.Q = Q;
   ap.K = K;
   ap.V = V;
@@ -817,10 +866,15 @@ namespace {
 // The decode step: selection kernel (tables, scores, exact top-k -> index list)
 // then the attention kernel (programmatic dependent launch), or the unfused
 // chain when the selection cannot keep a pair's keys on chip.
+// per_head: every query head is its own unit (its own table, index set and
+// attention); the kernels then see Hq "KV heads" of group size 1, each unit
+// reading the cache of KV head h / G.
 int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, const void* ids,
-                const void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k,
-                float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, bool hata, bool attend,
-                cudaStream_t s, bool after_append = false) {
+                const void* norms, int B, int Hq, int Hkv_cache, int Ncap, int N, int d, int L, int P, float tau,
+                int k, float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, bool hata, bool attend,
+                cudaStream_t s, bool after_append = false, bool per_head = false) {
+  const int pair_div = per_head ? Hq / Hkv_cache : 1;
+  const int Hkv = per_head ? Hq : Hkv_cache;
   const int pairs = B * Hkv, G = Hq / Hkv;
   if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
   const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, hata, max_cluster_size());
@@ -838,11 +892,11 @@ int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const 
     int* idx = idx_out ? idx_out : reinterpret_cast<int*>(w);
     w += align256((size_t)pairs * k * 4);
     SK_TRY(launch_tables(Q, kv, R, B, Hq, Hkv, d, L, P, tau, T, s));
-    SK_TRY(launch_score(T, ids, norms, pairs, Ncap, N, L, scores, s));
+    SK_TRY(launch_score(T, ids, norms, pairs, Ncap, N, L, scores, s, pair_div));
     SK_TRY(launch_topk(scores, pairs, Ncap, N, k, idx, s));
     if (!attend) return SK_OK;
     return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, w,
-                         attend_ws_bytes(pairs, attend_splits(k, pairs, false), G, d), false, true, s);
+                         attend_ws_bytes(pairs, attend_splits(k, pairs, false), G, d), false, true, s, true, pair_div);
   }
   int* idx = idx_out ? idx_out : reinterpret_cast<int*>(w);
   const int splits = attend_splits(k, pairs, false);
@@ -874,10 +928,45 @@ int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const 
   p.chunk = fp.chunk;
   p.tau = tau;
   p.scale = scale;
+  p.pair_div = pair_div;
   SK_TRY(launch_select(p, pairs, d, kv, hata, after_append, s));
   if (!attend) return SK_OK;
   return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, w, attend_ws_bytes(pairs, splits, G, d),
-                       true, false, s);
+                       true, false, s, true, pair_div);
+}
+
+// Workspace of the adaptive decode chain (units = B Hkv or B Hq): tables,
+// scores, then the attention workspace planned for k_max keys per unit.
+size_t adaptive_ws_bytes(int B, int Hq, int Hu, int Ncap, int d, int L, int k_max) {
+  const int units = B * Hu, G = Hq / Hu;
+  return align256(table_image_bytes(units, L)) + align256((size_t)units * Ncap * 4) +
+         attend_ws_bytes(units, attend_splits(k_max, units, false), G, d);
+}
+
+// The adaptive decode: bucket tables -> scores -> adaptive top-k -> attention
+// over each unit's kcount keys.
+int adaptive_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, const void* ids,
+                  const void* norms, int B, int Hq, int Hkv_cache, int Ncap, int N, int d, int L, int P, float tau,
+                  bool per_head, float mass, int k_min, int k_max, float scale, float* O, int* idx, int* kcount,
+                  void* ws, size_t ws_bytes, cudaStream_t s) {
+  const int pair_div = per_head ? Hq / Hkv_cache : 1;
+  const int Hu = per_head ? Hq : Hkv_cache;
+  const int units = B * Hu, G = Hq / Hu;
+  if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
+  const size_t need = adaptive_ws_bytes(B, Hq, Hu, Ncap, d, L, k_max);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
+  char* w = reinterpret_cast<char*>(ws);
+  float* T = reinterpret_cast<float*>(w);
+  w += align256(table_image_bytes(units, L));
+  float* scores = reinterpret_cast<float*>(w);
+  w += align256((size_t)units * Ncap * 4);
+  SK_TRY(launch_tables(Q, kv, R, B, Hq, Hu, d, L, P, tau, T, s));
+  SK_TRY(launch_score(T, ids, norms, units, Ncap, N, L, scores, s, pair_div));
+  SK_TRY(launch_adaptive_topk(scores, units, Ncap, N, mass, k_min, k_max, idx, kcount, s));
+  return launch_attend(Q, K, V, kv, idx, B, Hq, Hu, Ncap, k_max, d, scale, O, w,
+                       attend_ws_bytes(units, attend_splits(k_max, units, false), G, d), false, true, s, true,
+                       pair_div, kcount);
 }
 
 }  // namespace
@@ -962,6 +1051,62 @@ int socket_select(const void* Q, sk_dtype q, const void* R, const void* ids, con
   if (k < 1 || k > N) return fail(SK_ERR_INVALID_ARG, "k=%d must be in [1, N=%d]", k, N);
   return decode_impl(Q, nullptr, nullptr, q, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, 0.f, nullptr, idx,
                      ws, ws_bytes, false, false, as_stream(stream));
+}
+
+int socket_decode_heads(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, const void* ids,
+                        const void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau,
+                        int k, float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  SK_NONNULL(Q);
+  SK_NONNULL(K);
+  SK_NONNULL(V);
+  SK_NONNULL(R);
+  SK_NONNULL(ids);
+  SK_NONNULL(norms);
+  SK_NONNULL(O);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(K, 16);
+  SK_ALIGNED(V, 16);
+  SK_ALIGNED(R, 16);
+  SK_ALIGNED(ids, 32);
+  SK_ALIGNED(norms, 2);
+  SK_TRY(check_dtype(kv));
+  SK_TRY(check_heads(B, Hq, Hkv, d));
+  SK_TRY(check_cache(Ncap, N));
+  SK_TRY(check_tables(L, P, tau));
+  if (k < 1 || k > N) return fail(SK_ERR_INVALID_ARG, "k=%d must be in [1, N=%d]", k, N);
+  return decode_impl(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, scale, O, idx_out, ws, ws_bytes,
+                     false, true, as_stream(stream), false, /*per_head=*/true);
+}
+
+int socket_decode_adaptive(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, const void* ids,
+                           const void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau,
+                           int per_head, float mass, int k_min, int k_max, float scale, float* O, int* idx,
+                           int* kcount, void* ws, size_t ws_bytes, void* stream) {
+  SK_NONNULL(Q);
+  SK_NONNULL(K);
+  SK_NONNULL(V);
+  SK_NONNULL(R);
+  SK_NONNULL(ids);
+  SK_NONNULL(norms);
+  SK_NONNULL(O);
+  SK_NONNULL(idx);
+  SK_NONNULL(kcount);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(K, 16);
+  SK_ALIGNED(V, 16);
+  SK_ALIGNED(R, 16);
+  SK_ALIGNED(ids, 32);
+  SK_ALIGNED(norms, 2);
+  SK_TRY(check_dtype(kv));
+  SK_TRY(check_heads(B, Hq, Hkv, d));
+  SK_TRY(check_cache(Ncap, N));
+  SK_TRY(check_tables(L, P, tau));
+  if (per_head != 0 && per_head != 1) return fail(SK_ERR_INVALID_ARG, "per_head=%d must be 0 or 1", per_head);
+  if (!(mass > 0.f && mass <= 1.f)) return fail(SK_ERR_INVALID_ARG, "mass must be in (0, 1]");
+  if (k_min < 1 || k_min > k_max || k_max > N)
+    return fail(SK_ERR_INVALID_ARG, "need 1 <= k_min (%d) <= k_max (%d) <= N (%d)", k_min, k_max, N);
+  return adaptive_impl(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, per_head == 1, mass, k_min,
+                       k_max, scale, O, idx, kcount, ws, ws_bytes, as_stream(stream));
 }
 
 int hata_hash_keys(const void* K, sk_dtype kv, const void* R128, int B, int Hkv, int Ncap, int n_begin, int n_count,
@@ -1117,6 +1262,20 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
       const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, op == SK_OP_HATA_DECODE, 8);
       if (fp.C > 0 || op == SK_OP_HATA_DECODE) return decode_ws_bytes(B, Hq, Hkv, k, d);
       return chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
+    }
+    case SK_OP_DECODE_HEADS: {
+      // one unit per query head: Hq "KV heads" of group size 1
+      if (k < 1 || N < 1 || L < 1 || L > kMaxL || P < 1 || P > 8) return bad;
+      const FusedPlan fp = plan_select(B * Hq, N, k, 1, d, L, P, false, 8);
+      if (fp.C > 0) return decode_ws_bytes(B, Hq, Hq, k, d);
+      return chain_ws_bytes(B, Hq, Hq, Ncap, d, L, k);
+    }
+    case SK_OP_DECODE_ADAPTIVE:
+    case SK_OP_DECODE_ADAPTIVE_HEADS: {
+      // k is k_max
+      const int Hu = op == SK_OP_DECODE_ADAPTIVE_HEADS ? Hq : Hkv;
+      if (k < 1 || N < 1 || Hq / Hu > 8 || L < 1 || L > kMaxL || P < 1 || P > 8) return bad;
+      return adaptive_ws_bytes(B, Hq, Hu, Ncap, d, L, k);
     }
     default:
       return bad;

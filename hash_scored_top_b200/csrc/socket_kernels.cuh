@@ -58,6 +58,10 @@ struct FusedParams {
   unsigned long long* phase_ts;   // optional: [grid][PHASES] clock stamps (profiling)
   int Hq, Hkv, Ncap, N, L, P, k, C, blocks_per_cta, chunk;
   float tau, scale;
+  // units per cache pair: 1 (one index set per KV head), or G when every
+  // query head is its own unit (Hkv then counts query heads); the cached
+  // IDs, norms, keys and values of unit u are those of pair u / pair_div
+  int pair_div = 1;
 };
 
 constexpr int PHASES = 24;
@@ -276,7 +280,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
   const int blk1 = min(nblk_pair, blk0 + p.blocks_per_cta);
   const int n_local = max(0, min(p.N, blk1 * 32) - blk0 * 32);
   const int nb = max(0, (blk1 - blk0 - warp + FUSED_WARPS - 1) / FUSED_WARPS);
-  const size_t pair_keys = (size_t)pair * p.Ncap;
+  const size_t pair_keys = (size_t)(pair / p.pair_div) * p.Ncap;
   const uint8_t* ids_pair = p.ids + pair_keys * LP;
   const __half* norms_pair = p.norms + pair_keys;
 
@@ -458,8 +462,9 @@ struct ScoreParams {
   const float* T;
   const uint8_t* ids;
   const __half* norms;
-  float* scores;
+  float* scores;           // [units][Ncap]
   int Ncap, N, blocks_per_cta;
+  int pair_div = 1;        // units per cache pair, as in FusedParams
 };
 
 // grid = (pairs, chunks); the pair's table image is copied to 64 KB-aligned
@@ -483,7 +488,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_score_kernel(const Sc
     reinterpret_cast<float4*>(t)[e] = __ldg(src + e);
   __syncthreads();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  const size_t pair_keys = (size_t)pair * p.Ncap;
+  const size_t pair_keys = (size_t)(pair / p.pair_div) * p.Ncap;
   const int nblk = (p.N + 31) / 32;
   const int blk0 = blockIdx.y * p.blocks_per_cta;
   const int blk1 = min(nblk, blk0 + p.blocks_per_cta);
@@ -492,7 +497,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_score_kernel(const Sc
     KeyIds<LP> k;
     load_key_ids<LP, true>(k, p.ids + (pair_keys + key) * LP, p.norms + pair_keys + key);
     const float s = score_key<LP, true>(k, tbl + 4u * lane, tbl + TABLE_BYTES + 4u * lane);
-    if (key < p.N) p.scores[pair_keys + key] = s;
+    if (key < p.N) p.scores[(size_t)pair * p.Ncap + key] = s;
   }
 }
 
@@ -548,6 +553,8 @@ struct AttendParams {
   unsigned long long* phase_ts;  // optional: [pairs * splits][PHASES] clock stamps (profiling)
   int Hq, Hkv, Ncap, n, keys_per_split, splits;
   float scale;
+  int pair_div = 1;        // units per cache pair, as in FusedParams
+  const int* counts = nullptr;   // optional [units]: keys of each unit's list (<= n)
 };
 
 __device__ __forceinline__ void attend_stamp(unsigned long long* ts, int phase) {
@@ -588,8 +595,7 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
   const int G = p.Hq / p.Hkv;
   const int b = pair / p.Hkv, kvh = pair % p.Hkv;
   const int i0 = split * p.keys_per_split;
-  const int cnt = max(0, min(p.n - i0, p.keys_per_split));
-  const size_t pair_keys = (size_t)pair * p.Ncap;
+  const size_t pair_keys = (size_t)(pair / p.pair_div) * p.Ncap;
   const KVT* Qg = reinterpret_cast<const KVT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
   const uint32_t base = smem_u32(dyn);
   AttendSmem as;
@@ -613,6 +619,10 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
   attend_stamp(p.phase_ts, 1);
   asm volatile("griddepcontrol.wait;" ::: "memory");   // the key list is complete from here on
   attend_stamp(p.phase_ts, 2);
+  // this unit's list length: n, or its count (clamped to [0, n]) when the
+  // lists have per-unit lengths
+  const int n_unit = p.counts ? min(max(__ldcg(p.counts + pair), 0), p.n) : p.n;
+  const int cnt = max(0, min(n_unit - i0, p.keys_per_split));
   const KVT* Kp = reinterpret_cast<const KVT*>(p.K) + pair_keys * D;
   const KVT* Vp = reinterpret_cast<const KVT*>(p.V) + pair_keys * D;
   float *cM, *cL, *cO;

@@ -81,7 +81,10 @@ typedef enum {
   SK_OP_HATA_DECODE = 6,
   SK_OP_DENSE_DECODE = 7,
   SK_OP_SELECT = 8,
-  SK_OP_SOFT_COUNT = 9
+  SK_OP_SOFT_COUNT = 9,
+  SK_OP_DECODE_HEADS = 10,
+  SK_OP_DECODE_ADAPTIVE = 11,        /* k is k_max */
+  SK_OP_DECODE_ADAPTIVE_HEADS = 12   /* k is k_max */
 } sk_op;
 
 /*
@@ -215,6 +218,50 @@ int socket_decode_append(const void* Q, const void* K, const void* V, sk_dtype k
 int socket_select(const void* Q, sk_dtype q, const void* R, const void* ids, const void* norms,
                   int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k,
                   int* idx, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * socket_decode with one index set per QUERY head: head h scores the keys of
+ * KV head h / G with its own soft assignment, score_{h,n} = norm_n *
+ * sum_l p_{h,l}(id_l(n)) (no sum over the group), takes its own exact top-k
+ * (ties to the lower index) and attends over it. With G = 1 this is
+ * socket_decode. The same two kernels run with the B * Hq query heads as
+ * their units, each reading its KV head's cache, so the group's bucket IDs are
+ * read once per query head (from L2 after the first). idx_out (nullable):
+ * [B][Hq][k] ascending. Requires what socket_decode requires except G <= 8.
+ * ws: sk_workspace_bytes(SK_OP_DECODE_HEADS, ...) bytes.
+ */
+int socket_decode_heads(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R,
+                        const void* ids, const void* norms, int B, int Hq, int Hkv, int Ncap, int N,
+                        int d, int L, int P, float tau, int k, float scale, float* O, int* idx_out,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Decode with an adaptive k (Tactic digest, "Tactic: Adaptive Sparse
+ * Attention with Clustering and Distribution Fitting for Long-Context LLMs",
+ * aibr.jp/archives/79195, section 3 中核となる技術的要素: tokens are taken
+ * until their cumulative score reaches a target), applied to the soft
+ * collision scores: for every unit (per_head = 0: a KV head's group, scored
+ * by the group-summed table as in socket_decode; per_head = 1: one query
+ * head, as in socket_decode_heads),
+ *   k = min{ k : sum of the k largest scores >= mass * sum of all N scores },
+ * clamped to [k_min, k_max], then the exact top-k (ties to the lower index)
+ * and attention over it. idx: [units][k_max] int32, the first kcount[u]
+ * entries ascending and the rest -1; kcount: [units] int32; units = B * Hkv
+ * or B * Hq. The float64 score sum is formed in a fixed order and the
+ * cumulative masses are 64-bit fixed-point integers, so the result is
+ * deterministic; it can differ from an exact-arithmetic k only where the
+ * target lies within the scores' f32 rounding of a cumulative sum. Four
+ * kernels: bucket tables, scores (to ws), the adaptive top-k (one cluster per
+ * unit), attention. Requires 0 < mass <= 1, 1 <= k_min <= k_max <= N, and
+ * what socket_decode requires (G <= 8 only for per_head = 0).
+ * ws: sk_workspace_bytes(SK_OP_DECODE_ADAPTIVE or SK_OP_DECODE_ADAPTIVE_HEADS,
+ * ..., k = k_max) bytes.
+ */
+int socket_decode_adaptive(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R,
+                           const void* ids, const void* norms, int B, int Hq, int Hkv, int Ncap, int N,
+                           int d, int L, int P, float tau, int per_head, float mass, int k_min,
+                           int k_max, float scale, float* O, int* idx, int* kcount, void* ws,
+                           size_t ws_bytes, void* stream);
 
 /*
  * Hard-hash codes (HATA digest, section 3, with seeded random hyperplanes

@@ -663,42 +663,66 @@ int hash_launch(const void* K, const void* V, sk_dtype kv, const void* R, int B,
   return check_launch("hash_keys_simt_kernel");
 }
 
-// Soft-count estimator plan: keys per CTA (at most EST_MAX_KEYS, about two
-// CTAs per SM over all pairs) and tables per factor chunk (the largest
-// multiple of 4 whose float64 scratch leaves the whole plan within the
-// shared-memory limit).
+// Soft-count estimator plan: keys per CTA of the attend kernel. Two CTAs per
+// SM when a CTA's factor image and at least 32 keys fit half the shared
+// memory, else one; then as many keys per CTA as make the grid about one wave
+// (at least 64), within the shared memory.
 struct EstPlan {
-  int keys_per_split = 0, splits = 0, lchunk = 0;
+  int keys_per_split = 0, splits = 0;
   size_t smem = 0;
 };
 
-EstPlan plan_estimator(int pairs, int k, int G, int d, int L, int P) {
+EstPlan plan_estimator(int pairs, int k, int G, int d, int L, int kv_bytes) {
   EstPlan ep;
-  const int want_splits = std::max(1, (2 * kNumSMs + pairs - 1) / pairs);
-  int kps = (k + want_splits - 1) / want_splits;
-  kps = std::max(32, std::min(EST_MAX_KEYS, kps));
+  const size_t fixed = est_smem_plan(G, d, L, 0, kv_bytes).total + 64;   // plus alignment slack
+  const size_t per_key = est_bytes_per_key(G, d, L, kv_bytes);
+  const size_t half = (size_t)SMEM_DYN_MAX / 2 - 1024;
+  const bool two = fixed + 32 * per_key <= half;
+  const size_t budget = two ? half : (size_t)SMEM_DYN_MAX;
+  if (fixed + per_key > budget) return ep;                           // nothing fits
+  const int fit = (int)((budget - fixed) / per_key);
+  const int ctas = (two ? 2 : 1) * kNumSMs;
+  const int want_splits = std::max(1, (ctas + pairs - 1) / pairs);
+  // at least 64 keys per CTA (fewer splits to merge), as far as they fit
+  int kps = std::min(fit, std::max(64, (k + want_splits - 1) / want_splits));
+  kps = std::max(1, kps);
   ep.keys_per_split = kps;
   ep.splits = (k + kps - 1) / kps;
-  for (int lc = (L + 3) & ~3; lc >= 4; lc -= 4) {
-    const size_t sm = est_smem_bytes(G, d, lc, P);
-    if (sm <= (size_t)SMEM_DYN_MAX) {
-      ep.lchunk = lc;
-      ep.smem = sm;
-      break;
-    }
-  }
+  ep.smem = est_smem_plan(G, d, L, kps, kv_bytes).total;
   return ep;
 }
 
-size_t est_ws_bytes(int pairs, int splits, int G, int d) {
-  return align256((size_t)pairs * splits * G * (d + 1) * 4) + align256((size_t)pairs * 4);
+// Workspace of the estimator: the factor image, the split partials, the counters.
+size_t est_factor_bytes(int pairs, int G, int L) { return align256((size_t)pairs * G * L * EST_F * 4); }
+size_t est_part_bytes(int pairs, int splits, int G, int d) { return align256((size_t)pairs * splits * G * (d + 1) * 4); }
+size_t est_ws_bytes(int pairs, int splits, int G, int d, int L) {
+  return est_factor_bytes(pairs, G, L) + est_part_bytes(pairs, splits, G, d) + align256((size_t)pairs * 4);
 }
 
 template <int D, typename KVT>
-int launch_estimator_t(const EstParams& ep, int pairs, size_t smem, cudaStream_t s) {
+int launch_estimator_t(const EstFactorParams& fp, const EstParams& ep, int pairs, size_t smem, cudaStream_t s) {
+  const int G = fp.Hq / fp.Hkv;
+  auto fk = est_factor_kernel<D, KVT>;
+  const size_t fsm = est_factor_smem_bytes(G, D, fp.P);
+  if (set_kernel_smem(fk, fsm) != cudaSuccess) return check_launch("cudaFuncSetAttribute(estimator factors smem)");
+  fk<<<dim3(pairs, (fp.L + EST_TABLES_PER_CTA - 1) / EST_TABLES_PER_CTA), 256, fsm, s>>>(fp);
+  SK_TRY(check_launch("est_factor_kernel"));
   auto kern = soft_count_attend_kernel<D, KVT>;
   if (set_kernel_smem(kern, smem) != cudaSuccess) return check_launch("cudaFuncSetAttribute(estimator smem)");
-  kern<<<dim3(pairs, ep.splits), EST_THREADS, smem, s>>>(ep);
+  // programmatic dependent of the factor kernel: the copies of the keys' ID
+  // and value rows overlap it; the factor image is read after its completion
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(pairs, ep.splits, 1);
+  cfg.blockDim = dim3(EST_THREADS, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ep);
+  if (e != cudaSuccess) return fail(SK_ERR_CUDA, "estimator launch: %s", cudaGetErrorString(e));
   return check_launch("soft_count_attend_kernel");
 }
 
@@ -1189,20 +1213,29 @@ int socket_soft_count_attend(const void* Q, const void* V, sk_dtype kv, const vo
   if (k < 1) return fail(SK_ERR_INVALID_ARG, "k=%d must be >= 1", k);
   const int pairs = B * Hkv, G = Hq / Hkv;
   if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
-  const EstPlan plan = plan_estimator(pairs, k, G, d, L, P);
-  if (plan.lchunk == 0) return fail(SK_ERR_UNSUPPORTED, "estimator scratch does not fit (G=%d, P=%d)", G, P);
-  const size_t need = est_ws_bytes(pairs, plan.splits, G, d);
+  const EstPlan plan = plan_estimator(pairs, k, G, d, L, kv == SK_BF16 ? 2 : 4);
+  if (plan.splits == 0) return fail(SK_ERR_UNSUPPORTED, "estimator scratch does not fit (G=%d, L=%d)", G, L);
+  const size_t need = est_ws_bytes(pairs, plan.splits, G, d, L);
   if (ws == nullptr || ws_bytes < need)
     return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
+  char* w = reinterpret_cast<char*>(ws);
+  EstFactorParams fp;
+  fp.Q = Q;
+  fp.R = reinterpret_cast<const __nv_bfloat16*>(R);
+  fp.F = reinterpret_cast<float*>(w);
+  fp.Hq = Hq;
+  fp.Hkv = Hkv;
+  fp.L = L;
+  fp.P = P;
+  fp.tau = tau;
   EstParams ep;
-  ep.Q = Q;
   ep.V = V;
-  ep.R = reinterpret_cast<const __nv_bfloat16*>(R);
   ep.ids = reinterpret_cast<const uint8_t*>(ids);
   ep.idx = idx;
-  ep.part = reinterpret_cast<float*>(ws);
-  ep.counters = reinterpret_cast<unsigned int*>(reinterpret_cast<char*>(ws) +
-                                                align256((size_t)pairs * plan.splits * G * (d + 1) * 4));
+  ep.F = fp.F;
+  ep.part = reinterpret_cast<float*>(w + est_factor_bytes(pairs, G, L));
+  ep.counters = reinterpret_cast<unsigned int*>(w + est_factor_bytes(pairs, G, L) +
+                                                est_part_bytes(pairs, plan.splits, G, d));
   ep.O = O;
   ep.Hq = Hq;
   ep.Hkv = Hkv;
@@ -1212,15 +1245,14 @@ int socket_soft_count_attend(const void* Q, const void* V, sk_dtype kv, const vo
   ep.k = k;
   ep.keys_per_split = plan.keys_per_split;
   ep.splits = plan.splits;
-  ep.lchunk = plan.lchunk;
-  ep.tau = tau;
+  ep.phase_ts = g_phase_ts;
   cudaStream_t s = as_stream(stream);
   const cudaError_t e = cudaMemsetAsync(ep.counters, 0, (size_t)pairs * 4, s);
   if (e != cudaSuccess) return fail(SK_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
-  if (d == 128) return kv == SK_BF16 ? launch_estimator_t<128, __nv_bfloat16>(ep, pairs, plan.smem, s)
-                                     : launch_estimator_t<128, float>(ep, pairs, plan.smem, s);
-  return kv == SK_BF16 ? launch_estimator_t<64, __nv_bfloat16>(ep, pairs, plan.smem, s)
-                       : launch_estimator_t<64, float>(ep, pairs, plan.smem, s);
+  if (d == 128) return kv == SK_BF16 ? launch_estimator_t<128, __nv_bfloat16>(fp, ep, pairs, plan.smem, s)
+                                     : launch_estimator_t<128, float>(fp, ep, pairs, plan.smem, s);
+  return kv == SK_BF16 ? launch_estimator_t<64, __nv_bfloat16>(fp, ep, pairs, plan.smem, s)
+                       : launch_estimator_t<64, float>(fp, ep, pairs, plan.smem, s);
 }
 
 size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, int k) {
@@ -1243,7 +1275,10 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
       return attend_ws_bytes(pairs, attend_splits(N, pairs, true), G, d);
     case SK_OP_SOFT_COUNT: {
       if (k < 1 || G > 8 || L < 1 || L > kMaxL || P < 1 || P > 8) return bad;
-      return est_ws_bytes(pairs, plan_estimator(pairs, k, G, d, L, P).splits, G, d);
+      // the split count (hence the partials) depends on the value dtype:
+      // the larger of the two
+      const int sp = std::max(plan_estimator(pairs, k, G, d, L, 2).splits, plan_estimator(pairs, k, G, d, L, 4).splits);
+      return est_ws_bytes(pairs, sp, G, d, L);
     }
     case SK_OP_SELECT: {
       if (k < 1 || N < 1 || G > 8 || L < 1 || L > kMaxL || P < 1 || P > 8) return bad;

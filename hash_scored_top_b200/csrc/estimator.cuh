@@ -8,14 +8,23 @@
 // Only the selected keys' values and cached bucket IDs are read, not their
 // keys.
 //
-// grid = (pairs, splits), EST_THREADS threads; CTA (pair, s) takes keys
-// idx[s * keys_per_split ..]. Pass A, over chunks of lchunk tables: the
-// heads' per-bit factors of the chunk, then every key's counts (lanes over
-// tables, a fixed xor-tree sum over the lanes) added to a float64 count per
-// (key, head) in shared memory. Pass B: warps over keys, lanes over value
+// Two kernels. est_factor_kernel, grid (pairs, table chunks): the per-bit
+// factors of every head's soft assignment (the float64 lo / hi products of
+// table.cuh, rounded to f32), written once per pair to a factor image in the
+// workspace, F[pair][h][l][32] (lo at [0, 16), hi at [16, 32)).
+// soft_count_attend_kernel, grid (pairs, splits), launched as the factor
+// kernel's programmatic dependent: CTA (pair, s) takes keys
+// idx[s * keys_per_split ..], and first issues asynchronous copies of all
+// their ID rows and value rows into shared memory (every copy of the CTA in
+// flight at once), then, once the factor kernel is done, of the pair's factor
+// image. Pass A, one thread per key: c_{h,i} summed over the tables in f32
+// (all lanes of a warp read the same factor row, so the lookups do not
+// conflict; f32, whose count is within (L + 2) 2^-24 of the exact one,
+// because the SM's float64 pipe is far narrower). Pass B: warps over keys,
+// lanes over value
 // columns, f32 accumulation of c v and of c. The warps' partials are added in
-// warp order; the splits' partials go to the workspace and the last CTA of the
-// pair (counted with an atomic) adds them in split order and divides.
+// warp order; the splits' partials go to the workspace and the last CTA of
+// the pair (counted with an atomic) adds them in split order and divides.
 #pragma once
 
 #include "hash_kernels.cuh"
@@ -24,105 +33,251 @@
 
 namespace hst {
 
-constexpr int EST_THREADS = 512;
+constexpr int EST_THREADS = 256;
 constexpr int EST_WARPS = EST_THREADS / 32;
-constexpr int EST_MAX_KEYS = 512;      // keys per CTA at most (their counts stay in shared memory)
+constexpr int EST_F = 32;              // floats per (head, table) in the factor image
+constexpr int EST_TABLES_PER_CTA = 4;  // tables per CTA of the factor kernel
 
-struct EstParams {
+struct EstFactorParams {
   const void* Q;
-  const void* V;
   const __nv_bfloat16* R;
-  const uint8_t* ids;
-  const int* idx;                // [pairs][k]
-  float* part;                   // [pairs][splits][G][D + 1]: (sum c, sum c v) per head
-  unsigned int* counters;        // [pairs], zero on entry, left zero
-  float* O;                      // [B][Hq][D]
-  int Hq, Hkv, Ncap, L, P, k, keys_per_split, splits, lchunk;
+  float* F;                      // [pairs][G][L][EST_F]
+  int Hq, Hkv, L, P;
   float tau;
 };
 
-// Shared bytes: the factor scratch of one chunk (reused for the warps'
-// partials), then the counts, then a flag word.
-__host__ __device__ inline size_t est_region_a_bytes(int G, int d, int lchunk, int P) {
-  const size_t f = table_scratch_dbl_bytes(G, d, lchunk, P);
-  const size_t w = (size_t)EST_WARPS * G * (d + 1) * 4;
-  return ((f > w ? f : w) + 15) & ~(size_t)15;
+struct EstParams {
+  const void* V;
+  const uint8_t* ids;
+  const int* idx;                // [pairs][k]
+  const float* F;                // factor image
+  float* part;                   // [pairs][splits][G][D + 1]: (sum c, sum c v) per head
+  unsigned int* counters;        // [pairs], zero on entry, left zero
+  float* O;                      // [B][Hq][D]
+  unsigned long long* phase_ts;  // optional: [pairs * splits][24] clock stamps (profiling)
+  int Hq, Hkv, Ncap, L, P, k, keys_per_split, splits;
+};
+
+// Profiling stamps of the attend kernel (see sk_profile_phases): the SM clock
+// at each phase; the global timer at the start (slot 22) and the end (23).
+__device__ __forceinline__ void est_stamp(unsigned long long* ts, int phase) {
+  if (ts != nullptr && threadIdx.x == 0) {
+    const size_t cta = (size_t)blockIdx.y * gridDim.x + blockIdx.x;
+    ts[cta * 24 + phase] = (unsigned long long)clock64();
+    if (phase == 0 || phase == 7) {
+      unsigned long long t;
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+      ts[cta * 24 + 22 + (phase == 7)] = t;
+    }
+  }
 }
-__host__ __device__ inline size_t est_smem_bytes(int G, int d, int lchunk, int P) {
-  return est_region_a_bytes(G, d, lchunk, P) + (size_t)EST_MAX_KEYS * G * 8 + 16;
+
+// Shared bytes of the factor kernel (bucket_factors with staged rows).
+__host__ __device__ inline size_t est_factor_smem_bytes(int G, int d, int P) {
+  return table_scratch_bytes(G, d, EST_TABLES_PER_CTA, P);
+}
+
+__host__ __device__ inline size_t est_align16(size_t x) { return (x + 15) & ~(size_t)15; }
+
+// Shared-memory plan of the attend kernel for `kps` keys per CTA: the factor
+// image (reused for the warps' partials), the counts, the key indices, the
+// staged ID rows and value rows, a flag word. Offsets in bytes.
+struct EstSmem {
+  size_t counts, keys, idrows, vrows, flag, total;
+};
+__host__ __device__ inline EstSmem est_smem_plan(int G, int d, int L, int kps, int kv_bytes) {
+  EstSmem s;
+  const size_t f = (size_t)G * L * EST_F * 4;
+  const size_t w = (size_t)EST_WARPS * G * (d + 1) * 4;
+  s.counts = est_align16(f > w ? f : w);
+  s.keys = s.counts + est_align16((size_t)kps * G * 4);
+  s.idrows = s.keys + est_align16((size_t)kps * 4);
+  s.vrows = s.idrows + (size_t)kps * ids_bytes_per_key(L);
+  s.flag = s.vrows + (size_t)kps * d * kv_bytes;
+  s.total = s.flag + 16;
+  return s;
+}
+// Bytes of shared memory per key in the plan above (for the host's choice of kps).
+__host__ __device__ inline size_t est_bytes_per_key(int G, int d, int L, int kv_bytes) {
+  return (size_t)G * 4 + 4 + ids_bytes_per_key(L) + (size_t)d * kv_bytes;
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
+template <int D, typename QT>
+__global__ void __launch_bounds__(256) est_factor_kernel(const EstFactorParams p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  // the attend kernel, launched as this kernel's programmatic dependent, may
+  // start its copies now: it reads the factor image only after
+  // griddepcontrol.wait, i.e. after this grid has completed
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+  const int pair = blockIdx.x;
+  const int l0 = blockIdx.y * EST_TABLES_PER_CTA;
+  const int nl = min(EST_TABLES_PER_CTA, p.L - l0);
+  if (nl <= 0) return;                         // uniform over the CTA
+  const int G = p.Hq / p.Hkv;
+  const int b = pair / p.Hkv, kvh = pair % p.Hkv;
+  const QT* Qg = reinterpret_cast<const QT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
+  const BucketFactors bf = bucket_factors<D, QT>(Qg, G, p.R, p.P, p.tau, l0, nl, smem);
+  const int nhi = bf.shi - 1;
+  float* F = p.F + (size_t)pair * G * p.L * EST_F;
+  for (int e = threadIdx.x; e < G * nl * EST_F; e += blockDim.x) {
+    const int hl = e / EST_F, j = e % EST_F;   // hl = h * nl + li
+    const int h = hl / nl, li = hl % nl;
+    double v = 0.0;
+    if (j < 16) {
+      if (j < bf.nlo) v = bf.lo[hl * bf.slo + j];
+    } else if (j - 16 < nhi) {
+      v = bf.hi[hl * bf.shi + (j - 16)];
+    }
+    F[((size_t)h * p.L + l0 + li) * EST_F + j] = (float)v;
+  }
 }
 
 template <typename KVT>
-__device__ __forceinline__ void load_row4(const KVT* row, int lane, float (&v)[4]);
+__device__ __forceinline__ void row4_from_smem(const unsigned char* row, int lane, float (&v)[4]);
 template <>
-__device__ __forceinline__ void load_row4<__nv_bfloat16>(const __nv_bfloat16* row, int lane, float (&v)[4]) {
-  const uint2 w = __ldg(reinterpret_cast<const uint2*>(row) + lane);
+__device__ __forceinline__ void row4_from_smem<__nv_bfloat16>(const unsigned char* row, int lane, float (&v)[4]) {
+  const uint2 w = reinterpret_cast<const uint2*>(row)[lane];
   v[0] = bf16lo_to_f32(w.x);
   v[1] = bf16hi_to_f32(w.x);
   v[2] = bf16lo_to_f32(w.y);
   v[3] = bf16hi_to_f32(w.y);
 }
 template <>
-__device__ __forceinline__ void load_row4<float>(const float* row, int lane, float (&v)[4]) {
-  const float4 w = __ldg(reinterpret_cast<const float4*>(row) + lane);
+__device__ __forceinline__ void row4_from_smem<float>(const unsigned char* row, int lane, float (&v)[4]) {
+  const float4 w = reinterpret_cast<const float4*>(row)[lane];
   v[0] = w.x;
   v[1] = w.y;
   v[2] = w.z;
   v[3] = w.w;
 }
+template <typename KVT>
+__device__ __forceinline__ void row2_from_smem(const unsigned char* row, int lane, float (&v)[4]) {
+  const KVT* r = reinterpret_cast<const KVT*>(row);
+  v[0] = to_f32(r[2 * lane]);
+  v[1] = to_f32(r[2 * lane + 1]);
+  v[2] = v[3] = 0.f;
+}
 
 template <int D, typename KVT>
-__global__ void __launch_bounds__(EST_THREADS, 1) soft_count_attend_kernel(const EstParams p) {
+__global__ void __launch_bounds__(EST_THREADS, 2) soft_count_attend_kernel(const EstParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int VPL = D / 32;                        // value columns per lane (2 or 4)
+  constexpr int ROW = D * (int)sizeof(KVT);          // bytes of a value row
   const int pair = blockIdx.x, split = blockIdx.y;
   const int G = p.Hq / p.Hkv;
   const int b = pair / p.Hkv, kvh = pair % p.Hkv;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int L = p.L;
   const int i0 = split * p.keys_per_split;
   const int cnt = max(0, min(p.k - i0, p.keys_per_split));
   const size_t pair_keys = (size_t)pair * p.Ncap;
-  const KVT* Qg = reinterpret_cast<const KVT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
-  const int* list = p.idx + (size_t)pair * p.k + i0;
-  const int LPB = ids_bytes_per_key(p.L);
-  const size_t dbl = est_region_a_bytes(G, D, p.lchunk, p.P);
-  double* cnts = reinterpret_cast<double*>(smem + dbl);      // [cnt][G]
-  unsigned int* last_flag = reinterpret_cast<unsigned int*>(smem + dbl + (size_t)EST_MAX_KEYS * G * 8);
-  for (int e = tid; e < cnt * G; e += EST_THREADS) cnts[e] = 0.0;
+  const int LPB = ids_bytes_per_key(L);
+  const EstSmem sp = est_smem_plan(G, D, L, p.keys_per_split, (int)sizeof(KVT));
+  float* fs = reinterpret_cast<float*>(smem);                    // [G][L][EST_F]
+  float* cnts = reinterpret_cast<float*>(smem + sp.counts);      // [cnt][G]
+  int* keys_s = reinterpret_cast<int*>(smem + sp.keys);          // [cnt]
+  unsigned char* idrows = smem + sp.idrows;                      // [cnt][LPB]
+  unsigned char* vrows = smem + sp.vrows;                        // [cnt][ROW]
+  unsigned int* last_flag = reinterpret_cast<unsigned int*>(smem + sp.flag);
 
-  // ---- pass A: counts, table chunk by table chunk
-  for (int l0 = 0; l0 < p.L; l0 += p.lchunk) {
-    const int nl = min(p.lchunk, p.L - l0);
-    const BucketFactors bf = bucket_factors<D, KVT>(Qg, G, p.R, p.P, p.tau, l0, nl, smem, nullptr, nullptr, true);
-    for (int j = warp; j < cnt; j += EST_WARPS) {
-      const int key = min(max(__ldg(list + j), 0), p.Ncap - 1);
-      const uint8_t* idrow = p.ids + (pair_keys + key) * LPB;
-      // lane t: table l0 + t (and l0 + t + 32)
-      int idv[2] = {0, 0};
+  est_stamp(p.phase_ts, 0);
+  // ---- staging: the key list, then every ID row and value row of the CTA
+  const int* list = p.idx + (size_t)pair * p.k + i0;
+  for (int j = tid; j < cnt; j += EST_THREADS) keys_s[j] = min(max(__ldg(list + j), 0), p.Ncap - 1);
+  __syncthreads();
+  est_stamp(p.phase_ts, 1);
+  {
+    const int id_chunks = LPB / 16, v_chunks = ROW / 16;
+    const uint32_t id_base = smem_u32(idrows), v_base = smem_u32(vrows);
+    for (int e = tid; e < cnt * id_chunks; e += EST_THREADS) {
+      const int j = e / id_chunks, c = e % id_chunks;
+      cp_async16(id_base + (uint32_t)(j * LPB + 16 * c), p.ids + (pair_keys + keys_s[j]) * LPB + 16 * c);
+    }
+    const unsigned char* V = reinterpret_cast<const unsigned char*>(p.V);
+    for (int e = tid; e < cnt * v_chunks; e += EST_THREADS) {
+      const int j = e / v_chunks, c = e % v_chunks;
+      cp_async16(v_base + (uint32_t)(j * ROW + 16 * c), V + (pair_keys + keys_s[j]) * ROW + 16 * c);
+    }
+    cp_async_commit();
+    est_stamp(p.phase_ts, 2);
+    // the factor image is written by the factor kernel: copy it only once
+    // that grid has completed (a no-op wait for an ordinary launch)
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+    est_stamp(p.phase_ts, 3);
+    const float* F = p.F + (size_t)pair * G * L * EST_F;
+    const uint32_t f_base = smem_u32(fs);
+    for (int e = tid; e < G * L * EST_F / 4; e += EST_THREADS) cp_async16(f_base + 16u * e, F + 4 * e);
+    cp_async_commit();
+    cp_async_wait_all();
+  }
+  __syncthreads();
+  est_stamp(p.phase_ts, 4);
+
+  // ---- pass A: counts, one thread per key. Inside chunk c (tables 32c ..)
+  // the ID of table 32c + t sits at byte 32c + (t - key) mod S. Eight tables
+  // at a time: their IDs and factor pairs are loaded together, their
+  // probabilities (lo * hi) added as a fixed tree, then to the running count.
+  // The factors are float64 results rounded to f32, and the count is an f32
+  // sum: its relative error stays below (L + 2) 2^-24.
+  const int plo = p.P / 2;
+  const int mlo = (1 << plo) - 1;
+  for (int j = tid; j < cnt; j += EST_THREADS) {
+    const int key = keys_s[j];
+    const unsigned char* row = idrows + (size_t)j * LPB;
+    float c[8];
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int li = lane + 32 * r;
-        if (li < nl) idv[r] = idrow[id_byte_pos(p.L, l0 + li, key)];
-      }
-      for (int h = 0; h < G; ++h) {
-        double c = 0.0;
+    for (int h = 0; h < 8; ++h) c[h] = 0.f;
+    for (int ch = 0; 32 * ch < L; ++ch) {
+      const int S = id_chunk_size(L, ch);
+      const int nt = min(S, L - 32 * ch);
+      const int p0 = (S - key % S) % S;              // byte of table 32c + 0
+      for (int t0 = 0; t0 < nt; t0 += 8) {
+        // every load is unconditional (no branches in the unrolled body): a
+        // table past the chunk's last reads table nt - 1 and is masked out
+        int idv[8];
+        bool live[8];
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {
-          const int li = lane + 32 * r;
-          if (li < nl) {
-            const int hl = h * nl + li;
-            c += bf.lo[hl * bf.slo + (idv[r] & (bf.nlo - 1))] * bf.hi[hl * bf.shi + (idv[r] >> bf.plo)];
+        for (int u = 0; u < 8; ++u) {
+          const int t = min(t0 + u, nt - 1);
+          int pos = p0 + t;
+          pos = pos >= S ? pos - S : pos;
+          idv[u] = (int)row[32 * ch + pos];
+          live[u] = t0 + u < nt;
+        }
+        const float* fr = fs + (size_t)(32 * ch) * EST_F;
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+          if (h < G) {
+            const float* f = fr + (size_t)h * L * EST_F;
+            float q[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              const int t = min(t0 + u, nt - 1);
+              const float a = f[t * EST_F + (idv[u] & mlo)];
+              const float bq = f[t * EST_F + 16 + (idv[u] >> plo)];
+              q[u] = live[u] ? a * bq : 0.f;
+            }
+            c[h] += ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));
           }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(FULL, c, o);
-        if (lane == 0) cnts[j * G + h] += c;
       }
     }
-    __syncthreads();         // the factor scratch is reused by the next chunk
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+      if (h < G) cnts[j * G + h] = c[h];
   }
+  __syncthreads();
+  est_stamp(p.phase_ts, 5);
 
-  // ---- pass B: sum c v and sum c per head, warps over keys, lanes over columns
+  // ---- pass B: sum c v and sum c per head, warps over keys (each warp's
+  // keys in increasing order), lanes over value columns; four keys' rows
+  // and counts loaded at a time
   float acc[8][VPL];
   float csum[8];
 #pragma unroll
@@ -131,30 +286,35 @@ __global__ void __launch_bounds__(EST_THREADS, 1) soft_count_attend_kernel(const
 #pragma unroll
     for (int e = 0; e < VPL; ++e) acc[h][e] = 0.f;
   }
-  for (int j = warp; j < cnt; j += EST_WARPS) {
-    const int key = min(max(__ldg(list + j), 0), p.Ncap - 1);
-    const KVT* vrow = reinterpret_cast<const KVT*>(p.V) + (pair_keys + key) * D;
-    float v[4];
-    if constexpr (VPL == 4) {
-      load_row4<KVT>(vrow, lane, v);
-    } else {
-      const float a0 = to_f32(vrow[2 * lane]), a1 = to_f32(vrow[2 * lane + 1]);
-      v[0] = a0;
-      v[1] = a1;
-      v[2] = v[3] = 0.f;
+  for (int j0 = warp; j0 < cnt; j0 += 4 * EST_WARPS) {
+    float v[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int j = min(j0 + u * EST_WARPS, cnt - 1);
+      if constexpr (VPL == 4) {
+        row4_from_smem<KVT>(vrows + (size_t)j * ROW, lane, v[u]);
+      } else {
+        row2_from_smem<KVT>(vrows + (size_t)j * ROW, lane, v[u]);
+      }
     }
 #pragma unroll
-    for (int h = 0; h < 8; ++h) {
-      if (h < G) {
-        const float c = (float)cnts[j * G + h];
-        csum[h] += c;
+    for (int u = 0; u < 4; ++u) {
+      const int j = j0 + u * EST_WARPS;
+      if (j < cnt) {                                 // uniform over the warp
 #pragma unroll
-        for (int e = 0; e < VPL; ++e) acc[h][e] = fmaf(c, v[e], acc[h][e]);
+        for (int h = 0; h < 8; ++h) {
+          if (h < G) {
+            const float cf = cnts[j * G + h];
+            csum[h] += cf;
+#pragma unroll
+            for (int e = 0; e < VPL; ++e) acc[h][e] = fmaf(cf, v[u][e], acc[h][e]);
+          }
+        }
       }
     }
   }
   __syncthreads();
-  // warp partials into the (dead) factor scratch: [warp][G][D + 1]
+  // warp partials into the (dead) factor image: [warp][G][D + 1]
   float* wp = reinterpret_cast<float*>(smem);
   const int stride = G * (D + 1);
 #pragma unroll
@@ -174,22 +334,40 @@ __global__ void __launch_bounds__(EST_THREADS, 1) soft_count_attend_kernel(const
   }
   __threadfence();
   __syncthreads();
+  est_stamp(p.phase_ts, 6);
   if (tid == 0) *last_flag = (atomicAdd(&p.counters[pair], 1u) == (unsigned)p.splits - 1u) ? 1u : 0u;
   __syncthreads();
-  if (*last_flag == 0u) return;
+  if (*last_flag == 0u) {
+    est_stamp(p.phase_ts, 7);
+    return;
+  }
   // ---- last CTA of the pair: splits in order, then the division
   __threadfence();
   const float* part = p.part + (size_t)pair * p.splits * stride;
   for (int e = tid; e < G * D; e += EST_THREADS) {
     const int h = e / D, dv = e % D;
     float cs = 0.f, o = 0.f;
-    for (int s = 0; s < p.splits; ++s) {
-      cs += __ldcg(part + (size_t)s * stride + h * (D + 1));
-      o += __ldcg(part + (size_t)s * stride + h * (D + 1) + 1 + dv);
+    // eight splits' values loaded at a time, then added in split order
+    for (int s0 = 0; s0 < p.splits; s0 += 8) {
+      float a[8], bv[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int sp_ = min(s0 + u, p.splits - 1);
+        a[u] = __ldcg(part + (size_t)sp_ * stride + h * (D + 1));
+        bv[u] = __ldcg(part + (size_t)sp_ * stride + h * (D + 1) + 1 + dv);
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (s0 + u < p.splits) {
+          cs += a[u];
+          o += bv[u];
+        }
+      }
     }
     p.O[((size_t)b * p.Hq + kvh * G + h) * D + dv] = o / cs;
   }
   if (tid == 0) p.counters[pair] = 0u;
+  est_stamp(p.phase_ts, 7);
 }
 
 }  // namespace hst

@@ -304,8 +304,12 @@ int dense_decode(const void* Q, const void* K, const void* V, sk_dtype kv, int B
  * Reads the selected keys' values and cached bucket IDs, not their keys.
  * V: [B][Hkv][Ncap][d] (dtype kv); Q: [B][Hq][d] (dtype kv); R, ids as above;
  * idx: [B][Hkv][k] int32 in [0, Ncap) (any order; the result does not depend
- * on it beyond f32 rounding of the sums); O: [B][Hq][d] f32. The counts are
- * float64, the weighted sums f32 in a fixed order (deterministic).
+ * on it beyond f32 rounding of the sums); O: [B][Hq][d] f32. The soft
+ * assignment's factors are float64 rounded to f32; the counts (relative
+ * error below (L + 2) 2^-24) and the weighted sums are f32 sums in a fixed
+ * order (deterministic). Two
+ * kernels: the heads' soft-assignment factors once per pair (into ws), then
+ * the counts and weighted sums, split over the keys.
  * Requires 1 <= P <= 8, 1 <= L <= 64, tau > 0, k >= 1, G <= 8.
  * ws: sk_workspace_bytes(SK_OP_SOFT_COUNT, ..., k) bytes.
  */

@@ -26,6 +26,9 @@ Sources, cited by page title and section:
   Distribution Fitting for Long-Context LLMs" (aibr.jp/archives/79195),
   section 3 "中核となる技術的要素" (the cumulative score target): the
   adaptive k, and per-query-head index sets (``selection_ref``).
+* HATA digest, sections 3 and 4 (the offloaded KV cache), and the HGA page,
+  section 3 (hot and routed pages): the paged / host-resident K/V pool
+  (``paged_ref``).
 
 Pins. Every public function below is named in a ``-m "not gpu"`` test that
 a plausible slip in it would fail; the expected values there are closed
@@ -47,7 +50,11 @@ package's own output:
 * per_head_scores, socket_decode_pair_per_head, adaptive_k, select_adaptive,
   socket_decode_pair_adaptive: ``tests/test_oracle_selection.py`` (uniform
   and geometric closed forms, hand-built ties and clamps, a pure-Python
-  greedy loop, the one-head and equal-heads reductions, scipy's softmax).
+  greedy loop, the one-head and equal-heads reductions, scipy's softmax);
+* paged_rows, attend_subset_paged, socket_decode_pair_paged:
+  ``tests/test_oracle_paged.py`` (a hand-built pool, the identity and
+  permuted page tables against the contiguous functions, page size 1 and one
+  page per pair, scipy's softmax).
 """
 
 from .socket_ref import (
@@ -70,6 +77,7 @@ from .selection_ref import (
     select_adaptive,
     socket_decode_pair_adaptive,
 )
+from .paged_ref import paged_rows, attend_subset_paged, socket_decode_pair_paged
 
 __all__ = [
     "hash_key_ids",
@@ -94,4 +102,7 @@ __all__ = [
     "adaptive_k",
     "select_adaptive",
     "socket_decode_pair_adaptive",
+    "paged_rows",
+    "attend_subset_paged",
+    "socket_decode_pair_paged",
 ]

@@ -43,6 +43,9 @@ SIGNATURES = {
                                  _z, _p]),
     "socket_decode_adaptive": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _f, _i, _i,
                                     _f, _p, _p, _p, _p, _z, _p]),
+    "socket_sparse_attend_paged": (_i, [_p, _p, _p, _i, _p, _i, _i, _i, _p, _i, _i, _i, _i, _i, _f, _p, _p, _z, _p]),
+    "socket_decode_paged": (_i, [_p, _p, _p, _i, _p, _i, _i, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
+                                 _f, _p, _p, _p, _z, _p]),
     "sk_workspace_bytes": (_z, [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "sk_check_status": (_i, [_p]),
     "sk_profile_phases": (_i, [_p]),

@@ -19,7 +19,8 @@ from . import _lib
 
 SK_F32, SK_BF16 = 0, 1
 (OP_HASH_KEYS, OP_SCORE, OP_TOPK, OP_SPARSE_ATTEND, OP_DECODE, OP_HATA_HASH, OP_HATA_DECODE, OP_DENSE_DECODE,
- OP_SELECT, OP_SOFT_COUNT, OP_DECODE_HEADS, OP_DECODE_ADAPTIVE, OP_DECODE_ADAPTIVE_HEADS) = range(13)
+ OP_SELECT, OP_SOFT_COUNT, OP_DECODE_HEADS, OP_DECODE_ADAPTIVE, OP_DECODE_ADAPTIVE_HEADS, OP_SPARSE_ATTEND_PAGED,
+ OP_DECODE_PAGED) = range(15)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -37,6 +38,15 @@ def _ptr(t):
         raise ValueError("tensors must live on a CUDA device")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _pool_ptr(t):
+    """A K/V pool: device memory, or pinned host memory that the device reads directly."""
+    if t.is_cuda:
+        return _ptr(t)
+    if not (t.is_pinned() and t.is_contiguous()):
+        raise ValueError("host pools must be pinned and contiguous (the device reads them directly)")
     return ctypes.c_void_p(t.data_ptr())
 
 
@@ -263,6 +273,62 @@ def socket_decode_adaptive(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: 
                                          ctypes.c_float(mass), k_min, k_max, ctypes.c_float(scale), _ptr(O),
                                          _ptr(idx), _ptr(kcount), _ptr(ws), _ws_bytes(ws), _stream())
     _check(rc, "socket_decode_adaptive")
+
+
+def _want_pool(K_pool, V_pool, dtype, d):
+    if K_pool.dtype != dtype or V_pool.dtype != dtype:
+        raise TypeError(f"pools: dtypes {K_pool.dtype}, {V_pool.dtype}, expected {dtype}")
+    if K_pool.dim() != 3 or tuple(K_pool.shape) != tuple(V_pool.shape) or K_pool.shape[2] != d:
+        raise ValueError(f"pools: shapes {tuple(K_pool.shape)}, {tuple(V_pool.shape)}, expected [pages, page_size, {d}]")
+    if not (K_pool.is_contiguous() and V_pool.is_contiguous()):
+        raise ValueError("pools must be contiguous")
+    if K_pool.device.type == "cpu" and not (K_pool.is_pinned() and V_pool.is_pinned()):
+        raise ValueError("host pools must be pinned (the device reads them directly)")
+
+
+def socket_sparse_attend_paged(Q, K_pool, V_pool, page_table, idx, scale: float, O, ws=None):
+    """Sparse attention with K/V in a paged pool (device or pinned host memory).
+
+    K_pool, V_pool: [num_pages, page_size, d]; page_table: [B, Hkv, max_pages] int32 (device);
+    idx: [B, Hkv, k] int32 (device)."""
+    B, Hq, d = Q.shape
+    _, Hkv, max_pages = page_table.shape
+    num_pages, page_size, _ = K_pool.shape
+    k = idx.shape[-1]
+    _want_pool(K_pool, V_pool, Q.dtype, d)
+    _want(page_table, torch.int32, (B, Hkv, max_pages), "page_table")
+    _want(idx, torch.int32, (B, Hkv, k), "idx")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    ws = _workspace(workspace_bytes(OP_SPARSE_ATTEND_PAGED, B, Hq, Hkv, 32, k, d, 1, 1, k), Q.device, ws)
+    rc = _lib.lib.socket_sparse_attend_paged(_ptr(Q), _pool_ptr(K_pool), _pool_ptr(V_pool), _dtype_code(Q),
+                                             _ptr(page_table), max_pages, page_size, num_pages, _ptr(idx), B, Hq,
+                                             Hkv, d, k, ctypes.c_float(scale), _ptr(O), _ptr(ws), _ws_bytes(ws),
+                                             _stream())
+    _check(rc, "socket_sparse_attend_paged")
+
+
+def socket_decode_paged(Q, K_pool, V_pool, page_table, R, ids, norms, N: int, L: int, P: int, tau: float, k: int,
+                        scale: float, O, idx_out=None, ws=None):
+    """The decode step with a paged K/V cache; ids and norms are the contiguous hashed-key cache."""
+    B, Hq, d = Q.shape
+    _, Hkv, max_pages = page_table.shape
+    num_pages, page_size, _ = K_pool.shape
+    Ncap = ids.shape[2]
+    _want_pool(K_pool, V_pool, Q.dtype, d)
+    _want(page_table, torch.int32, (B, Hkv, max_pages), "page_table")
+    _want(R, torch.bfloat16, (L * P, d), "R")
+    _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
+    _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    if idx_out is not None:
+        _want(idx_out, torch.int32, (B, Hkv, k), "idx_out")
+    ws = _workspace(workspace_bytes(OP_DECODE_PAGED, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    rc = _lib.lib.socket_decode_paged(_ptr(Q), _pool_ptr(K_pool), _pool_ptr(V_pool), _dtype_code(Q),
+                                      _ptr(page_table), max_pages, page_size, num_pages, _ptr(R), _ptr(ids),
+                                      _ptr(norms), B, Hq, Hkv, Ncap, N, d, L, P, ctypes.c_float(tau), k,
+                                      ctypes.c_float(scale), _ptr(O), _ptr(idx_out), _ptr(ws), _ws_bytes(ws),
+                                      _stream())
+    _check(rc, "socket_decode_paged")
 
 
 def socket_decode_append(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k: int, scale: float, O,

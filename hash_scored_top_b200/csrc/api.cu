@@ -2,6 +2,7 @@
 // launches. Every entry point validates on the host before launching
 // anything, allocates nothing, and runs asynchronously on the caller's stream.
 #include <algorithm>
+#include <climits>
 #include <cstdarg>
 #include <cstdint>
 #include <cstdio>
@@ -510,12 +511,17 @@ int launch_attend_t(AttendParams ap, int pairs, int G, bool pdl, bool cluster, c
 int launch_attend(const void* Q, const void* K, const void* V, sk_dtype kv, const int* idx, int B, int Hq, int Hkv,
                   int Ncap, int n, int d, float scale, float* O, void* ws, size_t ws_bytes, bool pdl,
                   bool zero_counters, cudaStream_t s, bool allow_cluster = true, int pair_div = 1,
-                  const int* counts = nullptr) {
+                  const int* counts = nullptr, const int* page_table = nullptr, int max_pages = 0,
+                  int page_size = 0, int num_pages = 0) {
   const int pairs = B * Hkv, G = Hq / Hkv;
   if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
   AttendParams ap;
   ap.pair_div = pair_div;
   ap.counts = counts;
+  ap.page_table = page_table;
+  ap.max_pages = max_pages;
+  ap.page_size = page_size;
+  ap.num_pages = num_pages;
   ap.Q = Q;
   ap.K = K;
   ap.V = V;
@@ -545,6 +551,83 @@ int launch_attend(const void* Q, const void* K, const void* V, sk_dtype kv, cons
                                      : launch_attend_t<128, float>(ap, pairs, G, pdl, cluster, s);
   return kv == SK_BF16 ? launch_attend_t<64, __nv_bfloat16>(ap, pairs, G, pdl, cluster, s)
                        : launch_attend_t<64, float>(ap, pairs, G, pdl, cluster, s);
+}
+
+// ---------------------------------------------------------------- paged K/V
+// Where a pool lives: device memory (read by the attention kernel's bulk
+// copies through the page table) or host memory that the device can read
+// (gathered with plain loads first). Anything else is rejected.
+enum PoolKind { POOL_DEVICE = 0, POOL_HOST = 1, POOL_BAD = 2 };
+
+PoolKind pool_kind(const void* ptr) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return POOL_BAD;
+  }
+  if (a.type == cudaMemoryTypeDevice) return POOL_DEVICE;
+  if (a.type == cudaMemoryTypeHost || a.type == cudaMemoryTypeManaged) return a.devicePointer ? POOL_HOST : POOL_BAD;
+  return POOL_BAD;
+}
+
+// Workspace of the paged attention: for a host pool, the gathered K and V rows
+// and the attention workspace over them (dense, one split set per pair); for a
+// device pool, the sparse attention workspace. Sized for the larger.
+size_t paged_attend_ws_bytes(int pairs, int G, int d, int k, int kv_bytes) {
+  const size_t host = 2 * align256((size_t)pairs * k * d * kv_bytes) + attend_ws_bytes(pairs, attend_splits(k, pairs, true), G, d);
+  return std::max(host, attend_ws_bytes(pairs, attend_splits(k, pairs, false), G, d));
+}
+
+int launch_gather(const GatherParams& gp, int units, int row_bytes, cudaStream_t s) {
+  const dim3 grid(units, (gp.n + GATHER_KEYS - 1) / GATHER_KEYS);
+  switch (row_bytes) {
+    case 128: paged_gather_kernel<128><<<grid, GATHER_THREADS, 0, s>>>(gp); break;
+    case 256: paged_gather_kernel<256><<<grid, GATHER_THREADS, 0, s>>>(gp); break;
+    case 512: paged_gather_kernel<512><<<grid, GATHER_THREADS, 0, s>>>(gp); break;
+    default: return fail(SK_ERR_UNSUPPORTED, "row of %d bytes", row_bytes);
+  }
+  return check_launch("paged_gather_kernel");
+}
+
+// Attention over idx [units][k] with K/V in a paged pool (see AttendParams).
+int paged_attend_impl(const void* Q, const void* K_pool, const void* V_pool, sk_dtype kv, const int* page_table,
+                      int max_pages, int page_size, int num_pages, const int* idx, int B, int Hq, int Hkv, int d, int k,
+                      float scale, float* O, void* ws, size_t ws_bytes, cudaStream_t s, int pair_div = 1) {
+  const int pairs = B * Hkv, G = Hq / Hkv;
+  if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
+  const int esz = kv == SK_BF16 ? 2 : 4;
+  const PoolKind kk = pool_kind(K_pool), kvk = pool_kind(V_pool);
+  if (kk == POOL_BAD || kvk == POOL_BAD || kk != kvk)
+    return fail(SK_ERR_INVALID_ARG, "K_pool and V_pool must both be device memory or both device-readable host memory");
+  const size_t need = paged_attend_ws_bytes(pairs, G, d, k, esz);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
+  if (kk == POOL_DEVICE)
+    return launch_attend(Q, K_pool, V_pool, kv, idx, B, Hq, Hkv, 32, k, d, scale, O, ws, ws_bytes, false, true, s,
+                         true, pair_div, nullptr, page_table, max_pages, page_size, num_pages);
+  // host pool: gather the rows into the workspace, then dense attention over them
+  char* w = reinterpret_cast<char*>(ws);
+  void* Ks = w;
+  void* Vs = w + align256((size_t)pairs * k * d * esz);
+  char* aw = w + 2 * align256((size_t)pairs * k * d * esz);
+  GatherParams gp;
+  cudaPointerAttributes ak, av;
+  cudaPointerGetAttributes(&ak, K_pool);
+  cudaPointerGetAttributes(&av, V_pool);
+  gp.K = ak.devicePointer;
+  gp.V = av.devicePointer;
+  gp.page_table = page_table;
+  gp.idx = idx;
+  gp.Ks = Ks;
+  gp.Vs = Vs;
+  gp.n = k;
+  gp.max_pages = max_pages;
+  gp.page_size = page_size;
+  gp.num_pages = num_pages;
+  gp.pair_div = pair_div;
+  SK_TRY(launch_gather(gp, pairs, d * esz, s));
+  return launch_attend(Q, Ks, Vs, kv, nullptr, B, Hq, Hkv, k, k, d, scale, O, aw, ws_bytes - (size_t)(aw - w), false,
+                       true, s);
 }
 
 // Workspace of a decode step: the index list (when idx_out is NULL) then the
@@ -1133,6 +1216,79 @@ int socket_decode_adaptive(const void* Q, const void* K, const void* V, sk_dtype
                        k_max, scale, O, idx, kcount, ws, ws_bytes, as_stream(stream));
 }
 
+// Shared checks of the paged entry points.
+static int check_pages(const int* page_table, int max_pages, int page_size, int num_pages) {
+  SK_NONNULL(page_table);
+  if (max_pages < 1 || page_size < 1 || num_pages < 1)
+    return fail(SK_ERR_INVALID_ARG, "max_pages=%d, page_size=%d, num_pages=%d must be >= 1", max_pages, page_size,
+                num_pages);
+  if ((long long)max_pages * page_size > INT_MAX || (long long)num_pages * page_size > INT_MAX)
+    return fail(SK_ERR_UNSUPPORTED, "more than 2^31 - 1 rows per pair or per pool");
+  return SK_OK;
+}
+
+int socket_sparse_attend_paged(const void* Q, const void* K_pool, const void* V_pool, sk_dtype kv, const int* page_table,
+                               int max_pages, int page_size, int num_pages, const int* idx, int B, int Hq, int Hkv,
+                               int d, int k, float scale, float* O, void* ws, size_t ws_bytes, void* stream) {
+  SK_NONNULL(Q);
+  SK_NONNULL(K_pool);
+  SK_NONNULL(V_pool);
+  SK_NONNULL(idx);
+  SK_NONNULL(O);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(K_pool, 16);
+  SK_ALIGNED(V_pool, 16);
+  SK_TRY(check_dtype(kv));
+  SK_TRY(check_heads(B, Hq, Hkv, d));
+  SK_TRY(check_pages(page_table, max_pages, page_size, num_pages));
+  if (k < 1) return fail(SK_ERR_INVALID_ARG, "k=%d must be >= 1", k);
+  return paged_attend_impl(Q, K_pool, V_pool, kv, page_table, max_pages, page_size, num_pages, idx, B, Hq, Hkv, d, k,
+                           scale, O, ws, ws_bytes, as_stream(stream));
+}
+
+int socket_decode_paged(const void* Q, const void* K_pool, const void* V_pool, sk_dtype kv, const int* page_table,
+                        int max_pages, int page_size, int num_pages, const void* R, const void* ids, const void* norms,
+                        int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k, float scale,
+                        float* O, int* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  SK_NONNULL(Q);
+  SK_NONNULL(K_pool);
+  SK_NONNULL(V_pool);
+  SK_NONNULL(R);
+  SK_NONNULL(ids);
+  SK_NONNULL(norms);
+  SK_NONNULL(O);
+  SK_ALIGNED(Q, 16);
+  SK_ALIGNED(K_pool, 16);
+  SK_ALIGNED(V_pool, 16);
+  SK_ALIGNED(R, 16);
+  SK_ALIGNED(ids, 32);
+  SK_ALIGNED(norms, 2);
+  SK_TRY(check_dtype(kv));
+  SK_TRY(check_heads(B, Hq, Hkv, d));
+  SK_TRY(check_cache(Ncap, N));
+  SK_TRY(check_tables(L, P, tau));
+  SK_TRY(check_pages(page_table, max_pages, page_size, num_pages));
+  if (k < 1 || k > N) return fail(SK_ERR_INVALID_ARG, "k=%d must be in [1, N=%d]", k, N);
+  if ((long long)max_pages * page_size < N)
+    return fail(SK_ERR_INVALID_ARG, "max_pages * page_size = %lld < N = %d", (long long)max_pages * page_size, N);
+  const int pairs = B * Hkv, G = Hq / Hkv;
+  if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
+  const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, false, max_cluster_size());
+  const size_t list_bytes = align256((size_t)pairs * k * 4);
+  const size_t sel = align256(select_ws_bytes(fp, pairs, Ncap, L));
+  const size_t need = list_bytes + sel + paged_attend_ws_bytes(pairs, G, d, k, kv == SK_BF16 ? 2 : 4);
+  if (ws == nullptr || ws_bytes < need)
+    return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
+  char* w = reinterpret_cast<char*>(ws);
+  int* idx = idx_out ? idx_out : reinterpret_cast<int*>(w);
+  const cudaStream_t s = as_stream(stream);
+  // selection from the (contiguous) hashed-key cache, then the paged attention
+  SK_TRY(decode_impl(Q, nullptr, nullptr, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, 0.f, nullptr, idx,
+                     w + list_bytes, sel, false, false, s));
+  return paged_attend_impl(Q, K_pool, V_pool, kv, page_table, max_pages, page_size, num_pages, idx, B, Hq, Hkv, d, k,
+                           scale, O, w + list_bytes + sel, ws_bytes - list_bytes - sel, s);
+}
+
 int hata_hash_keys(const void* K, sk_dtype kv, const void* R128, int B, int Hkv, int Ncap, int n_begin, int n_count,
                    int d, void* codes, void* stream) {
   SK_NONNULL(K);
@@ -1305,6 +1461,15 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
       if (fp.C > 0) return decode_ws_bytes(B, Hq, Hq, k, d);
       return chain_ws_bytes(B, Hq, Hq, Ncap, d, L, k);
     }
+    case SK_OP_SPARSE_ATTEND_PAGED:
+      if (k < 1 || G > 8) return bad;
+      return paged_attend_ws_bytes(pairs, G, d, k, 4);          // f32 rows: the larger staging
+    case SK_OP_DECODE_PAGED: {
+      if (k < 1 || N < 1 || G > 8 || L < 1 || L > kMaxL || P < 1 || P > 8) return bad;
+      const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, false, 8);
+      return align256((size_t)pairs * k * 4) + align256(select_ws_bytes(fp, pairs, Ncap, L)) +
+             paged_attend_ws_bytes(pairs, G, d, k, 4);
+    }
     case SK_OP_DECODE_ADAPTIVE:
     case SK_OP_DECODE_ADAPTIVE_HEADS: {
       // k is k_max
@@ -1332,6 +1497,8 @@ int sk_check_status(void* stream) {
     const unsigned int zero = 0;
     cudaMemcpyToSymbol(g_error_word, &zero, sizeof(zero));
     if (word & ERR_TIMEOUT) return fail(SK_ERR_TIMEOUT, "a device-side bounded wait gave up");
+    if (word & ERR_RANGE)
+      return fail(SK_ERR_INVALID_ARG, "a page-table entry was outside [0, num_pages); its rows were read from page 0");
     return fail(SK_ERR_UNSUPPORTED, "a kernel's shared-memory plan did not fit; it wrote nothing");
   }
   return SK_OK;

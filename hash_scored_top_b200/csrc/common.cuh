@@ -17,6 +17,7 @@ constexpr unsigned FULL = 0xffffffffu;
 __device__ unsigned int g_error_word = 0u;
 constexpr unsigned ERR_TIMEOUT = 1u;   // a bounded wait gave up
 constexpr unsigned ERR_LAYOUT = 2u;    // a launch's shared-memory plan did not fit
+constexpr unsigned ERR_RANGE = 4u;     // a page-table entry outside the pool (read as page 0)
 
 // ---------------------------------------------------------------- bucket-ID cache layout
 // Each key stores its L bucket IDs in LP bytes, split in chunks of S_0, S_1

@@ -555,6 +555,10 @@ struct AttendParams {
   float scale;
   int pair_div = 1;        // units per cache pair, as in FusedParams
   const int* counts = nullptr;   // optional [units]: keys of each unit's list (<= n)
+  // paged K/V (with idx): K and V are pools [num_pages][page_size][D] and key
+  // n of cache pair c is row n % page_size of page page_table[c][n / page_size]
+  const int* page_table = nullptr;   // [cache pairs][max_pages]
+  int max_pages = 0, page_size = 0, num_pages = 0;
 };
 
 __device__ __forceinline__ void attend_stamp(unsigned long long* ts, int phase) {
@@ -623,15 +627,35 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
   // lists have per-unit lengths
   const int n_unit = p.counts ? min(max(__ldcg(p.counts + pair), 0), p.n) : p.n;
   const int cnt = max(0, min(n_unit - i0, p.keys_per_split));
-  const KVT* Kp = reinterpret_cast<const KVT*>(p.K) + pair_keys * D;
-  const KVT* Vp = reinterpret_cast<const KVT*>(p.V) + pair_keys * D;
+  const bool paged = p.page_table != nullptr;
+  const size_t key0 = paged ? 0 : pair_keys;            // a paged pool is addressed by physical row
+  const KVT* Kp = reinterpret_cast<const KVT*>(p.K) + key0 * D;
+  const KVT* Vp = reinterpret_cast<const KVT*>(p.V) + key0 * D;
   float *cM, *cL, *cO;
   if (p.idx) {
     const int* list = p.idx + (size_t)pair * p.n + i0;      // one coalesced load of this CTA's indices
-    for (int i = threadIdx.x; i < cnt; i += blockDim.x) list_s[i] = __ldcg(list + i);
+    int nrows = p.Ncap;
+    if (paged) {
+      // logical key -> physical pool row; an entry outside the pool is
+      // flagged and read as page 0 (every access stays inside the pool)
+      const int* pt = p.page_table + (size_t)(pair / p.pair_div) * p.max_pages;
+      const int last = p.max_pages * p.page_size - 1;
+      for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+        const int n = min(max(__ldcg(list + i), 0), last);
+        int pg = __ldg(pt + n / p.page_size);
+        if (pg < 0 || pg >= p.num_pages) {
+          atomicOr(&g_error_word, ERR_RANGE);
+          pg = 0;
+        }
+        list_s[i] = pg * p.page_size + n % p.page_size;
+      }
+      nrows = p.num_pages * p.page_size;
+    } else {
+      for (int i = threadIdx.x; i < cnt; i += blockDim.x) list_s[i] = __ldcg(list + i);
+    }
     __syncthreads();
     attend_stamp(p.phase_ts, 3);
-    attend_and_merge<D, KVT>(dyn, base, as, Qg, Kp, Vp, G, p.scale, [=](int i) { return list_s[i]; }, cnt, p.Ncap,
+    attend_and_merge<D, KVT>(dyn, base, as, Qg, Kp, Vp, G, p.scale, [=](int i) { return list_s[i]; }, cnt, nrows,
                              cM, cL, cO);
   } else {
     attend_and_merge<D, KVT>(dyn, base, as, Qg, Kp, Vp, G, p.scale, [=](int i) { return i0 + i; }, cnt, p.Ncap, cM,
@@ -708,6 +732,74 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
   if (threadIdx.x == 0) p.counters[pair] = 0u;
   attend_stamp(p.phase_ts, 6);
   attend_stamp(p.phase_ts, 7);
+}
+
+// ---------------------------------------------------------------- paged gather
+// Copies the selected keys' K and V rows from a paged pool into contiguous
+// rows Ks, Vs [units][n][ROW bytes], with plain 16-byte loads: the pool may be
+// pinned host memory (read over the host link) as well as device memory. Half
+// a warp copies one K row and the other half the matching V row; each warp
+// keeps GATHER_UNROLL row pairs in flight. grid = (units, chunks of
+// GATHER_KEYS keys).
+struct GatherParams {
+  const void* K;
+  const void* V;
+  const int* page_table;   // [cache pairs][max_pages]
+  const int* idx;          // [units][n]
+  void* Ks;
+  void* Vs;
+  int n, max_pages, page_size, num_pages, pair_div;
+};
+
+constexpr int GATHER_THREADS = 256;
+constexpr int GATHER_KEYS = 64;
+constexpr int GATHER_UNROLL = 4;
+
+template <int ROW>
+__global__ void __launch_bounds__(GATHER_THREADS) paged_gather_kernel(const GatherParams p) {
+  constexpr int CH = ROW / 16;                       // 16-byte chunks per row: 8, 16 or 32
+  constexpr int CPL = (CH + 15) / 16;                // chunks per lane of the half warp
+  const int unit = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int half = lane >> 4, c = lane & 15;
+  const int* pt = p.page_table + (size_t)(unit / p.pair_div) * p.max_pages;
+  const int last = p.max_pages * p.page_size - 1;
+  const unsigned char* src_base = reinterpret_cast<const unsigned char*>(half ? p.V : p.K);
+  unsigned char* dst_base = reinterpret_cast<unsigned char*>(half ? p.Vs : p.Ks) + (size_t)unit * p.n * ROW;
+  const int j_end = min(p.n, (int)(blockIdx.y + 1) * GATHER_KEYS);
+  for (int j0 = blockIdx.y * GATHER_KEYS + warp; j0 < j_end; j0 += (GATHER_THREADS / 32) * GATHER_UNROLL) {
+    uint4 v[GATHER_UNROLL][CPL];
+    size_t row[GATHER_UNROLL];
+#pragma unroll
+    for (int u = 0; u < GATHER_UNROLL; ++u) {
+      const int j = j0 + u * (GATHER_THREADS / 32);
+      row[u] = 0;
+      if (j < j_end) {
+        const int n = min(max(__ldg(p.idx + (size_t)unit * p.n + j), 0), last);
+        int pg = __ldg(pt + n / p.page_size);
+        if (pg < 0 || pg >= p.num_pages) {
+          atomicOr(&g_error_word, ERR_RANGE);
+          pg = 0;
+        }
+        row[u] = (size_t)pg * p.page_size + n % p.page_size;
+      }
+#pragma unroll
+      for (int q = 0; q < CPL; ++q) {
+        const int ch = c + 16 * q;
+        v[u][q] = (j < j_end && ch < CH) ? *reinterpret_cast<const uint4*>(src_base + row[u] * ROW + 16 * ch)
+                                         : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < GATHER_UNROLL; ++u) {
+      const int j = j0 + u * (GATHER_THREADS / 32);
+#pragma unroll
+      for (int q = 0; q < CPL; ++q) {
+        const int ch = c + 16 * q;
+        if (j < j_end && ch < CH) *reinterpret_cast<uint4*>(dst_base + (size_t)j * ROW + 16 * ch) = v[u][q];
+      }
+    }
+  }
 }
 
 }  // namespace hst

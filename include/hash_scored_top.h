@@ -84,7 +84,9 @@ typedef enum {
   SK_OP_SOFT_COUNT = 9,
   SK_OP_DECODE_HEADS = 10,
   SK_OP_DECODE_ADAPTIVE = 11,        /* k is k_max */
-  SK_OP_DECODE_ADAPTIVE_HEADS = 12   /* k is k_max */
+  SK_OP_DECODE_ADAPTIVE_HEADS = 12,  /* k is k_max */
+  SK_OP_SPARSE_ATTEND_PAGED = 13,
+  SK_OP_DECODE_PAGED = 14
 } sk_op;
 
 /*
@@ -262,6 +264,40 @@ int socket_decode_adaptive(const void* Q, const void* K, const void* V, sk_dtype
                            int d, int L, int P, float tau, int per_head, float mass, int k_min,
                            int k_max, float scale, float* O, int* idx, int* kcount, void* ws,
                            size_t ws_bytes, void* stream);
+
+/*
+ * Sparse attention (as socket_sparse_attend) with K and V in a paged pool
+ * (HATA digest, sections 3-4: the offloaded KV cache; HGA page, section 3:
+ * hot and routed pages). K_pool, V_pool: [num_pages][page_size][d] (dtype kv);
+ * page_table: [B][Hkv][max_pages] int32 device array; key n of pair p is row
+ * n % page_size of page page_table[p][n / page_size]. idx: [B][Hkv][k] key
+ * indices in [0, max_pages * page_size). The pools may be device memory
+ * (the attention kernel reads the selected rows through the page table) or
+ * pinned host memory that the device can address (the selected rows are first
+ * copied into ws with plain loads over the host link, then attended). Both
+ * pools must be of the same kind. A page-table entry outside [0, num_pages) is
+ * read as page 0 and reported by sk_check_status (SK_ERR_INVALID_ARG).
+ * Requires max_pages, page_size, num_pages >= 1, G <= 8, and fewer than 2^31
+ * rows per pool. ws: sk_workspace_bytes(SK_OP_SPARSE_ATTEND_PAGED, ..., k).
+ */
+int socket_sparse_attend_paged(const void* Q, const void* K_pool, const void* V_pool, sk_dtype kv,
+                               const int* page_table, int max_pages, int page_size, int num_pages,
+                               const int* idx, int B, int Hq, int Hkv, int d, int k, float scale,
+                               float* O, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The decode step of socket_decode with a paged K/V cache: the selection
+ * (steps 2-4) reads the contiguous hashed-key cache (ids, norms as above),
+ * then socket_sparse_attend_paged gathers the selected rows from the pools.
+ * Same results as socket_decode over the cache the pages describe.
+ * Requires max_pages * page_size >= N and what both calls require.
+ * ws: sk_workspace_bytes(SK_OP_DECODE_PAGED, ...) bytes.
+ */
+int socket_decode_paged(const void* Q, const void* K_pool, const void* V_pool, sk_dtype kv,
+                        const int* page_table, int max_pages, int page_size, int num_pages,
+                        const void* R, const void* ids, const void* norms, int B, int Hq, int Hkv,
+                        int Ncap, int N, int d, int L, int P, float tau, int k, float scale, float* O,
+                        int* idx_out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * Hard-hash codes (HATA digest, section 3, with seeded random hyperplanes

@@ -416,6 +416,7 @@ def run_ours(args, world, rank, local):
         result["soft_count_estimator"] = run_estimator(w, api, caches, device, rb, peak)
         result["per_head_decode"] = run_heads(w, api, caches, device, peak)
         result["adaptive_decode"] = run_adaptive(w, api, caches, device, peak)
+        result["paged_decode"] = run_paged(w, api, caches, device, rb, peak)
         if rank == 0 and world == 1:
             result["cpu_baseline"] = cpu_baseline(w, caches[0], sample_pairs=8)
     del g_step, g_dec, g_sel
@@ -668,6 +669,87 @@ def run_adaptive(w, api, caches, device, peak):
             "k_mean": mean_k, "k_range": [min(ks), max(ks)], "required_bytes": nbytes, "hbm_gbs": gbs,
             "frac_of_peak": gbs / peak, "frac_of_nominal_8tbs": gbs / NOMINAL_HBM_GBS,
             "launch": f"CUDA graph of {len(caches)} calls (one per cache)"}
+
+
+PAGE_SIZE = 64
+
+
+def _to_pages(K, V, page_size, seed):
+    """The cache [B, Hkv, Ncap, d] scattered over a shuffled pool of pages, and its page table."""
+    import torch
+    B, Hkv, Ncap, d = K.shape
+    per = Ncap // page_size
+    g = torch.Generator().manual_seed(seed)
+    phys = torch.randperm(B * Hkv * per, generator=g).to(K.device)
+    Kp = torch.empty(B * Hkv * per, page_size, d, dtype=K.dtype, device=K.device)
+    Vp = torch.empty_like(Kp)
+    Kp[phys] = K.reshape(-1, page_size, d)
+    Vp[phys] = V.reshape(-1, page_size, d)
+    return Kp, Vp, phys.view(B, Hkv, per).int().contiguous()
+
+
+def run_paged(w, api, caches, device, rb, peak):
+    """The decode step with the K/V cache in a pool of 64-key pages
+    (socket_decode_paged): device-resident pools (one per cache, pages
+    shuffled), and one pinned host pool, whose selected rows cross the host
+    link. The host-link peak is the measured pinned host-to-device copy rate."""
+    import torch
+    Ncap = caches[0]["K"].shape[2]
+    if Ncap % PAGE_SIZE:
+        return {"skipped": f"Ncap {Ncap} is not a multiple of the page size {PAGE_SIZE}"}
+    pools = [_to_pages(c["K"], c["V"], PAGE_SIZE, 17 + i) for i, c in enumerate(caches)]
+    O = torch.empty(w.B, w.Hq, w.d, device=device)
+    ws = torch.empty(api.workspace_bytes(api.OP_DECODE_PAGED, w.B, w.Hq, w.Hkv, Ncap, w.N, w.d, w.L, w.P, w.k),
+                     dtype=torch.uint8, device=device)
+
+    def dev_call(i):
+        c = caches[i]
+        Kp, Vp, tab = pools[i]
+        api.socket_decode_paged(c["Q"], Kp, Vp, tab, c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k,
+                                w.scale, O, None, ws)
+
+    us_dev = _time_calls(dev_call, len(caches))
+    api.check_status()
+    rec = {"page_size": PAGE_SIZE, "device_pool": {
+        "us": us_dev, "steps_per_s": 1e6 / us_dev, "required_bytes": rb["decode"],
+        "hbm_gbs": rb["decode"] / (us_dev * 1e-6) / 1e9, "frac_of_peak": rb["decode"] / (us_dev * 1e-6) / 1e9 / peak,
+        "kernels": "socket_select_kernel -> socket_attend_kernel (rows through the page table)",
+        "launch": f"CUDA graph of {len(caches)} calls (one per cache)"}}
+    # the host link: pinned -> device copy rate of 256 MB
+    src = torch.empty(256 << 20, dtype=torch.uint8).pin_memory()
+    dst = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for _ in range(2):
+        dst.copy_(src, non_blocking=True)
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(5):
+        dst.copy_(src, non_blocking=True)
+    e.record()
+    torch.cuda.synchronize()
+    link_gbs = 5 * (256 << 20) / (s.elapsed_time(e) * 1e-3) / 1e9
+    del src, dst
+    Kp, Vp, tab = pools[0]
+    Kh, Vh = Kp.cpu().pin_memory(), Vp.cpu().pin_memory()
+
+    def host_call(i):
+        c = caches[0]
+        api.socket_decode_paged(c["Q"], Kh, Vh, tab, c["R"], c["ids"], c["norms"], w.N, w.L, w.P, w.tau, w.k,
+                                w.scale, O, None, ws)
+
+    us_host = _time_calls(host_call, 1, reps=10, warm=2)
+    api.check_status()
+    link_bytes = w.pairs * w.k * 2 * w.d * 2
+    rec["host_pool"] = {
+        "us": us_host, "steps_per_s": 1e6 / us_host, "host_link_bytes": link_bytes,
+        "host_link_gbs": link_bytes / (us_host * 1e-6) / 1e9, "host_link_peak_gbs": link_gbs,
+        "frac_of_link_peak": link_bytes / (us_host * 1e-6) / 1e9 / link_gbs,
+        "kernels": "socket_select_kernel -> paged_gather_kernel (plain loads of pinned host rows) -> "
+                   "socket_attend_kernel (dense over the gathered rows)",
+        "launch": "CUDA graph of 1 call, 10 replays (the one host pool)"}
+    del pools, Kh, Vh, ws
+    torch.cuda.empty_cache()
+    return rec
 
 
 def run_dense(w, api, caches, device, rb, peak):

@@ -49,6 +49,7 @@ SIGNATURES = {
     "sk_workspace_bytes": (_z, [_i, _i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "sk_check_status": (_i, [_p]),
     "sk_profile_phases": (_i, [_p]),
+    "sk_test_set_wait_limit": (_i, [ctypes.c_longlong]),
     "sk_last_error": (ctypes.c_char_p, []),
     "sk_version": (ctypes.c_char_p, []),
 }

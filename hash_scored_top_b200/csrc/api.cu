@@ -308,12 +308,52 @@ int launch_tables(const void* Q, sk_dtype q, const void* R, int B, int Hq, int H
 
 constexpr int kScoreBlocksPerCta = 256;
 
-template <int LP>
+template <int LP, bool NORM = true>
 int launch_score_t(const ScoreParams& sp, dim3 grid, cudaStream_t s) {
   const int smem = (int)(kTableAddr + table_chunks(LP) * TABLE_BYTES - SMEM_BASE_EXPECTED);
-  set_kernel_smem(socket_score_kernel<LP>, smem);
-  socket_score_kernel<LP><<<grid, FUSED_THREADS, smem, s>>>(sp);
+  set_kernel_smem(socket_score_kernel<LP, NORM>, smem);
+  socket_score_kernel<LP, NORM><<<grid, FUSED_THREADS, smem, s>>>(sp);
   return check_launch("socket_score_kernel");
+}
+
+// The hard-hash variant's tables (16 byte-tables from R128) into T.
+int launch_hamming_tables(const void* Q, sk_dtype q, const void* R128, int B, int Hq, int Hkv, int d, float* T,
+                          cudaStream_t s) {
+  TableParams tp;
+  tp.Q = Q;
+  tp.R = reinterpret_cast<const __nv_bfloat16*>(R128);
+  tp.T = T;
+  tp.Hq = Hq;
+  tp.Hkv = Hkv;
+  tp.L = 16;
+  tp.P = 8;
+  tp.tau = 1.f;
+  const int G = Hq / Hkv, pairs = B * Hkv;
+  const size_t smem = hamming_scratch_bytes(G, d, 16);
+  if (d == 128) {
+    auto kern = q == SK_BF16 ? hamming_table_kernel<128, __nv_bfloat16> : hamming_table_kernel<128, float>;
+    set_kernel_smem(kern, smem);
+    kern<<<pairs, 256, smem, s>>>(tp);
+  } else {
+    auto kern = q == SK_BF16 ? hamming_table_kernel<64, __nv_bfloat16> : hamming_table_kernel<64, float>;
+    set_kernel_smem(kern, smem);
+    kern<<<pairs, 256, smem, s>>>(tp);
+  }
+  return check_launch("hamming_table_kernel");
+}
+
+// Hard-hash scores from the codes (16 bytes per key, no norms).
+int launch_hamming_score(const float* T, const void* codes, int pairs, int Ncap, int N, float* scores, cudaStream_t s) {
+  ScoreParams sp;
+  sp.T = T;
+  sp.ids = reinterpret_cast<const uint8_t*>(codes);
+  sp.norms = nullptr;
+  sp.scores = scores;
+  sp.Ncap = Ncap;
+  sp.N = N;
+  sp.blocks_per_cta = kScoreBlocksPerCta;
+  const int nblk = (N + 31) / 32;
+  return launch_score_t<16, false>(sp, dim3(pairs, (nblk + kScoreBlocksPerCta - 1) / kScoreBlocksPerCta), s);
 }
 
 int launch_score(const float* T, const void* ids, const void* norms, int pairs, int Ncap, int N, int L, float* scores,
@@ -985,7 +1025,7 @@ int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const 
   const int pairs = B * Hkv, G = Hq / Hkv;
   if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
   const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, hata, max_cluster_size());
-  if (fp.C == 0 && hata) return fail(SK_ERR_UNSUPPORTED, "hard-hash decode: N=%d too large for one cluster", N);
+
   const size_t need = !attend ? select_ws_bytes(fp, pairs, Ncap, L)
                       : fp.C > 0 ? decode_ws_bytes(B, Hq, Hkv, k, d) : chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
   if (need > 0 && (ws == nullptr || ws_bytes < need))
@@ -998,8 +1038,13 @@ int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const 
     w += align256((size_t)pairs * Ncap * 4);
     int* idx = idx_out ? idx_out : reinterpret_cast<int*>(w);
     w += align256((size_t)pairs * k * 4);
-    SK_TRY(launch_tables(Q, kv, R, B, Hq, Hkv, d, L, P, tau, T, s));
-    SK_TRY(launch_score(T, ids, norms, pairs, Ncap, N, L, scores, s, pair_div));
+    if (hata) {            // hard-hash chain: byte-tables, integer scores from the codes
+      SK_TRY(launch_hamming_tables(Q, kv, R, B, Hq, Hkv, d, T, s));
+      SK_TRY(launch_hamming_score(T, ids, pairs, Ncap, N, scores, s));
+    } else {
+      SK_TRY(launch_tables(Q, kv, R, B, Hq, Hkv, d, L, P, tau, T, s));
+      SK_TRY(launch_score(T, ids, norms, pairs, Ncap, N, L, scores, s, pair_div));
+    }
     SK_TRY(launch_topk(scores, pairs, Ncap, N, k, idx, s));
     if (!attend) return SK_OK;
     return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, w,
@@ -1451,7 +1496,7 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
       // the unfused chain runs when the selection cannot hold a pair's keys on
       // chip; 8-CTA clusters are always available, 16-CTA ones may not be
       const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, op == SK_OP_HATA_DECODE, 8);
-      if (fp.C > 0 || op == SK_OP_HATA_DECODE) return decode_ws_bytes(B, Hq, Hkv, k, d);
+      if (fp.C > 0) return decode_ws_bytes(B, Hq, Hkv, k, d);
       return chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
     }
     case SK_OP_DECODE_HEADS: {
@@ -1480,6 +1525,13 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
     default:
       return bad;
   }
+}
+
+int sk_test_set_wait_limit(long long cycles) {
+  const long long v = cycles > 0 ? cycles : kWaitLimit;
+  const cudaError_t e = cudaMemcpyToSymbol(g_tc_wait_limit, &v, sizeof(v));
+  if (e != cudaSuccess) return fail(SK_ERR_CUDA, "wait limit: %s", cudaGetErrorString(e));
+  return SK_OK;
 }
 
 int sk_profile_phases(unsigned long long* device_buffer) {

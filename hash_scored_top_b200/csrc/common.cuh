@@ -178,13 +178,36 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t addr, uint32_t parity) {
   return ok != 0;
 }
 
-// Waits for the phase with the given parity to complete, for at most about
-// one second of SM clock; on giving up sets ERR_TIMEOUT and returns false.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity) {
+// Non-blocking: whether the phase with the given parity has completed.
+__device__ __forceinline__ bool mbar_test_wait(uint32_t addr, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\tmbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\tselp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(addr), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Waits for the phase with the given parity to complete, for at most `limit`
+// SM clocks (by default about one second); on giving up sets ERR_TIMEOUT and
+// returns false.
+constexpr long long kWaitLimit = 2000000000LL;
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t addr, uint32_t parity, long long limit = kWaitLimit) {
+  if (limit < kWaitLimit) {
+    // a lowered limit (test hook only): the blocking try_wait below may itself
+    // wait longer than the limit, so test once without blocking, then poll
+    if (mbar_test_wait(addr, parity)) return true;
+    const long long t0 = clock64();
+    while (clock64() - t0 <= limit)
+      if (mbar_test_wait(addr, parity)) return true;
+    atomicOr(&g_error_word, ERR_TIMEOUT);
+    return false;
+  }
   if (mbar_try_wait(addr, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(addr, parity)) {
-    if (clock64() - t0 > 2000000000LL) {
+    if (clock64() - t0 > limit) {
       atomicOr(&g_error_word, ERR_TIMEOUT);
       return false;
     }

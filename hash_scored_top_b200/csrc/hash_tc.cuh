@@ -247,6 +247,10 @@ __device__ __forceinline__ bool tc_row(const HashParams& p, const TcTile& t, int
 // box 64 x 128, 128-byte swizzle (rows past the last pair read as zero).
 // mapR: the hyperplanes [8L rows][D], box 64 x 32, 128-byte swizzle (rows
 // past 8L read as zero).
+// Limit (SM clocks) of the main loop's waits; the drain on the way out always
+// waits up to kWaitLimit. Lowered only by the test hook sk_test_set_wait_limit.
+__device__ long long g_tc_wait_limit = kWaitLimit;
+
 template <int D>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     hash_keys_tcgen05_kernel(const HashParams p, const TcRows tr, const __grid_constant__ CUtensorMap mapK,
@@ -271,6 +275,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t fullK = s0 + pl.ctl_off, fullV = fullK + 32, mmab = fullK + 48, rbar = fullK + 64;
   const uint32_t tslot = fullK + kTslot;
   volatile int* fail = reinterpret_cast<volatile int*>(dyn + pl.ctl_off + kFail);
+  const long long lim = g_tc_wait_limit;
+  // thread 128's record of the ring positions it issued and saw complete, for
+  // the drain on the way out (the loop stops early after a wait gave up)
+  int k_issued = 0, k_seen = 0, v_issued = 0, v_seen = 0, m_issued = 0;
+  bool r_seen = false;
   auto kstage = [&](int j) { return s0 + pl.k_off + (uint32_t)(j % SK) * pl.tile_bytes; };
   auto vstage = [&](int j) { return s0 + pl.v_off + (uint32_t)(j % (SV > 0 ? SV : 1)) * pl.tile_bytes; };
 
@@ -292,17 +301,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   }
 
   // thread 128: TMA copies of ring position j's keys (or values)
-  auto tma_rows = [&](const CUtensorMap* map, int j, uint32_t dst, uint32_t bar) {
+  auto tma_rows = [&](const CUtensorMap* map, int j, uint32_t dst, uint32_t bar) -> bool {
     const int u = (int)blockIdx.x + j * (int)gridDim.x;
-    if (u >= tr.n_tiles) return;
+    if (u >= tr.n_tiles) return false;
     const TcTile t = tc_tile(tr, u);
     const int row = t.pair * p.Ncap + t.key0;
     mbar_arrive_expect_tx(bar, pl.tile_bytes);
 #pragma unroll
     for (int a = 0; a < NATOM; ++a) tma_load_2d(dst + (uint32_t)a * TC_ATOM, map, 64 * a, row, bar);
+    return true;
   };
-  auto tma_keys = [&](int j) { tma_rows(&mapK, j, kstage(j), fullK + 8u * (uint32_t)(j % SK)); };
-  auto tma_values = [&](int j) { tma_rows(&mapV, j, vstage(j), fullV + 8u * (uint32_t)(j % SV)); };
+  auto tma_keys = [&](int j) {
+    if (tma_rows(&mapK, j, kstage(j), fullK + 8u * (uint32_t)(j % SK))) k_issued = j + 1;
+  };
+  auto tma_values = [&](int j) {
+    if (tma_rows(&mapV, j, vstage(j), fullV + 8u * (uint32_t)(j % SV))) v_issued = j + 1;
+  };
   // accumulator buffer of ring position j, and the parity of its mbarrier phase
   auto buf_of = [&](int j) { return A ? (uint32_t)(j & 1) : 0u; };
   auto par_of = [&](int j) { return A ? (uint32_t)((j >> 1) & 1) : (uint32_t)(j & 1); };
@@ -310,8 +324,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   bool r_ready = false;
   auto issue_mma = [&](int j, uint32_t tbase) {
     if (!r_ready) {
-      if (!mbar_wait_bounded(rbar, 0u)) *fail = 1;
-      r_ready = true;
+      if (!mbar_wait_bounded(rbar, 0u, lim)) {
+        *fail = 1;
+        return;                              // no MMA on operands that have not arrived
+      }
+      r_ready = r_seen = true;
     }
     tc_fence_after_sync();
     const uint32_t buf = buf_of(j);
@@ -329,9 +346,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       }
     }
     tc_commit(mmab + 8u * buf);
+    m_issued = j + 1;
   };
-  auto wait_keys = [&](int j) {
-    if (!mbar_wait_bounded(fullK + 8u * (uint32_t)(j % SK), (uint32_t)((j / SK) & 1))) *fail = 1;
+  // the keys of ring position j have landed (else the loop stops; no MMA is
+  // issued on them)
+  auto wait_keys = [&](int j) -> bool {
+    if (!mbar_wait_bounded(fullK + 8u * (uint32_t)(j % SK), (uint32_t)((j / SK) & 1), lim)) {
+      *fail = 1;
+      return false;
+    }
+    k_seen = j + 1;
+    return true;
   };
 
   const int G = (int)gridDim.x;
@@ -345,8 +370,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   tc_fence_after_sync();
   const uint32_t tbase = *reinterpret_cast<volatile uint32_t*>(dyn + pl.ctl_off + kTslot);
   if (A && tid == TC_M && my_tiles > 0) {
-    wait_keys(0);
-    issue_mma(0, tbase);
+    if (wait_keys(0)) issue_mma(0, tbase);
   }
 
   for (int i = 0; i < my_tiles; ++i) {
@@ -364,13 +388,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tma_keys(i + SK - 1);                // into the stages of tile i - 1
         if (SV > 0) tma_values(i + SV - 1);
         const int j = i + A;
-        if (j < my_tiles) {
-          wait_keys(j);
-          issue_mma(j, tbase);
-        }
+        if (j < my_tiles && wait_keys(j)) issue_mma(j, tbase);
       }
-      if (SV > 0 && !mbar_wait_bounded(fullV + 8u * (uint32_t)(i % SV), (uint32_t)((i / SV) & 1))) *fail = 1;
-      if (values) {
+      bool okv = true;
+      if (SV > 0) {
+        okv = mbar_wait_bounded(fullV + 8u * (uint32_t)(i % SV), (uint32_t)((i / SV) & 1), lim);
+        if (!okv) *fail = 1;
+        else if (tid == TC_M) v_seen = i + 1;
+      }
+      if (values && okv) {
         const double nrm = value_norm_tile<D>(vstage(i), m);
         if (mine) p.norms[kidx] = __double2half(nrm);
       }
@@ -378,7 +404,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // the row's signs: bit j of word b is column 32b + j, i.e. hyperplane
       // j % 8 of table 4b + j / 8; columns >= 8L are zero and give zero bits
       const uint32_t buf = buf_of(i);
-      if (!mbar_wait_bounded(mmab + 8u * buf, par_of(i))) *fail = 1;
+      if (!mbar_wait_bounded(mmab + 8u * buf, par_of(i), lim)) {
+        *fail = 1;                           // the accumulators are not ready: leave the row unwritten
+        continue;
+      }
       tc_fence_after_sync();
       const uint32_t ta = tbase + ((uint32_t)(32 * warp) << 16) + buf * (uint32_t)pl.ncols;
       uint32_t w[16];
@@ -422,6 +451,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
       }
     }
+  }
+  // Drain: everything thread 128 issued and did not see complete (after a
+  // wait gave up, the loop stopped with copies and MMAs still in flight) is
+  // waited for, up to the full limit each, before the tensor memory is freed
+  // and the CTA's shared memory is released.
+  if (tid == TC_M) {
+    if (!r_seen) mbar_wait_bounded(rbar, 0u);
+    for (int j = k_seen; j < k_issued; ++j) mbar_wait_bounded(fullK + 8u * (uint32_t)(j % SK), (uint32_t)((j / SK) & 1));
+    for (int j = v_seen; j < v_issued; ++j) mbar_wait_bounded(fullV + 8u * (uint32_t)(j % SV), (uint32_t)((j / SV) & 1));
+    for (int j = max(0, m_issued - (A ? 2 : 1)); j < m_issued; ++j) mbar_wait_bounded(mmab + 8u * buf_of(j), par_of(j));
   }
   tc_fence_before_sync();
   __syncthreads();

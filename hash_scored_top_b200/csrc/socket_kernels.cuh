@@ -458,6 +458,22 @@ __global__ void __launch_bounds__(256) bucket_table_kernel(const TableParams p) 
                         });
 }
 
+// The hard-hash variant's 16 byte-tables of a pair into its table image (one
+// 64-column chunk, table m in columns m, m + 16, m + 32, m + 48). grid = pairs.
+template <int D, typename QT>
+__global__ void __launch_bounds__(256) hamming_table_kernel(const TableParams p) {
+  extern __shared__ __align__(1024) unsigned char dyn[];
+  const int pair = blockIdx.x;
+  const int G = p.Hq / p.Hkv;
+  const int b = pair / p.Hkv, kvh = pair % p.Hkv;
+  const QT* Qg = reinterpret_cast<const QT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
+  float* T = p.T + (size_t)pair * 256 * TABLE_COLS;
+  build_hamming_table<D>(Qg, G, p.R, 0, 16, dyn, [&](int x, int m, float v) {
+    float* row = T + (size_t)x * TABLE_COLS;
+    for (int c = m; c < TABLE_COLS; c += 16) row[c] = v;
+  });
+}
+
 struct ScoreParams {
   const float* T;
   const uint8_t* ids;
@@ -468,8 +484,9 @@ struct ScoreParams {
 };
 
 // grid = (pairs, chunks); the pair's table image is copied to 64 KB-aligned
-// shared memory, then each lane scores one key.
-template <int LP>
+// shared memory, then each lane scores one key. NORM = false: hard-hash
+// scores (ids holds the 128-bit codes, the image the 16 byte-tables, no norm).
+template <int LP, bool NORM = true>
 __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_score_kernel(const ScoreParams p) {
   extern __shared__ __align__(1024) unsigned char dyn[];
   constexpr int NCH = table_chunks(LP);
@@ -495,8 +512,8 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_score_kernel(const Sc
   for (int blk = blk0 + warp; blk < blk1; blk += nw) {
     const int key = blk * 32 + lane;
     KeyIds<LP> k;
-    load_key_ids<LP, true>(k, p.ids + (pair_keys + key) * LP, p.norms + pair_keys + key);
-    const float s = score_key<LP, true>(k, tbl + 4u * lane, tbl + TABLE_BYTES + 4u * lane);
+    load_key_ids<LP, NORM>(k, p.ids + (pair_keys + key) * LP, p.norms + pair_keys + key);
+    const float s = score_key<LP, NORM>(k, tbl + 4u * lane, tbl + TABLE_BYTES + 4u * lane);
     if (key < p.N) p.scores[(size_t)pair * p.Ncap + key] = s;
   }
 }

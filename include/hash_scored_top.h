@@ -376,6 +376,18 @@ int sk_check_status(void* stream);
  * Pass NULL to turn it off. One store per phase per CTA. */
 int sk_profile_phases(unsigned long long* device_buffer);
 
+/*
+ * Test hook, not for production use: sets the limit, in SM clocks, of the
+ * main-loop waits of the tensor-core hashing kernel (socket_hash_keys /
+ * hata_hash_keys on bf16 keys with P = 8; cycles <= 0 restores the default of
+ * about one second). With a tiny limit its waits give up while its copies and
+ * MMAs are still in flight, which exercises the failure path: the kernel
+ * stops, waits (with the default limit) for everything it issued, frees its
+ * tensor memory and returns; the next sk_check_status reports
+ * SK_ERR_TIMEOUT. Affects every later call on the current device until reset.
+ */
+int sk_test_set_wait_limit(long long cycles);
+
 /* Thread-local description of the last non-OK return (never NULL). */
 const char* sk_last_error(void);
 

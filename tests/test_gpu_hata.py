@@ -83,3 +83,22 @@ def test_hata_self_query_key_selected(api):
     for b in range(w.B):
         for h in range(w.Hkv):
             assert pos in idx[b, h].cpu().tolist()
+
+
+def test_hata_decode_large_n_runs_the_unfused_chain(api):
+    """700K keys of one pair do not fit one cluster's shared memory: the hard-hash
+    decode then runs the unfused chain (byte-tables, scores through HBM, radix
+    top-k, attention) and still matches the oracle exactly on the index set."""
+    w = wl.shrink(wl.HATA_16, B=1, Hkv=1, Hq=4, N=700_000, k=2048)
+    inp = wl.make_inputs(w, DEV)
+    codes_nat, _ = pa.oracle_codes(inp, w)
+    codes = api.natural_to_ids(torch.from_numpy(codes_nat)).to(DEV)
+    O = torch.empty(w.B, w.Hq, w.d, device=DEV)
+    idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=DEV)
+    api.hata_decode(inp["Q"], inp["K"], inp["V"], inp["R128"], codes, w.N, w.k, w.scale, O, idx)
+    api.check_status()
+    R = inp["R128"].double().cpu().numpy()
+    Qg, K, V = pa.pair_arrays(inp, w, 0, 0)
+    o_ref, idx_ref, _ = ho.hata_decode_pair(Qg, K, V, R, codes_nat[0, 0, : w.N], w.k, w.scale)
+    assert np.array_equal(idx[0, 0].cpu().numpy(), idx_ref)
+    assert pa.row_rel_err(O[0].cpu().numpy(), o_ref) < pa.out_tol(w)

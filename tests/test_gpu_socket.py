@@ -482,3 +482,29 @@ def test_hash_keys_sign_band_statistics(api, capsys):
               f"({f32_band / tot:.2e}); differing: {diff_lit} in the 1e-6 band, {diff_f32} in the f32 band, "
               f"{diff_out} outside it")
     assert diff_out == 0
+
+
+def test_hash_tc_wait_timeout_drains_and_recovers(api):
+    """The tensor-core hashing kernel's failure path: with its main-loop wait
+    limit lowered to one clock (test hook), its waits give up while its TMA
+    copies and MMAs are in flight. It must stop, drain what it issued, free its
+    tensor memory and report SK_ERR_TIMEOUT; with the limit restored the next
+    call on the same context is bit-identical to a run before the failure."""
+    from hash_scored_top_b200 import _lib
+    w = wl.shrink(wl.LLAMA_8B, B=1, Hkv=2, Hq=8, N=8192, k=256)
+    inp = wl.make_inputs(w, DEV)
+    Ncap = inp["K"].shape[2]
+    ids0, nrm0 = api.empty_ids(w.B, w.Hkv, Ncap, w.L, DEV), api.empty_norms(w.B, w.Hkv, Ncap, DEV)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids0, nrm0, 0, w.N)
+    api.check_status()
+    ids1, nrm1 = api.empty_ids(w.B, w.Hkv, Ncap, w.L, DEV), api.empty_norms(w.B, w.Hkv, Ncap, DEV)
+    try:
+        assert _lib.lib.sk_test_set_wait_limit(1) == 0
+        api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids1, nrm1, 0, w.N)
+        with pytest.raises(RuntimeError, match="bounded wait"):
+            api.check_status()
+    finally:
+        assert _lib.lib.sk_test_set_wait_limit(0) == 0
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids1, nrm1, 0, w.N)
+    api.check_status()
+    assert torch.equal(ids0, ids1) and torch.equal(nrm0, nrm1)

@@ -8,7 +8,7 @@ are mapped to binary hash codes, and the top-k keys are ranked by comparing
 codes instead of computing exact q.k scores; section 2 states that only the
 rank order has to be preserved. The learned hash functions of the page need
 training and weights; seeded random hyperplanes stand in for them. Readings
-(listed in DESIGN.md):
+(each one pinned by a test):
 
 * code bit m of a row x is [x . r_m > 0] for 128 hyperplanes r_m, packed
   least significant bit first: bit m goes to byte m // 8, bit m % 8;

@@ -21,7 +21,7 @@ The page prints no formula for step 2. The form used here is
 p_l(b) = softmax_b( sum_j s_bj * z_lj / tau ), s_bj = +1 if bit j of b is
 set else -1, z_lj = q_hat . r_lj -- the plain reading of "projections ... go
 through a temperature softmax over all buckets". Readings adopted where the
-page is silent (all listed in the design doc):
+page is silent (each one pinned by a test):
 
 * the query is normalised before projecting (q_hat = q / |q|);
 * bit j of a bucket ID is hyperplane j of the table, least significant bit

@@ -1,6 +1,6 @@
 """Helpers shared by the GPU parity tests: oracle caches and comparisons.
 
-Tolerances (derived from the arithmetic, also listed in the design doc):
+Tolerances (derived from the arithmetic):
 
 * bucket IDs and hard-hash codes: bit-exact, except tables / code bytes with a
   projection |k . r| below max(1e-6, d * 2^-24 * sum_c |k_c r_c|) -- the f32

@@ -19,8 +19,9 @@
 // flight at once), then, once the factor kernel is done, of the pair's factor
 // image. Pass A, one thread per key: c_{h,i} summed over the tables in f32
 // (all lanes of a warp read the same factor row, so the lookups do not
-// conflict; f32, whose count is within (L + 2) 2^-24 of the exact one,
-// because the SM's float64 pipe is far narrower). Pass B: warps over keys,
+// conflict; f32: the counts feed an f32 weighted sum anyway, each is within
+// (L + 2) 2^-24 of the exact one, and the f32 factor image is half the
+// shared memory of a float64 one). Pass B: warps over keys,
 // lanes over value
 // columns, f32 accumulation of c v and of c. The warps' partials are added in
 // warp order; the splits' partials go to the workspace and the last CTA of

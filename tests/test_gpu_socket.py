@@ -508,3 +508,27 @@ def test_hash_tc_wait_timeout_drains_and_recovers(api):
     api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids1, nrm1, 0, w.N)
     api.check_status()
     assert torch.equal(ids0, ids1) and torch.equal(nrm0, nrm1)
+
+
+@pytest.mark.parametrize("tau", [1e-3, 1e4])
+def test_decode_at_the_temperature_limits(api, tau):
+    """Degenerate temperatures: tau -> 0 makes the soft assignment one-hot (the
+    score counts hard collisions, many keys tie), tau -> infinity makes every
+    table uniform (the score is the norm times a constant, ties wherever f16
+    norms are equal). The selection must stay a valid top-k with ties to the
+    lower index, and match the oracle's output where the sets agree."""
+    w = wl.shrink(wl.LLAMA_8B, B=1, Hkv=2, Hq=8, N=5000, k=5000 // 33, tau=tau)
+    inp = wl.make_inputs(w, DEV)
+    ids, nrm, ids_nat, norms, _ = _cache(api, w, inp)
+    _decode_and_compare(api, w, inp, ids, nrm, ids_nat, norms, pa.out_tol(w))
+
+
+def test_hash_keys_empty_range_is_a_no_op(api):
+    w = _w("g2_small_n")
+    inp = wl.make_inputs(w, DEV)
+    Ncap = inp["K"].shape[2]
+    ids = torch.full((w.B, w.Hkv, Ncap, api.ids_bytes_per_key(w.L)), 7, dtype=torch.uint8, device=DEV)
+    nrm = torch.full((w.B, w.Hkv, Ncap), 3.0, dtype=torch.float16, device=DEV)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, nrm, 5, 0)
+    api.check_status()
+    assert (ids == 7).all() and (nrm == 3.0).all()

@@ -5,6 +5,9 @@ pointers and sizes to the C entry point of the same name, and raises
 ``RuntimeError`` with the library's message on a non-zero status. All
 compute happens in the library's CUDA kernels on the current torch stream;
 torch only provides device memory (outputs and workspaces) and the stream.
+Without a ``ws`` argument a workspace of the size sk_workspace_bytes gives is
+allocated for the call; a ``ws`` that is passed goes to the library as it is
+(no size query on the host), which rejects one that is too small.
 There is no CPU fallback: if the library is missing the import of
 ``_lib`` fails loudly.
 """
@@ -156,7 +159,8 @@ def socket_score(Q, R, ids, norms, N: int, L: int, P: int, tau: float, scores, w
     _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
     _want(scores, torch.float32, (B, Hkv, Ncap), "scores")
     _want(R, torch.bfloat16, (L * P, d), "R")
-    ws = _workspace(workspace_bytes(OP_SCORE, B, Hq, Hkv, Ncap, N, d, L, P, 0), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_SCORE, B, Hq, Hkv, Ncap, N, d, L, P, 0), Q.device, ws)
     rc = _lib.lib.socket_score(_ptr(Q), _dtype_code(Q), _ptr(R), _ptr(ids), _ptr(norms), B, Hq, Hkv, Ncap, N, d, L, P,
                                ctypes.c_float(tau), _ptr(scores), _ptr(ws), _ws_bytes(ws), _stream())
     _check(rc, "socket_score")
@@ -180,7 +184,8 @@ def socket_sparse_attend(Q, K, V, idx, scale: float, O, ws=None):
     _want(V, Q.dtype, K.shape, "V")
     _want(idx, torch.int32, (B, Hkv, k), "idx")
     _want(O, torch.float32, (B, Hq, d), "O")
-    ws = _workspace(workspace_bytes(OP_SPARSE_ATTEND, B, Hq, Hkv, Ncap, k, d, 0, 0, k), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_SPARSE_ATTEND, B, Hq, Hkv, Ncap, k, d, 0, 0, k), Q.device, ws)
     rc = _lib.lib.socket_sparse_attend(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(idx), B, Hq, Hkv, Ncap, d, k,
                                        ctypes.c_float(scale), _ptr(O), _ptr(ws), _ws_bytes(ws), _stream())
     _check(rc, "socket_sparse_attend")
@@ -225,7 +230,8 @@ def socket_decode(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: float, k:
     _want(O, torch.float32, (B, Hq, d), "O")
     if idx_out is not None:
         _want(idx_out, torch.int32, (B, Hkv, k), "idx_out")
-    ws = _workspace(workspace_bytes(OP_DECODE, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_DECODE, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
     rc = _lib.lib.socket_decode(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R), _ptr(ids), _ptr(norms), B, Hq, Hkv,
                                 Ncap, N, d, L, P, ctypes.c_float(tau), k, ctypes.c_float(scale), _ptr(O),
                                 _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
@@ -245,7 +251,8 @@ def socket_decode_heads(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: flo
     _want(O, torch.float32, (B, Hq, d), "O")
     if idx_out is not None:
         _want(idx_out, torch.int32, (B, Hq, k), "idx_out")
-    ws = _workspace(workspace_bytes(OP_DECODE_HEADS, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_DECODE_HEADS, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
     rc = _lib.lib.socket_decode_heads(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R), _ptr(ids), _ptr(norms), B,
                                       Hq, Hkv, Ncap, N, d, L, P, ctypes.c_float(tau), k, ctypes.c_float(scale),
                                       _ptr(O), _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
@@ -267,7 +274,8 @@ def socket_decode_adaptive(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: 
     _want(idx, torch.int32, (B, U, k_max), "idx")
     _want(kcount, torch.int32, (B, U), "kcount")
     op = OP_DECODE_ADAPTIVE_HEADS if per_head else OP_DECODE_ADAPTIVE
-    ws = _workspace(workspace_bytes(op, B, Hq, Hkv, Ncap, N, d, L, P, k_max), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(op, B, Hq, Hkv, Ncap, N, d, L, P, k_max), Q.device, ws)
     rc = _lib.lib.socket_decode_adaptive(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R), _ptr(ids), _ptr(norms),
                                          B, Hq, Hkv, Ncap, N, d, L, P, ctypes.c_float(tau), int(bool(per_head)),
                                          ctypes.c_float(mass), k_min, k_max, ctypes.c_float(scale), _ptr(O),
@@ -299,7 +307,8 @@ def socket_sparse_attend_paged(Q, K_pool, V_pool, page_table, idx, scale: float,
     _want(page_table, torch.int32, (B, Hkv, max_pages), "page_table")
     _want(idx, torch.int32, (B, Hkv, k), "idx")
     _want(O, torch.float32, (B, Hq, d), "O")
-    ws = _workspace(workspace_bytes(OP_SPARSE_ATTEND_PAGED, B, Hq, Hkv, 32, k, d, 1, 1, k), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_SPARSE_ATTEND_PAGED, B, Hq, Hkv, 32, k, d, 1, 1, k), Q.device, ws)
     rc = _lib.lib.socket_sparse_attend_paged(_ptr(Q), _pool_ptr(K_pool), _pool_ptr(V_pool), _dtype_code(Q),
                                              _ptr(page_table), max_pages, page_size, num_pages, _ptr(idx), B, Hq,
                                              Hkv, d, k, ctypes.c_float(scale), _ptr(O), _ptr(ws), _ws_bytes(ws),
@@ -322,7 +331,8 @@ def socket_decode_paged(Q, K_pool, V_pool, page_table, R, ids, norms, N: int, L:
     _want(O, torch.float32, (B, Hq, d), "O")
     if idx_out is not None:
         _want(idx_out, torch.int32, (B, Hkv, k), "idx_out")
-    ws = _workspace(workspace_bytes(OP_DECODE_PAGED, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_DECODE_PAGED, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
     rc = _lib.lib.socket_decode_paged(_ptr(Q), _pool_ptr(K_pool), _pool_ptr(V_pool), _dtype_code(Q),
                                       _ptr(page_table), max_pages, page_size, num_pages, _ptr(R), _ptr(ids),
                                       _ptr(norms), B, Hq, Hkv, Ncap, N, d, L, P, ctypes.c_float(tau), k,
@@ -344,7 +354,8 @@ def socket_decode_append(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: fl
     _want(O, torch.float32, (B, Hq, d), "O")
     if idx_out is not None:
         _want(idx_out, torch.int32, (B, Hkv, k), "idx_out")
-    ws = _workspace(workspace_bytes(OP_DECODE, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_DECODE, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
     rc = _lib.lib.socket_decode_append(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R), _ptr(ids), _ptr(norms), B,
                                        Hq, Hkv, Ncap, N, d, L, P, ctypes.c_float(tau), k, ctypes.c_float(scale),
                                        _ptr(O), _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
@@ -359,7 +370,8 @@ def socket_select(Q, R, ids, norms, N: int, L: int, P: int, tau: float, k: int, 
     _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
     _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
     _want(idx, torch.int32, (B, Hkv, k), "idx")
-    ws = _workspace(workspace_bytes(OP_SELECT, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_SELECT, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
     rc = _lib.lib.socket_select(_ptr(Q), _dtype_code(Q), _ptr(R), _ptr(ids), _ptr(norms), B, Hq, Hkv, Ncap, N, d, L,
                                 P, ctypes.c_float(tau), k, _ptr(idx), _ptr(ws), _ws_bytes(ws), _stream())
     _check(rc, "socket_select")
@@ -387,7 +399,8 @@ def hata_decode(Q, K, V, R128, codes, N: int, k: int, scale: float, O, idx_out=N
     _want(O, torch.float32, (B, Hq, d), "O")
     if idx_out is not None:
         _want(idx_out, torch.int32, (B, Hkv, k), "idx_out")
-    ws = _workspace(workspace_bytes(OP_HATA_DECODE, B, Hq, Hkv, Ncap, N, d, 16, 8, k), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_HATA_DECODE, B, Hq, Hkv, Ncap, N, d, 16, 8, k), Q.device, ws)
     rc = _lib.lib.hata_decode(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), _ptr(R128), _ptr(codes), B, Hq, Hkv, Ncap, N,
                               d, k, ctypes.c_float(scale), _ptr(O), _ptr(idx_out), _ptr(ws), _ws_bytes(ws), _stream())
     _check(rc, "hata_decode")
@@ -400,7 +413,8 @@ def dense_decode(Q, K, V, N: int, scale: float, O, ws=None):
     _want(K, Q.dtype, K.shape, "K")
     _want(V, Q.dtype, K.shape, "V")
     _want(O, torch.float32, (B, Hq, d), "O")
-    ws = _workspace(workspace_bytes(OP_DENSE_DECODE, B, Hq, Hkv, Ncap, N, d), Q.device, ws)
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_DENSE_DECODE, B, Hq, Hkv, Ncap, N, d), Q.device, ws)
     rc = _lib.lib.dense_decode(_ptr(Q), _ptr(K), _ptr(V), _dtype_code(K), B, Hq, Hkv, Ncap, N, d, ctypes.c_float(scale),
                                _ptr(O), _ptr(ws), _ws_bytes(ws), _stream())
     _check(rc, "dense_decode")
@@ -417,7 +431,8 @@ def socket_soft_count_attend(Q, V, R, ids, idx, L: int, P: int, tau: float, O, w
     _want(idx, torch.int32, (B, Hkv, k), "idx")
     _want(O, torch.float32, (B, Hq, d), "O")
     if ws is None:              # a caller's workspace is passed as it is: the library checks its size
-        ws = _workspace(workspace_bytes(OP_SOFT_COUNT, B, Hq, Hkv, Ncap, k, d, L, P, k), Q.device, ws)
+        if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+            ws = _workspace(workspace_bytes(OP_SOFT_COUNT, B, Hq, Hkv, Ncap, k, d, L, P, k), Q.device, ws)
     rc = _lib.lib.socket_soft_count_attend(_ptr(Q), _ptr(V), _dtype_code(V), _ptr(R), _ptr(ids), _ptr(idx), B, Hq,
                                            Hkv, Ncap, d, L, P, ctypes.c_float(tau), k, _ptr(O), _ptr(ws),
                                            _ws_bytes(ws), _stream())

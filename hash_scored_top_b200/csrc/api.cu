@@ -670,17 +670,19 @@ int paged_attend_impl(const void* Q, const void* K_pool, const void* V_pool, sk_
                        true, s);
 }
 
-// Workspace of a decode step: the index list (when idx_out is NULL) then the
-// attention workspace.
-size_t decode_ws_bytes(int B, int Hq, int Hkv, int k, int d) {
+// Workspace of a decode step: the index list (when idx_out is NULL), the
+// attention workspace, then room for the units' table images (used when the
+// selection takes more than one wave of clusters; see decode_impl).
+size_t decode_ws_bytes(int B, int Hq, int Hkv, int k, int d, int L) {
   const int pairs = B * Hkv, G = Hq / Hkv;
-  return align256((size_t)pairs * k * 4) + attend_ws_bytes(pairs, attend_splits(k, pairs, false), G, d);
+  return align256((size_t)pairs * k * 4) + attend_ws_bytes(pairs, attend_splits(k, pairs, false), G, d) +
+         align256(table_image_bytes(pairs, L));
 }
 
 // Workspace of the unfused decode chain: tables, scores, then a decode workspace.
 size_t chain_ws_bytes(int B, int Hq, int Hkv, int Ncap, int d, int L, int k) {
   const int pairs = B * Hkv;
-  return align256(table_image_bytes(pairs, L)) + align256((size_t)pairs * Ncap * 4) + decode_ws_bytes(B, Hq, Hkv, k, d);
+  return align256(table_image_bytes(pairs, L)) + align256((size_t)pairs * Ncap * 4) + decode_ws_bytes(B, Hq, Hkv, k, d, L);
 }
 
 // Workspace of the selection alone: none when it runs as one cluster kernel,
@@ -1027,7 +1029,7 @@ int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const 
   const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, hata, max_cluster_size());
 
   const size_t need = !attend ? select_ws_bytes(fp, pairs, Ncap, L)
-                      : fp.C > 0 ? decode_ws_bytes(B, Hq, Hkv, k, d) : chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
+                      : fp.C > 0 ? decode_ws_bytes(B, Hq, Hkv, k, d, L) : chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
   if (need > 0 && (ws == nullptr || ws_bytes < need))
     return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
   char* w = reinterpret_cast<char*>(ws);
@@ -1081,7 +1083,18 @@ int decode_impl(const void* Q, const void* K, const void* V, sk_dtype kv, const 
   p.tau = tau;
   p.scale = scale;
   p.pair_div = pair_div;
-  SK_TRY(launch_select(p, pairs, d, kv, hata, after_append, s));
+  // A selection of more than one wave of clusters gets its units' tables
+  // from a table kernel run once beforehand: every later wave would otherwise
+  // rebuild them (the hard-hash byte-tables take ~13 us per CTA). The
+  // selection then starts after that kernel (an ordinary launch).
+  const bool precompute = attend && (long)pairs * fp.C > kNumSMs;
+  if (precompute) {
+    float* T = reinterpret_cast<float*>(w + attend_ws_bytes(pairs, splits, G, d));
+    if (hata) SK_TRY(launch_hamming_tables(Q, kv, R, B, Hq, Hkv, d, T, s));
+    else SK_TRY(launch_tables(Q, kv, R, B, Hq, Hkv, d, L, P, tau, T, s));
+    p.tables = T;
+  }
+  SK_TRY(launch_select(p, pairs, d, kv, hata, after_append && !precompute, s));
   if (!attend) return SK_OK;
   return launch_attend(Q, K, V, kv, idx, B, Hq, Hkv, Ncap, k, d, scale, O, w, attend_ws_bytes(pairs, splits, G, d),
                        true, false, s, true, pair_div);
@@ -1175,7 +1188,7 @@ int socket_decode_append(const void* Q, const void* K, const void* V, sk_dtype k
     const int pairs = B * Hkv, G = Hq / Hkv;
     if (G > 8) return fail(SK_ERR_UNSUPPORTED, "group size G=%d > 8", G);
     const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, false, max_cluster_size());
-    const size_t need = fp.C > 0 ? decode_ws_bytes(B, Hq, Hkv, k, d) : chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
+    const size_t need = fp.C > 0 ? decode_ws_bytes(B, Hq, Hkv, k, d, L) : chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
     if (ws == nullptr || ws_bytes < need)
       return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
   }
@@ -1496,14 +1509,14 @@ size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d
       // the unfused chain runs when the selection cannot hold a pair's keys on
       // chip; 8-CTA clusters are always available, 16-CTA ones may not be
       const FusedPlan fp = plan_select(pairs, N, k, G, d, L, P, op == SK_OP_HATA_DECODE, 8);
-      if (fp.C > 0) return decode_ws_bytes(B, Hq, Hkv, k, d);
+      if (fp.C > 0) return decode_ws_bytes(B, Hq, Hkv, k, d, L);
       return chain_ws_bytes(B, Hq, Hkv, Ncap, d, L, k);
     }
     case SK_OP_DECODE_HEADS: {
       // one unit per query head: Hq "KV heads" of group size 1
       if (k < 1 || N < 1 || L < 1 || L > kMaxL || P < 1 || P > 8) return bad;
       const FusedPlan fp = plan_select(B * Hq, N, k, 1, d, L, P, false, 8);
-      if (fp.C > 0) return decode_ws_bytes(B, Hq, Hq, k, d);
+      if (fp.C > 0) return decode_ws_bytes(B, Hq, Hq, k, d, L);
       return chain_ws_bytes(B, Hq, Hq, Ncap, d, L, k);
     }
     case SK_OP_SPARSE_ATTEND_PAGED:

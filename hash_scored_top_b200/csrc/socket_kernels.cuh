@@ -62,6 +62,10 @@ struct FusedParams {
   // query head is its own unit (Hkv then counts query heads); the cached
   // IDs, norms, keys and values of unit u are those of pair u / pair_div
   int pair_div = 1;
+  // optional: the units' table images [units][nch][256][64], built by a
+  // table kernel beforehand (bucket_table_kernel / hamming_table_kernel);
+  // every CTA copies its unit's image instead of building tables
+  const float* tables = nullptr;
 };
 
 constexpr int PHASES = 24;
@@ -302,7 +306,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
   }
   if (tid == 0) sh->over_local = 0u;
   for (int i = tid; i < BIN_COUNT; i += blockDim.x) hist[0][i] = 0u;     // hist0 + hist1: the selection bins
-  zero_table_padding_all<LP>(tab0, tab1, p.L, p.P);
+  if (p.tables == nullptr) zero_table_padding_all<LP>(tab0, tab1, p.L, p.P);   // a copied image has its zeros
   if (rank == 0 && tid == 0 && p.counters) p.counters[pair] = 0u;     // for the attention kernel's merge
   stamp(p.phase_ts, 8);
 
@@ -310,7 +314,14 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
   // stores every entry into all its column copies in every CTA of the cluster.
   const QT* Qg = reinterpret_cast<const QT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
   const int per = ((p.L + C - 1) / C + 3) & ~3;
-  {
+  if (p.tables != nullptr) {
+    // precomputed: this CTA copies its unit's image (L2-resident) into its
+    // own tables; no table entry crosses CTAs
+    const uint4* src = reinterpret_cast<const uint4*>(p.tables + (size_t)pair * NCH * 256 * TABLE_COLS);
+    uint4* dst = reinterpret_cast<uint4*>(tab0);           // tab1 follows tab0 directly
+    for (int e = tid; e < NCH * 256 * TABLE_COLS / 4; e += blockDim.x) dst[e] = __ldg(src + e);
+    cluster_wait();                                          // pairs with the arrive at entry
+  } else {
     const int l0 = min(p.L, rank * per);
     const int nl = min(p.L, l0 + per) - l0;
     const uint32_t t0a = fs.tbl0, t1a = fs.tbl1;
@@ -337,8 +348,9 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
     auto before_store = [] { cluster_wait(); };    // every CTA of the cluster has started
     void* scratch = sptr<void>(dyn, fs.base, fs.keysA);
     if constexpr (HATA) {
-      // the 16 byte-tables of the hard-hash variant are cheap (popcounts of
-      // the query codes): every CTA builds all of them in its own memory
+      // the 16 byte-tables of the hard-hash variant (popcounts of the query
+      // codes): every CTA builds all of them in its own memory (about 13 us;
+      // decodes of several waves copy them from a table kernel's image instead)
       auto local_store = [=](int bb, int l, float v) {
         float* row = tab0 + bb * TABLE_COLS;
         for (int x = l; x < TABLE_COLS; x += 16) row[x] = v;
@@ -357,7 +369,11 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
     }
   }
   stamp(p.phase_ts, 9);
-  if constexpr (!HATA) cluster_sync();     // every table entry has landed in every CTA
+  if (p.tables != nullptr) {
+    __syncthreads();                       // this CTA's copy is complete
+  } else if constexpr (!HATA) {
+    cluster_sync();                        // every table entry has landed in every CTA
+  }
   // Launched as the programmatic dependent of the key-append kernel, the
   // kernel got here while that kernel may still run: the bucket IDs and norms
   // are read only after it completed (a no-op for an ordinary launch).

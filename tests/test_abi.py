@@ -46,9 +46,13 @@ def test_every_declared_symbol_is_exported(lib):
 def test_workspace_sizes(lib):
     from hash_scored_top_b200 import api
     # decode at the 100K-token Llama-8B-like shape: index list + attention partials + counters
+    # + room for the pairs' table images (one 64 KB chunk each, used when the
+    # selection takes more than one wave)
     idx_bytes = 397312                       # 32 pairs x 3103 int32, rounded up to 256 bytes
     part_bytes = 32 * 9 * 4 * 130 * 4        # 9 splits x 4 heads x (m, l, o[128]) per pair
-    assert api.workspace_bytes(api.OP_DECODE, 4, 32, 8, 102400, 102400, 128, 32, 8, 3103) == idx_bytes + part_bytes + 256
+    tables = 32 * 65536
+    assert (api.workspace_bytes(api.OP_DECODE, 4, 32, 8, 102400, 102400, 128, 32, 8, 3103)
+            == idx_bytes + part_bytes + 256 + tables)
     assert api.workspace_bytes(api.OP_SCORE, 4, 32, 8, 102400, 102400, 128, 32, 8, 0) == 32 * 65536
     assert api.workspace_bytes(api.OP_SCORE, 8, 32, 4, 143360, 143360, 128, 48, 8, 0) == 32 * 2 * 65536
     n = api.workspace_bytes(api.OP_SPARSE_ATTEND, 4, 32, 8, 102400, 102400, 128, 0, 0, 3103)

@@ -102,3 +102,30 @@ def test_hata_decode_large_n_runs_the_unfused_chain(api):
     o_ref, idx_ref, _ = ho.hata_decode_pair(Qg, K, V, R, codes_nat[0, 0, : w.N], w.k, w.scale)
     assert np.array_equal(idx[0, 0].cpu().numpy(), idx_ref)
     assert pa.row_rel_err(O[0].cpu().numpy(), o_ref) < pa.out_tol(w)
+
+
+def test_hata_decode_over_several_waves(api):
+    """128 pairs of 40K keys need 2-CTA clusters, 256 CTAs: more than one wave,
+    so the decode builds the byte-tables once in a table kernel and the
+    selection copies them. Sampled pairs carry the oracle's codes and are
+    compared exactly on the index set."""
+    w = wl.shrink(wl.HATA_16, B=16, Hkv=8, Hq=32, N=40000, k=1024)
+    inp = wl.make_inputs(w, DEV)
+    sample = [(0, 0), (5, 3), (11, 6), (15, 7)]
+    codes_nat, _ = pa.oracle_codes(inp, w, sample)
+    Ncap = inp["K"].shape[2]
+    codes = api.empty_codes(w.B, w.Hkv, Ncap, DEV)
+    api.hata_hash_keys(inp["K"], inp["R128"], codes)
+    codes_o = api.natural_to_ids(torch.from_numpy(codes_nat)).to(DEV)
+    for b, h in sample:
+        codes[b, h] = codes_o[b, h]
+    O = torch.empty(w.B, w.Hq, w.d, device=DEV)
+    idx = torch.empty(w.B, w.Hkv, w.k, dtype=torch.int32, device=DEV)
+    api.hata_decode(inp["Q"], inp["K"], inp["V"], inp["R128"], codes, w.N, w.k, w.scale, O, idx)
+    api.check_status()
+    R = inp["R128"].double().cpu().numpy()
+    for b, h in sample:
+        Qg, K, V = pa.pair_arrays(inp, w, b, h)
+        o_ref, idx_ref, _ = ho.hata_decode_pair(Qg, K, V, R, codes_nat[b, h, : w.N], w.k, w.scale)
+        assert np.array_equal(idx[b, h].cpu().numpy(), idx_ref), (b, h)
+        assert pa.row_rel_err(O[b, h * w.G:(h + 1) * w.G].cpu().numpy(), o_ref) < pa.out_tol(w)

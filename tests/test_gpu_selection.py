@@ -195,3 +195,41 @@ def test_decode_adaptive_rejects_bad_arguments(api):
         with pytest.raises(RuntimeError):
             api.socket_decode_adaptive(inp["Q"], inp["K"], inp["V"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, mass,
                                        k_min, k_max, w.scale, O, idx, kc)
+
+
+def test_decode_heads_over_several_waves(api):
+    """128 query-head units of 40K keys need 2-CTA clusters, 256 CTAs: more
+    than one wave, so the decode builds the units' tables once in a table
+    kernel and the selection copies them. Sampled units against the oracle."""
+    w = wl.shrink(wl.LLAMA_8B, B=4, Hkv=8, Hq=32, N=40000, k=40000 // 33, needles=0)
+    inp = wl.make_inputs(w, DEV)
+    sample = [(0, 0), (1, 3), (2, 5), (3, 7)]
+    ids_nat, norms, _ = pa.oracle_socket_cache(inp, w, sample)
+    # every pair needs a cache; the sampled pairs carry the oracle's
+    Ncap = inp["K"].shape[2]
+    ids = api.empty_ids(w.B, w.Hkv, Ncap, w.L, DEV)
+    nrm = api.empty_norms(w.B, w.Hkv, Ncap, DEV)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, nrm)
+    ids_o, nrm_o = pa.to_device_cache(ids_nat, norms, DEV)
+    for b, h in sample:
+        ids[b, h] = ids_o[b, h]
+        nrm[b, h] = nrm_o[b, h]
+    O = torch.empty(w.B, w.Hq, w.d, device=DEV)
+    idx = torch.empty(w.B, w.Hq, w.k, dtype=torch.int32, device=DEV)
+    api.socket_decode_heads(inp["Q"], inp["K"], inp["V"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, w.k, w.scale, O,
+                            idx)
+    api.check_status()
+    R = inp["R"].double().cpu().numpy()
+    compared = 0
+    for b, h in sample:
+        Qg, K, V = pa.pair_arrays(inp, w, b, h)
+        o_ref, idx_ref, s_ref = sr.socket_decode_pair_per_head(Qg, K, V, R, ids_nat[b, h, : w.N], norms[b, h, : w.N],
+                                                               w.L, w.P, w.tau, w.k, w.scale)
+        for g in range(w.G):
+            got = idx[b, h * w.G + g].cpu().numpy()
+            assert pa.check_selection(s_ref[g], got, w.k) == [], (b, h, g)
+            if np.array_equal(got, idx_ref[g]):
+                compared += 1
+                err = pa.row_rel_err(O[b, h * w.G + g:h * w.G + g + 1].cpu().numpy(), o_ref[g:g + 1])
+                assert err < pa.out_tol(w), (err, b, h, g)
+    assert compared >= 12

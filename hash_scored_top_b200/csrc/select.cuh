@@ -520,24 +520,11 @@ __device__ bool binned_select(KeyAt key_at, KeyAddr key_addr, int n, uint32_t k,
     bool ok = over < k && warp_pick_desc(ch, cl, over, k, 63, cb, before, ccnt);
     if (ok) {
       const int f_hi = cb * 64 + 63 - 2 * lane;
-      // every CTA's two fine bins loaded first (the remote loads overlap),
-      // then added in rank order
-      uint32_t vh[SEL_MAX_C], vl[SEL_MAX_C];
-#pragma unroll
-      for (int c = 0; c < SEL_MAX_C; ++c) {
-        if (c < C) {
-          const uint32_t* h = cluster.map_shared_rank(hist, c);
-          vh[c] = h[f_hi];
-          vl[c] = h[f_hi - 1];
-        }
-      }
       uint32_t fh = 0, fl = 0;
-#pragma unroll
-      for (int c = 0; c < SEL_MAX_C; ++c) {
-        if (c < C) {
-          fh += vh[c];
-          fl += vl[c];
-        }
+      for (int c = 0; c < C; ++c) {
+        const uint32_t* h = cluster.map_shared_rank(hist, c);
+        fh += h[f_hi];
+        fl += h[f_hi - 1];
       }
       ok = warp_pick_desc(fh, fl, before, k, cb * 64 + 63, bstar, above, in_bin);
     }

@@ -128,3 +128,66 @@ def test_host_validation_rejects_without_launching(lib):
     # unknown dtype
     rc, msg = _rc_and_msg(lib, L.dense_decode, p, p, p, 7, 1, 4, 1, 64, 64, 128, 0.1, p, p, 1 << 20, null)
     assert rc == 1 and "dtype" in msg
+
+
+def test_host_validation_of_the_later_entry_points(lib):
+    """The per-head, adaptive, estimator and paged entry points reject bad
+    arguments on the host, before any launch or device query."""
+    L = lib.lib
+    p = ctypes.c_void_p(256)
+    null = None
+    # per-head decode: k > N
+    rc, msg = _rc_and_msg(lib, L.socket_decode_heads, p, p, p, 1, p, p, p, 1, 8, 2, 64, 32, 128, 8, 4, 0.5, 40,
+                          0.1, p, null, null, 0, null)
+    assert rc == 1 and "k=40" in msg
+    # adaptive decode: mass outside (0, 1], k_min > k_max, k_max > N, per_head not 0/1
+    for mass, kmin, kmax, ph, want in [(0.0, 1, 8, 0, "mass"), (1.5, 1, 8, 0, "mass"), (0.5, 9, 8, 0, "k_min"),
+                                       (0.5, 1, 65, 0, "k_min"), (0.5, 1, 8, 2, "per_head")]:
+        rc, msg = _rc_and_msg(lib, L.socket_decode_adaptive, p, p, p, 1, p, p, p, 1, 8, 2, 64, 64, 128, 8, 4, 0.5, ph,
+                              mass, kmin, kmax, 0.1, p, p, p, null, 0, null)
+        assert rc == 1 and want in msg, (mass, kmin, kmax, ph, msg)
+    # adaptive decode: the index list and counts are required
+    rc, msg = _rc_and_msg(lib, L.socket_decode_adaptive, p, p, p, 1, p, p, p, 1, 8, 2, 64, 64, 128, 8, 4, 0.5, 0,
+                          0.5, 1, 8, 0.1, p, null, p, null, 0, null)
+    assert rc == 1 and "idx is NULL" in msg
+    # estimator: group of 9 heads, k = 0, no workspace
+    rc, msg = _rc_and_msg(lib, L.socket_soft_count_attend, p, p, 1, p, p, p, 1, 9, 1, 64, 128, 8, 4, 0.5, 8, p,
+                          null, 0, null)
+    assert rc == 2 and "G=9" in msg
+    rc, msg = _rc_and_msg(lib, L.socket_soft_count_attend, p, p, 1, p, p, p, 1, 8, 2, 64, 128, 8, 4, 0.5, 0, p,
+                          null, 0, null)
+    assert rc == 1 and "k=0" in msg
+    rc, msg = _rc_and_msg(lib, L.socket_soft_count_attend, p, p, 1, p, p, p, 1, 8, 2, 64, 128, 8, 4, 0.5, 8, p,
+                          null, 0, null)
+    assert rc == 5 and "workspace" in msg
+    # paged attention: page parameters must be >= 1, the page table present
+    rc, msg = _rc_and_msg(lib, L.socket_sparse_attend_paged, p, p, p, 1, p, 4, 0, 8, p, 1, 8, 2, 128, 16, 0.1, p,
+                          null, 0, null)
+    assert rc == 1 and "page_size=0" in msg
+    rc, msg = _rc_and_msg(lib, L.socket_sparse_attend_paged, p, p, p, 1, null, 4, 16, 8, p, 1, 8, 2, 128, 16, 0.1,
+                          p, null, 0, null)
+    assert rc == 1 and "page_table is NULL" in msg
+    # paged decode: the pages must cover N keys
+    rc, msg = _rc_and_msg(lib, L.socket_decode_paged, p, p, p, 1, p, 2, 16, 8, p, p, p, 1, 8, 2, 64, 64, 128, 8, 4,
+                          0.5, 8, 0.1, p, null, null, 0, null)
+    assert rc == 1 and "< N" in msg
+
+
+def test_workspace_queries_of_the_later_entry_points(lib):
+    from hash_scored_top_b200 import api
+    # per-query-head decode: 128 units of group size 1
+    n_heads = api.workspace_bytes(api.OP_DECODE_HEADS, 4, 32, 8, 102400, 102400, 128, 32, 8, 3103)
+    n_group = api.workspace_bytes(api.OP_DECODE, 4, 32, 8, 102400, 102400, 128, 32, 8, 3103)
+    assert n_heads > n_group > 0
+    # adaptive decode: tables, scores (4 B per key and unit) and attention for k_max
+    n_ad = api.workspace_bytes(api.OP_DECODE_ADAPTIVE, 4, 32, 8, 102400, 102400, 128, 32, 8, 12412)
+    assert n_ad > 32 * 65536 + 32 * 102400 * 4
+    assert api.workspace_bytes(api.OP_DECODE_ADAPTIVE_HEADS, 4, 32, 8, 102400, 102400, 128, 32, 8, 12412) > n_ad
+    # estimator: factor image (f32, 32 per head and table), partials, counters
+    n_est = api.workspace_bytes(api.OP_SOFT_COUNT, 4, 32, 8, 102400, 3103, 128, 32, 8, 3103)
+    assert n_est >= 32 * 4 * 32 * 32 * 4
+    # paged: a host pool stages k rows of K and V per pair
+    n_pg = api.workspace_bytes(api.OP_SPARSE_ATTEND_PAGED, 4, 32, 8, 32, 3103, 128, 1, 1, 3103)
+    assert n_pg >= 2 * 32 * 3103 * 128 * 4
+    with pytest.raises(ValueError):
+        api.workspace_bytes(api.OP_SOFT_COUNT, 1, 9, 1, 64, 8, 128, 8, 4, 8)       # G = 9

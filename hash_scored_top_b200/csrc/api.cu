@@ -807,7 +807,7 @@ EstPlan plan_estimator(int pairs, int k, int G, int d, int L, int kv_bytes) {
   if (fixed + per_key > budget) return ep;                           // nothing fits
   const int fit = (int)((budget - fixed) / per_key);
   const int ctas = (two ? 2 : 1) * kNumSMs;
-  const int want_splits = std::max(1, (ctas + pairs - 1) / pairs);
+  const int want_splits = std::max(1, ctas / pairs);                  // at most one wave
   // at least 64 keys per CTA (fewer splits to merge), as far as they fit
   int kps = std::min(fit, std::max(64, (k + want_splits - 1) / want_splits));
   kps = std::max(1, kps);
@@ -824,7 +824,7 @@ size_t est_ws_bytes(int pairs, int splits, int G, int d, int L) {
   return est_factor_bytes(pairs, G, L) + est_part_bytes(pairs, splits, G, d) + align256((size_t)pairs * 4);
 }
 
-template <int D, typename KVT>
+template <int D, typename KVT, int LP>
 int launch_estimator_t(const EstFactorParams& fp, const EstParams& ep, int pairs, size_t smem, cudaStream_t s) {
   const int G = fp.Hq / fp.Hkv;
   auto fk = est_factor_kernel<D, KVT>;
@@ -832,7 +832,7 @@ int launch_estimator_t(const EstFactorParams& fp, const EstParams& ep, int pairs
   if (set_kernel_smem(fk, fsm) != cudaSuccess) return check_launch("cudaFuncSetAttribute(estimator factors smem)");
   fk<<<dim3(pairs, (fp.L + EST_TABLES_PER_CTA - 1) / EST_TABLES_PER_CTA), 256, fsm, s>>>(fp);
   SK_TRY(check_launch("est_factor_kernel"));
-  auto kern = soft_count_attend_kernel<D, KVT>;
+  auto kern = soft_count_attend_kernel<D, KVT, LP>;
   if (set_kernel_smem(kern, smem) != cudaSuccess) return check_launch("cudaFuncSetAttribute(estimator smem)");
   // programmatic dependent of the factor kernel: the copies of the keys' ID
   // and value rows overlap it; the factor image is read after its completion
@@ -849,6 +849,15 @@ int launch_estimator_t(const EstFactorParams& fp, const EstParams& ep, int pairs
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, ep);
   if (e != cudaSuccess) return fail(SK_ERR_CUDA, "estimator launch: %s", cudaGetErrorString(e));
   return check_launch("soft_count_attend_kernel");
+}
+
+template <int LP>
+int launch_estimator_d(const EstFactorParams& fp, const EstParams& ep, int pairs, size_t smem, int d, sk_dtype kv,
+                       cudaStream_t s) {
+  if (d == 128) return kv == SK_BF16 ? launch_estimator_t<128, __nv_bfloat16, LP>(fp, ep, pairs, smem, s)
+                                     : launch_estimator_t<128, float, LP>(fp, ep, pairs, smem, s);
+  return kv == SK_BF16 ? launch_estimator_t<64, __nv_bfloat16, LP>(fp, ep, pairs, smem, s)
+                       : launch_estimator_t<64, float, LP>(fp, ep, pairs, smem, s);
 }
 
 }  // namespace
@@ -1463,10 +1472,12 @@ int socket_soft_count_attend(const void* Q, const void* V, sk_dtype kv, const vo
   cudaStream_t s = as_stream(stream);
   const cudaError_t e = cudaMemsetAsync(ep.counters, 0, (size_t)pairs * 4, s);
   if (e != cudaSuccess) return fail(SK_ERR_CUDA, "counter reset: %s", cudaGetErrorString(e));
-  if (d == 128) return kv == SK_BF16 ? launch_estimator_t<128, __nv_bfloat16>(fp, ep, pairs, plan.smem, s)
-                                     : launch_estimator_t<128, float>(fp, ep, pairs, plan.smem, s);
-  return kv == SK_BF16 ? launch_estimator_t<64, __nv_bfloat16>(fp, ep, pairs, plan.smem, s)
-                       : launch_estimator_t<64, float>(fp, ep, pairs, plan.smem, s);
+  switch (ids_bytes_per_key(L)) {
+    case 16: return launch_estimator_d<16>(fp, ep, pairs, plan.smem, d, kv, s);
+    case 32: return launch_estimator_d<32>(fp, ep, pairs, plan.smem, d, kv, s);
+    case 48: return launch_estimator_d<48>(fp, ep, pairs, plan.smem, d, kv, s);
+    default: return launch_estimator_d<64>(fp, ep, pairs, plan.smem, d, kv, s);
+  }
 }
 
 size_t sk_workspace_bytes(int op, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, int k) {

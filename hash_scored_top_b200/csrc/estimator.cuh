@@ -15,9 +15,9 @@
 // soft_count_attend_kernel, grid (pairs, splits), launched as the factor
 // kernel's programmatic dependent: CTA (pair, s) takes keys
 // idx[s * keys_per_split ..], and first issues asynchronous copies of all
-// their ID rows and value rows into shared memory (every copy of the CTA in
-// flight at once), then, once the factor kernel is done, of the pair's factor
-// image. Pass A, one thread per key: c_{h,i} summed over the tables in f32
+// their value rows into shared memory (every copy of the CTA in flight at
+// once), then, once the factor kernel is done, of the pair's factor image;
+// each key's ID row is read into registers when its count is formed. Pass A, one thread per key: c_{h,i} summed over the tables in f32
 // (all lanes of a warp read the same factor row, so the lookups do not
 // conflict; f32: the counts feed an f32 weighted sum anyway, each is within
 // (L + 2) 2^-24 of the exact one, and the f32 factor image is half the
@@ -29,6 +29,7 @@
 #pragma once
 
 #include "hash_kernels.cuh"
+#include "hash_tc.cuh"
 #include "score.cuh"
 #include "table.cuh"
 
@@ -84,7 +85,7 @@ __host__ __device__ inline size_t est_align16(size_t x) { return (x + 15) & ~(si
 // image (reused for the warps' partials), the counts, the key indices, the
 // staged ID rows and value rows, a flag word. Offsets in bytes.
 struct EstSmem {
-  size_t counts, keys, idrows, vrows, flag, total;
+  size_t counts, keys, vrows, flag, total;
 };
 __host__ __device__ inline EstSmem est_smem_plan(int G, int d, int L, int kps, int kv_bytes) {
   EstSmem s;
@@ -92,15 +93,53 @@ __host__ __device__ inline EstSmem est_smem_plan(int G, int d, int L, int kps, i
   const size_t w = (size_t)EST_WARPS * G * (d + 1) * 4;
   s.counts = est_align16(f > w ? f : w);
   s.keys = s.counts + est_align16((size_t)kps * G * 4);
-  s.idrows = s.keys + est_align16((size_t)kps * 4);
-  s.vrows = s.idrows + (size_t)kps * ids_bytes_per_key(L);
+  s.vrows = s.keys + est_align16((size_t)kps * 4);
   s.flag = s.vrows + (size_t)kps * d * kv_bytes;
   s.total = s.flag + 16;
   return s;
 }
 // Bytes of shared memory per key in the plan above (for the host's choice of kps).
 __host__ __device__ inline size_t est_bytes_per_key(int G, int d, int L, int kv_bytes) {
-  return (size_t)G * 4 + 4 + ids_bytes_per_key(L) + (size_t)d * kv_bytes;
+  (void)L;
+  return (size_t)G * 4 + 4 + (size_t)d * kv_bytes;
+}
+
+// The ID bytes of one key in table order: its rotated row (see common.cuh)
+// loaded into registers and rotated back per chunk, so that byte l holds the
+// ID of table l (a compile-time position in the unrolled loops below).
+template <int LP>
+struct KeyRowIds {
+  uint32_t w[LP / 4];
+};
+template <int LP>
+__device__ __forceinline__ void load_key_row_ids(KeyRowIds<LP>& r, const uint8_t* __restrict__ row, int key) {
+#pragma unroll
+  for (int i = 0; i < LP / 16; ++i) {
+    const uint4 x = ldg_stream(row + 16 * i);
+    r.w[4 * i] = x.x;
+    r.w[4 * i + 1] = x.y;
+    r.w[4 * i + 2] = x.z;
+    r.w[4 * i + 3] = x.w;
+  }
+  // chunk 0: S = 16 (LP = 16) or 32; byte j holds table (j + key) mod S
+  constexpr int S0 = LP == 16 ? 16 : 32;
+  {
+    uint32_t c[S0 / 4];
+#pragma unroll
+    for (int i = 0; i < S0 / 4; ++i) c[i] = r.w[i];
+    rotate_bytes<S0 / 4>(c, (S0 - key % S0) % S0);
+#pragma unroll
+    for (int i = 0; i < S0 / 4; ++i) r.w[i] = c[i];
+  }
+  if constexpr (LP > 32) {
+    constexpr int S1 = LP - 32;
+    uint32_t c[S1 / 4];
+#pragma unroll
+    for (int i = 0; i < S1 / 4; ++i) c[i] = r.w[8 + i];
+    rotate_bytes<S1 / 4>(c, (S1 - key % S1) % S1);
+#pragma unroll
+    for (int i = 0; i < S1 / 4; ++i) r.w[8 + i] = c[i];
+  }
 }
 
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
@@ -165,7 +204,7 @@ __device__ __forceinline__ void row2_from_smem(const unsigned char* row, int lan
   v[2] = v[3] = 0.f;
 }
 
-template <int D, typename KVT>
+template <int D, typename KVT, int LP>
 __global__ void __launch_bounds__(EST_THREADS, 2) soft_count_attend_kernel(const EstParams p) {
   extern __shared__ __align__(16) unsigned char smem[];
   constexpr int VPL = D / 32;                        // value columns per lane (2 or 4)
@@ -178,12 +217,10 @@ __global__ void __launch_bounds__(EST_THREADS, 2) soft_count_attend_kernel(const
   const int i0 = split * p.keys_per_split;
   const int cnt = max(0, min(p.k - i0, p.keys_per_split));
   const size_t pair_keys = (size_t)pair * p.Ncap;
-  const int LPB = ids_bytes_per_key(L);
   const EstSmem sp = est_smem_plan(G, D, L, p.keys_per_split, (int)sizeof(KVT));
   float* fs = reinterpret_cast<float*>(smem);                    // [G][L][EST_F]
   float* cnts = reinterpret_cast<float*>(smem + sp.counts);      // [cnt][G]
   int* keys_s = reinterpret_cast<int*>(smem + sp.keys);          // [cnt]
-  unsigned char* idrows = smem + sp.idrows;                      // [cnt][LPB]
   unsigned char* vrows = smem + sp.vrows;                        // [cnt][ROW]
   unsigned int* last_flag = reinterpret_cast<unsigned int*>(smem + sp.flag);
 
@@ -194,12 +231,8 @@ __global__ void __launch_bounds__(EST_THREADS, 2) soft_count_attend_kernel(const
   __syncthreads();
   est_stamp(p.phase_ts, 1);
   {
-    const int id_chunks = LPB / 16, v_chunks = ROW / 16;
-    const uint32_t id_base = smem_u32(idrows), v_base = smem_u32(vrows);
-    for (int e = tid; e < cnt * id_chunks; e += EST_THREADS) {
-      const int j = e / id_chunks, c = e % id_chunks;
-      cp_async16(id_base + (uint32_t)(j * LPB + 16 * c), p.ids + (pair_keys + keys_s[j]) * LPB + 16 * c);
-    }
+    const int v_chunks = ROW / 16;
+    const uint32_t v_base = smem_u32(vrows);
     const unsigned char* V = reinterpret_cast<const unsigned char*>(p.V);
     for (int e = tid; e < cnt * v_chunks; e += EST_THREADS) {
       const int j = e / v_chunks, c = e % v_chunks;
@@ -220,48 +253,44 @@ __global__ void __launch_bounds__(EST_THREADS, 2) soft_count_attend_kernel(const
   __syncthreads();
   est_stamp(p.phase_ts, 4);
 
-  // ---- pass A: counts, one thread per key. Inside chunk c (tables 32c ..)
-  // the ID of table 32c + t sits at byte 32c + (t - key) mod S. Eight tables
-  // at a time: their IDs and factor pairs are loaded together, their
-  // probabilities (lo * hi) added as a fixed tree, then to the running count.
-  // The factors are float64 results rounded to f32, and the count is an f32
-  // sum: its relative error stays below (L + 2) 2^-24.
+  // ---- pass A: counts, one thread per key. The key's ID row is read into
+  // registers and rotated back to table order (load_key_row_ids), so table l
+  // is byte l. Eight tables at a time: their IDs and factor pairs are loaded
+  // together, their probabilities (lo * hi) added as a fixed tree, then to the
+  // running count. The factors are float64 results rounded to f32, and the
+  // count is an f32 sum: its relative error stays below (L + 2) 2^-24.
   const int plo = p.P / 2;
   const int mlo = (1 << plo) - 1;
   for (int j = tid; j < cnt; j += EST_THREADS) {
     const int key = keys_s[j];
-    const unsigned char* row = idrows + (size_t)j * LPB;
+    KeyRowIds<LP> r;
+    load_key_row_ids<LP>(r, p.ids + (pair_keys + key) * LP, key);
     float c[8];
 #pragma unroll
     for (int h = 0; h < 8; ++h) c[h] = 0.f;
-    for (int ch = 0; 32 * ch < L; ++ch) {
-      const int S = id_chunk_size(L, ch);
-      const int nt = min(S, L - 32 * ch);
-      const int p0 = (S - key % S) % S;              // byte of table 32c + 0
-      for (int t0 = 0; t0 < nt; t0 += 8) {
-        // every load is unconditional (no branches in the unrolled body): a
-        // table past the chunk's last reads table nt - 1 and is masked out
+#pragma unroll
+    for (int l0 = 0; l0 < LP; l0 += 8) {
+      if (l0 < L) {
+        // every load is unconditional inside the group: a table past the
+        // last reads table L - 1 and is masked out
         int idv[8];
         bool live[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          const int t = min(t0 + u, nt - 1);
-          int pos = p0 + t;
-          pos = pos >= S ? pos - S : pos;
-          idv[u] = (int)row[32 * ch + pos];
-          live[u] = t0 + u < nt;
+          const int l = l0 + u;
+          idv[u] = (int)((r.w[l >> 2] >> (8 * (l & 3))) & 255u);
+          live[u] = l < L;
         }
-        const float* fr = fs + (size_t)(32 * ch) * EST_F;
 #pragma unroll
         for (int h = 0; h < 8; ++h) {
           if (h < G) {
-            const float* f = fr + (size_t)h * L * EST_F;
+            const float* f = fs + (size_t)h * L * EST_F;
             float q[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-              const int t = min(t0 + u, nt - 1);
-              const float a = f[t * EST_F + (idv[u] & mlo)];
-              const float bq = f[t * EST_F + 16 + (idv[u] >> plo)];
+              const int lc = min(l0 + u, L - 1);
+              const float a = f[lc * EST_F + (idv[u] & mlo)];
+              const float bq = f[lc * EST_F + 16 + (idv[u] >> plo)];
               q[u] = live[u] ? a * bq : 0.f;
             }
             c[h] += ((q[0] + q[1]) + (q[2] + q[3])) + ((q[4] + q[5]) + (q[6] + q[7]));

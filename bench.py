@@ -52,6 +52,9 @@ def parse_args():
     ap.add_argument("--no-others", action="store_true", help="skip the records of the other workloads")
     ap.add_argument("--prefill-only", action="store_true",
                     help="build one cache and time only the prefill hashing (a small command for profilers)")
+    ap.add_argument("--estimator-only", action="store_true",
+                    help="build one cache and time only the soft-count estimator over its selection "
+                         "(a small command for profilers)")
     ap.add_argument("--clock-window", type=float, default=0.5,
                     help="seconds of untimed replays under the clock sampler right before the timed region")
     return ap.parse_args()
@@ -238,8 +241,14 @@ def run_ours(args, world, rank, local):
     w = wl.WORKLOADS[args.workload]
     device = torch.device("cuda", local)
     # one cache already streams more than L2 per step for the hard-hash workload (17 GB of K/V each)
-    n_caches = 1 if (w.hata or args.prefill_only) else args.caches
+    n_caches = 1 if (w.hata or args.prefill_only or args.estimator_only) else args.caches
     caches = build_caches(w, api, wl, n_caches, device, rank)
+    if args.estimator_only:
+        peak, _ = load_peaks()
+        rec = run_estimator(w, api, caches, device, required_bytes(w), peak)
+        rec.update({"workload": w.name, "launches": "1 selection, then the factor and attend kernels of "
+                                                     "4 warm-up calls, then CUDA graph replays"})
+        return rec
     if args.prefill_only:
         peak, _ = load_peaks()
         rec = run_prefill_hash(w, api, caches, device, peak)

@@ -420,20 +420,24 @@ def run_ours(args, world, rank, local):
         "gpu_launches": 3 * steps,
         "clocks": clocks,
     }
-    if not args.no_others:
+    # the records beyond the headline run at N = 1 only: the scaling runs hold
+    # every GPU of the node, and these records add minutes and per-rank host
+    # memory (pinned pools) without measuring scaling
+    if not args.no_others and world == 1:
         result["workloads"] = {}
         for name in wl.WORKLOADS:
             if name != w.name:
                 result["workloads"][name] = run_workload_record(name, api, wl, device, peak)
     if not args.no_extras and not w.hata:
         result["e2e"] = run_e2e(args, w, api, caches, device, world, ws)
+    if not args.no_extras and not w.hata and world == 1:
         result["dense_decode"] = run_dense(w, api, caches, device, rb, peak)
         result["prefill_hash"] = run_prefill_hash(w, api, caches, device, peak)
         result["soft_count_estimator"] = run_estimator(w, api, caches, device, rb, peak)
         result["per_head_decode"] = run_heads(w, api, caches, device, peak)
         result["adaptive_decode"] = run_adaptive(w, api, caches, device, peak)
         result["paged_decode"] = run_paged(w, api, caches, device, rb, peak)
-        if rank == 0 and world == 1:
+        if rank == 0:
             result["cpu_baseline"] = cpu_baseline(w, caches[0], sample_pairs=8)
     del g_step, g_dec, g_sel
     return result

@@ -181,9 +181,11 @@ size_t sk_noalloc_scratch_bytes(void);
  * attention kernel, launched as its programmatic dependent, gathers the
  * selected K/V rows and merges its key splits in a fixed order. The result
  * equals socket_score -> socket_topk -> socket_sparse_attend. idx_out
- * (nullable) receives the selected indices [B][Hkv][k] ascending. Shapes
- * whose keys do not fit one cluster's shared memory run that unfused chain
- * instead (same results). Requires 1 <= P <= 8, 1 <= L <= 64, 1 <= k <= N,
+ * (nullable) receives the selected indices [B][Hkv][k] ascending. When the
+ * selection takes more than one wave of clusters, a table kernel first builds
+ * every pair's bucket tables once (into ws) and the selection kernel copies
+ * them (same tables, same results). Shapes whose keys do not fit one
+ * cluster's shared memory run that unfused chain instead (same results). Requires 1 <= P <= 8, 1 <= L <= 64, 1 <= k <= N,
  * tau > 0, G <= 8. ws: sk_workspace_bytes(SK_OP_DECODE, ...) bytes.
  */
 int socket_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R,

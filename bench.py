@@ -52,6 +52,8 @@ def parse_args():
     ap.add_argument("--no-others", action="store_true", help="skip the records of the other workloads")
     ap.add_argument("--prefill-only", action="store_true",
                     help="build one cache and time only the prefill hashing (a small command for profilers)")
+    ap.add_argument("--adaptive-only", action="store_true",
+                    help="build the caches and time only the adaptive-k decode (a small command for profilers)")
     ap.add_argument("--estimator-only", action="store_true",
                     help="build one cache and time only the soft-count estimator over its selection "
                          "(a small command for profilers)")
@@ -243,6 +245,11 @@ def run_ours(args, world, rank, local):
     # one cache already streams more than L2 per step for the hard-hash workload (17 GB of K/V each)
     n_caches = 1 if (w.hata or args.prefill_only or args.estimator_only) else args.caches
     caches = build_caches(w, api, wl, n_caches, device, rank)
+    if args.adaptive_only:
+        peak, _ = load_peaks()
+        rec = run_adaptive(w, api, caches, device, peak)
+        rec.update({"workload": w.name})
+        return rec
     if args.estimator_only:
         peak, _ = load_peaks()
         rec = run_estimator(w, api, caches, device, required_bytes(w), peak)

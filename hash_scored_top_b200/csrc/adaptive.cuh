@@ -16,6 +16,12 @@
 // the decision is deterministic. Truncation moves a unit's mass by at most
 // one part in 2^62 / (keys), far below the scores' own f32 rounding. Then the
 // plain count-based radix select takes the top k.
+//
+// Shared-memory traffic: a bin's mass is two 32-bit words (low word, high
+// word plus the carry out of the low word), so every histogram update is a
+// native 32-bit atomic; the level-0 key counts are taken while the scores
+// are loaded and serve both the mass search and the top-k; each level of the
+// mass search has bins of its own, so one cluster barrier per level suffices.
 #pragma once
 
 #include "select.cuh"
@@ -38,9 +44,10 @@ struct AdaptShared {
   uint32_t bin, cnt_above, found, pad;
 };
 
-constexpr uint32_t kAdaptFixedBytes = (uint32_t)(((sizeof(SelShared) + 15) & ~15) +
-                                                 4 * (hist_words(0) + hist_words(1) + hist_words(2)) +
-                                                 8 * (1 << 11) + ((sizeof(AdaptShared) + 15) & ~15));
+constexpr int kAdaptHistWords = hist_words(0) + hist_words(1) + hist_words(2);
+// counts (one word per bin) and masses (two words per bin) of the three levels
+constexpr uint32_t kAdaptFixedBytes = (uint32_t)(((sizeof(SelShared) + 15) & ~15) + 4 * kAdaptHistWords +
+                                                 8 * kAdaptHistWords + ((sizeof(AdaptShared) + 15) & ~15));
 
 // Block-wide exclusive scan of one unsigned 64-bit value per thread.
 __device__ __forceinline__ unsigned long long block_exclusive_scan_u64(unsigned long long v, AdaptShared* as) {
@@ -71,9 +78,10 @@ __device__ __forceinline__ unsigned long long block_exclusive_scan_u64(unsigned 
 // One level of the mass search over nbins bins (descending bin order across
 // the threads, BPT bins each): the cluster-wide mass and count of every bin,
 // then the bin where the running mass from the top first reaches `need`.
+// mlo, mhi: the level's low and high mass words; hc: its key counts.
 template <int BPT>
-__device__ void resolve_mass_level(const unsigned long long* mh, const uint32_t* hc, int nbins, unsigned long long need,
-                                   int C, SelShared* sh, AdaptShared* as) {
+__device__ void resolve_mass_level(const uint32_t* mlo, const uint32_t* mhi, const uint32_t* hc, int nbins,
+                                   unsigned long long need, int C, SelShared* sh, AdaptShared* as) {
   cg::cluster_group cluster = cg::this_cluster();
   const int tid = threadIdx.x;
   const int base = nbins - (tid + 1) * BPT;
@@ -93,11 +101,12 @@ __device__ void resolve_mass_level(const unsigned long long* mh, const uint32_t*
   }
   if (mine) {
     for (int r = 0; r < C; ++r) {
-      const unsigned long long* pm = cluster.map_shared_rank(mh, r) + base;
+      const uint32_t* pl = cluster.map_shared_rank(mlo, r) + base;
+      const uint32_t* ph = cluster.map_shared_rank(mhi, r) + base;
       const uint32_t* pc = cluster.map_shared_rank(hc, r) + base;
 #pragma unroll
       for (int j = 0; j < BPT; ++j) {
-        m[j] += pm[j];
+        m[j] += ((unsigned long long)ph[j] << 32) | pl[j];
         c[j] += pc[j];
       }
     }
@@ -129,8 +138,16 @@ __device__ void resolve_mass_level(const unsigned long long* mh, const uint32_t*
   __syncthreads();
 }
 
+// floor(x * 2^sc) for the bit pattern `key` of a finite float x >= 0, from
+// its IEEE-754 binary32 fields: x = (2^23 + f) * 2^(e - 150) for a biased
+// exponent e >= 1, and f * 2^-149 for e = 0. Callers have x <= S < 2^(62 - sc),
+// so a left shift stays below 2^62; a right shift truncates, as floor does.
 __device__ __forceinline__ unsigned long long fixed_mass(uint32_t key, int sc) {
-  return __double2ull_rz(ldexp((double)__uint_as_float(key), sc));
+  const uint32_t e = key >> 23, f = key & 0x7fffffu;
+  const unsigned long long m = e != 0u ? (unsigned long long)(f | 0x800000u) : (unsigned long long)f;
+  const int sh = (e != 0u ? (int)e - 150 : -149) + sc;
+  if (sh >= 0) return m << sh;
+  return sh > -32 ? (m >> -sh) : 0ull;
 }
 
 __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(const AdaptParams p) {
@@ -146,9 +163,9 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
   uint32_t* h0 = reinterpret_cast<uint32_t*>(a);
   uint32_t* h1 = h0 + hist_words(0);
   uint32_t* h2 = h1 + hist_words(1);
-  a += 4 * (hist_words(0) + hist_words(1) + hist_words(2));
-  unsigned long long* mh = reinterpret_cast<unsigned long long*>(a);   // [2048] mass per bin
-  a += 8 * (1 << 11);
+  // masses, level by level: low words of the level's bins, then high words
+  uint32_t* mass_words = h0 + kAdaptHistWords;
+  a += 12 * kAdaptHistWords;
   AdaptShared* as = reinterpret_cast<AdaptShared*>(a);
   a += (sizeof(AdaptShared) + 15) & ~15;
   uint32_t* keys = reinterpret_cast<uint32_t*>(a);
@@ -157,16 +174,37 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
   // store into another CTA (every CTA of the cluster has started by then)
   cluster_arrive_relaxed();
 
-  for (int i = tid; i < hist_words(0) + hist_words(1) + hist_words(2); i += blockDim.x) h0[i] = 0u;
-  for (int i = tid; i < (1 << 11); i += blockDim.x) mh[i] = 0ull;
+  for (int i = tid; i < 3 * kAdaptHistWords; i += blockDim.x) h0[i] = 0u;
+  __syncthreads();
   const int k0 = rank * p.keys_per_cta;
   const int n_local = max(0, min(p.N - k0, p.keys_per_cta));
   const float* src = p.scores + (size_t)unit * p.Ncap + k0;
+  constexpr uint32_t mask0 = (1u << sel_bits(0)) - 1u;
+  // the keys, this CTA's float64 sum and its level-0 key counts
   double ssum = 0.0;
-  for (int i = tid; i < n_local; i += blockDim.x) {
+  int n_vec = 0;
+  if ((reinterpret_cast<uintptr_t>(src) & 15) == 0) {
+    n_vec = n_local & ~3;
+    for (int g = tid; g < n_vec / 4; g += blockDim.x) {
+      const float4 v = reinterpret_cast<const float4*>(src)[g];
+      const uint4 kk = make_uint4(key_of(fmaxf(v.x, 0.0f)), key_of(fmaxf(v.y, 0.0f)), key_of(fmaxf(v.z, 0.0f)),
+                                  key_of(fmaxf(v.w, 0.0f)));
+      reinterpret_cast<uint4*>(keys)[g] = kk;
+      ssum += (double)__uint_as_float(kk.x);
+      ssum += (double)__uint_as_float(kk.y);
+      ssum += (double)__uint_as_float(kk.z);
+      ssum += (double)__uint_as_float(kk.w);
+      atomicAdd(&h0[(kk.x >> sel_shift(0)) & mask0], 1u);
+      atomicAdd(&h0[(kk.y >> sel_shift(0)) & mask0], 1u);
+      atomicAdd(&h0[(kk.z >> sel_shift(0)) & mask0], 1u);
+      atomicAdd(&h0[(kk.w >> sel_shift(0)) & mask0], 1u);
+    }
+  }
+  for (int i = n_vec + tid; i < n_local; i += blockDim.x) {
     const uint32_t key = key_of(fmaxf(src[i], 0.0f));
     keys[i] = key;
     ssum += (double)__uint_as_float(key);
+    atomicAdd(&h0[(key >> sel_shift(0)) & mask0], 1u);
   }
   // the CTA's sum in a fixed order (lanes, then warps), sent to every CTA
 #pragma unroll
@@ -181,7 +219,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
     for (int r = 0; r < C; ++r) *cluster.map_shared_rank(&as->part[rank], r) = t;
   }
   __syncthreads();
-  cluster_sync();
+  cluster_sync();   // every CTA's sum and level-0 counts are complete
   double S = 0.0;
   for (int r = 0; r < C; ++r) S += as->part[r];
 
@@ -199,29 +237,33 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
     uint32_t prefix = 0, cnt_total = 0;
     int pshift = 32;
     bool reached = true;
+    uint32_t* mlo = mass_words;
 #pragma unroll 1
     for (int lvl = 0; lvl < SEL_LEVELS; ++lvl) {
       const int bits = sel_bits(lvl), shift = sel_shift(lvl);
       const uint32_t mask = (1u << bits) - 1u;
+      uint32_t* mhi = mlo + (1 << bits);
+      uint32_t* hc = hist[lvl];
       for (int i = tid; i < n_local; i += blockDim.x) {
         const uint32_t k = keys[i];
         if (pshift >= 32 || (k >> pshift) == prefix) {
           const uint32_t bn = (k >> shift) & mask;
-          atomicAdd(&mh[bn], fixed_mass(k, sc));
-          atomicAdd(&hist[lvl][bn], 1u);
+          const unsigned long long fm = fixed_mass(k, sc);
+          const uint32_t lo = (uint32_t)fm;
+          const uint32_t old = atomicAdd(&mlo[bn], lo);
+          const uint32_t hi = (uint32_t)(fm >> 32) + (old + lo < old ? 1u : 0u);   // carry out of the low word
+          if (hi != 0u) atomicAdd(&mhi[bn], hi);
+          if (lvl > 0) atomicAdd(&hc[bn], 1u);      // level 0 was counted with the load
         }
       }
       __syncthreads();
       cluster_sync();
-      if (bits == 11) resolve_mass_level<2>(mh, hist[lvl], 1 << 11, need, C, sh, as);
-      else resolve_mass_level<1>(mh, hist[lvl], 1 << 9, need, C, sh, as);
+      if (bits == 11) resolve_mass_level<2>(mlo, mhi, hc, 1 << 11, need, C, sh, as);
+      else resolve_mass_level<1>(mlo, mhi, hc, 1 << 9, need, C, sh, as);
       const bool found = as->found != 0u;
       const uint32_t bn = as->bin, ca = as->cnt_above;
       const unsigned long long ma = as->mass_above;
-      cluster_sync();                              // every CTA has read every CTA's bins
-      for (int i = tid; i < (1 << 11); i += blockDim.x) mh[i] = 0ull;
-      for (int i = tid; i < hist_words(lvl); i += blockDim.x) hist[lvl][i] = 0u;
-      __syncthreads();
+      // the next level writes bins of its own, so other CTAs may still read these
       if (!found) {                                // the whole unit's mass stays below the target
         reached = false;
         break;
@@ -230,6 +272,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
       cnt_total += ca;
       prefix = (prefix << bits) | bn;
       pshift = shift;
+      mlo = mhi + (1 << bits);
     }
     if (reached) {
       const unsigned long long ft = fixed_mass(prefix, sc);   // every key of the final bin equals prefix
@@ -237,13 +280,14 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
     } else {
       k_mass = n_all;
     }
+    cluster_sync();                                // every CTA has read every CTA's level-1 and level-2 bins
+    for (int i = tid; i < hist_words(1) + hist_words(2); i += blockDim.x) h1[i] = 0u;
+    __syncthreads();
   }
   const int k = max(p.k_min, min(k_mass, min(p.k_max, n_all)));
 
-  // ---- the exact top-k with that k (the bins are zero again)
-  histogram_pass([&](int i) { return keys[i]; }, n_local, sel_shift(0), sel_bits(0), 32, 0u, h0);
-  __syncthreads();
-  cluster_sync();
+  // ---- the exact top-k with that k (level-0 counts from the load, published
+  // by the barrier after the sums; the other levels are zero)
   auto key_at = [&](int i) -> uint32_t { return keys[i]; };
   const SelThreshold th = cluster_threshold<FUSED_THREADS>(key_at, n_local, hist, (uint32_t)k, C, sh);
   int* out = p.idx + (size_t)unit * p.k_max;

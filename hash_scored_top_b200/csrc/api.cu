@@ -423,9 +423,11 @@ int launch_topk(const float* scores, int pairs, int Ncap, int N, int k, int* idx
 int launch_adaptive_topk(const float* scores, int units, int Ncap, int N, float mass, int k_min, int k_max, int* idx,
                          int* kcount, cudaStream_t s) {
   const int cap = (int)((SMEM_DYN_MAX - kAdaptFixedBytes) / 4);
+  // keys per CTA: a multiple of 4, so every CTA's scores start on 16 bytes
+  auto per_cta = [&](int c) { return ((N + c - 1) / c + 3) & ~3; };
   int C = 0;
   for (int c = 1; c <= max_cluster_size(); c *= 2)
-    if ((N + c - 1) / c <= cap) {
+    if (per_cta(c) <= cap) {
       C = c;
       break;
     }
@@ -439,7 +441,7 @@ int launch_adaptive_topk(const float* scores, int units, int Ncap, int N, float 
   ap.k_min = k_min;
   ap.k_max = k_max;
   ap.C = C;
-  ap.keys_per_cta = (N + C - 1) / C;
+  ap.keys_per_cta = per_cta(C);
   ap.mass = mass;
   const size_t smem = kAdaptFixedBytes + (size_t)ap.keys_per_cta * 4;
   auto kern = socket_adaptive_topk_kernel;

@@ -104,10 +104,29 @@ __device__ void resolve_mass_level(const uint32_t* mlo, const uint32_t* mhi, con
       const uint32_t* pl = cluster.map_shared_rank(mlo, r) + base;
       const uint32_t* ph = cluster.map_shared_rank(mhi, r) + base;
       const uint32_t* pc = cluster.map_shared_rank(hc, r) + base;
+      if constexpr (BPT % 4 == 0) {
+        // 16-byte reads: a read of another CTA's shared memory costs about
+        // the same whatever its width
 #pragma unroll
-      for (int j = 0; j < BPT; ++j) {
-        m[j] += ((unsigned long long)ph[j] << 32) | pl[j];
-        c[j] += pc[j];
+        for (int j = 0; j < BPT; j += 4) {
+          const uint4 l = *reinterpret_cast<const uint4*>(pl + j);
+          const uint4 h = *reinterpret_cast<const uint4*>(ph + j);
+          const uint4 n = *reinterpret_cast<const uint4*>(pc + j);
+          m[j] += ((unsigned long long)h.x << 32) | l.x;
+          m[j + 1] += ((unsigned long long)h.y << 32) | l.y;
+          m[j + 2] += ((unsigned long long)h.z << 32) | l.z;
+          m[j + 3] += ((unsigned long long)h.w << 32) | l.w;
+          c[j] += n.x;
+          c[j + 1] += n.y;
+          c[j + 2] += n.z;
+          c[j + 3] += n.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < BPT; ++j) {
+          m[j] += ((unsigned long long)ph[j] << 32) | pl[j];
+          c[j] += pc[j];
+        }
       }
     }
   }
@@ -149,6 +168,24 @@ __device__ __forceinline__ unsigned long long fixed_mass(uint32_t key, int sc) {
   if (sh >= 0) return m << sh;
   return sh > -32 ? (m >> -sh) : 0ull;
 }
+
+// f(key) for this CTA's keys i < n, read four at a time (keys: 16-byte
+// aligned, readable up to n rounded up to 4).
+template <typename F>
+__device__ __forceinline__ void for_each_key4(const uint32_t* keys, int n, F f) {
+  const int n4 = (n + 3) >> 2;
+  for (int g = threadIdx.x; g < n4; g += blockDim.x) {
+    const uint4 q = reinterpret_cast<const uint4*>(keys)[g];
+    const uint32_t kv[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j)
+      if (4 * g + j < n) f(kv[j]);
+  }
+}
+
+// Keys a CTA holds in shared memory: room for a multiple of 128 keys (the
+// compaction reads whole 128-key chunks).
+__host__ __device__ constexpr int adapt_key_slots(int keys_per_cta) { return (keys_per_cta + 127) & ~127; }
 
 __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(const AdaptParams p) {
   extern __shared__ __align__(1024) unsigned char dyn[];
@@ -206,6 +243,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
     ssum += (double)__uint_as_float(key);
     atomicAdd(&h0[(key >> sel_shift(0)) & mask0], 1u);
   }
+  for (int i = n_local + tid; i < ((n_local + 127) & ~127); i += blockDim.x) keys[i] = 0u;   // the last chunk's tail
   // the CTA's sum in a fixed order (lanes, then warps), sent to every CTA
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ssum += __shfl_xor_sync(FULL, ssum, o);
@@ -244,8 +282,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
       const uint32_t mask = (1u << bits) - 1u;
       uint32_t* mhi = mlo + (1 << bits);
       uint32_t* hc = hist[lvl];
-      for (int i = tid; i < n_local; i += blockDim.x) {
-        const uint32_t k = keys[i];
+      for_each_key4(keys, n_local, [&](uint32_t k) {
         if (pshift >= 32 || (k >> pshift) == prefix) {
           const uint32_t bn = (k >> shift) & mask;
           const unsigned long long fm = fixed_mass(k, sc);
@@ -255,11 +292,10 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
           if (hi != 0u) atomicAdd(&mhi[bn], hi);
           if (lvl > 0) atomicAdd(&hc[bn], 1u);      // level 0 was counted with the load
         }
-      }
+      });
       __syncthreads();
       cluster_sync();
-      if (bits == 11) resolve_mass_level<2>(mlo, mhi, hc, 1 << 11, need, C, sh, as);
-      else resolve_mass_level<1>(mlo, mhi, hc, 1 << 9, need, C, sh, as);
+      resolve_mass_level<4>(mlo, mhi, hc, 1 << bits, need, C, sh, as);
       const bool found = as->found != 0u;
       const uint32_t bn = as->bin, ca = as->cnt_above;
       const unsigned long long ma = as->mass_above;
@@ -287,13 +323,23 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
   const int k = max(p.k_min, min(k_mass, min(p.k_max, n_all)));
 
   // ---- the exact top-k with that k (level-0 counts from the load, published
-  // by the barrier after the sums; the other levels are zero)
-  auto key_at = [&](int i) -> uint32_t { return keys[i]; };
-  const SelThreshold th = cluster_threshold<FUSED_THREADS>(key_at, n_local, hist, (uint32_t)k, C, sh);
+  // by the barrier after the sums; the other levels are zero), then the
+  // thread-contiguous compaction, staged in the mass bins, which no CTA reads
+  // any more
+  auto pass = [&](int shift, int bits, int pshift, uint32_t prefix, uint32_t* h) {
+    const uint32_t mask = (1u << bits) - 1u;
+    for_each_key4(keys, n_local, [&](uint32_t key) {
+      if (pshift >= 32 || (key >> pshift) == prefix) atomicAdd(&h[(key >> shift) & mask], 1u);
+    });
+  };
+  const SelThreshold th = cluster_threshold_by<FUSED_THREADS / 2>(pass, hist, (uint32_t)k, C, sh);
   int* out = p.idx + (size_t)unit * p.k_max;
-  ordered_compact(key_at, n_local, th, C, rank, sh, [&](uint32_t pos, int i) {
+  const uint32_t keys_s = (uint32_t)__cvta_generic_to_shared(keys);
+  auto key_addr = [&](int i) -> uint32_t { return keys_s + 4u * (uint32_t)i; };
+  auto g0_of = [&](int c) { return c * p.keys_per_cta; };
+  contiguous_compact(key_addr, n_local, th, C, rank, g0_of, sh, [&](uint32_t pos, int i) {
     if (pos < (uint32_t)k) out[pos] = k0 + i;
-  });
+  }, out, (uint32_t)k, mass_words, 2 * kAdaptHistWords);
   if (rank == 0) {
     for (int j = k + tid; j < p.k_max; j += blockDim.x) out[j] = -1;
     if (tid == 0) p.kcount[unit] = k;

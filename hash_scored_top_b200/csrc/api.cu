@@ -427,7 +427,7 @@ int launch_adaptive_topk(const float* scores, int units, int Ncap, int N, float 
   auto per_cta = [&](int c) { return ((N + c - 1) / c + 3) & ~3; };
   int C = 0;
   for (int c = 1; c <= max_cluster_size(); c *= 2)
-    if (per_cta(c) <= cap) {
+    if (adapt_key_slots(per_cta(c)) <= cap) {
       C = c;
       break;
     }
@@ -443,7 +443,7 @@ int launch_adaptive_topk(const float* scores, int units, int Ncap, int N, float 
   ap.C = C;
   ap.keys_per_cta = per_cta(C);
   ap.mass = mass;
-  const size_t smem = kAdaptFixedBytes + (size_t)ap.keys_per_cta * 4;
+  const size_t smem = kAdaptFixedBytes + (size_t)adapt_key_slots(ap.keys_per_cta) * 4;
   auto kern = socket_adaptive_topk_kernel;
   if (set_kernel_smem(kern, smem, C > 8) != cudaSuccess) return check_launch("cudaFuncSetAttribute(adaptive smem)");
   cudaLaunchConfig_t cfg = {};

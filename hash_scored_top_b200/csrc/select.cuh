@@ -161,12 +161,14 @@ struct SelThreshold {
   uint32_t take_eq;  // keys == t: the first take_eq of them in index order (UINT_MAX: all)
 };
 
-// The three-level search (NT threads per CTA). hist[0] holds this CTA's
-// level-0 histogram and the cluster has synchronised since it was filled;
-// hist[1], hist[2] are zeroed.
-template <int NT, typename KeyAt>
-__device__ SelThreshold cluster_threshold(KeyAt key_at, int n_local, uint32_t* const* hist, uint32_t k, int C,
-                                          SelShared* sh, unsigned long long* ts = nullptr) {
+// The three-level search (bins resolved as if by NT threads per CTA: 2048 / NT
+// bins per thread). hist[0] holds this CTA's level-0 histogram and the
+// cluster has synchronised since it was filled; hist[1], hist[2] are zeroed.
+// pass(shift, bits, pshift, prefix, hist) counts this CTA's keys that match
+// the prefix into the level's histogram, as histogram_pass does.
+template <int NT, typename Pass>
+__device__ SelThreshold cluster_threshold_by(Pass pass, uint32_t* const* hist, uint32_t k, int C, SelShared* sh,
+                                             unsigned long long* ts = nullptr) {
   uint32_t need = k;
   uint32_t prefix = 0;
   int pshift = 32;
@@ -174,7 +176,7 @@ __device__ SelThreshold cluster_threshold(KeyAt key_at, int n_local, uint32_t* c
 #pragma unroll
   for (int lvl = 0; lvl < SEL_LEVELS; ++lvl) {
     if (lvl > 0) {
-      histogram_pass(key_at, n_local, sel_shift(lvl), sel_bits(lvl), pshift, prefix, hist[lvl]);
+      pass(sel_shift(lvl), sel_bits(lvl), pshift, prefix, hist[lvl]);
       __syncthreads();
       sel_stamp(ts, 14 + 2 * lvl);
       cluster_sync();
@@ -195,6 +197,16 @@ __device__ SelThreshold cluster_threshold(KeyAt key_at, int n_local, uint32_t* c
     }
   }
   return th;
+}
+
+// cluster_threshold_by with the plain histogram pass over key_at(i), i < n_local.
+template <int NT, typename KeyAt>
+__device__ SelThreshold cluster_threshold(KeyAt key_at, int n_local, uint32_t* const* hist, uint32_t k, int C,
+                                          SelShared* sh, unsigned long long* ts = nullptr) {
+  auto pass = [&](int shift, int bits, int pshift, uint32_t prefix, uint32_t* h) {
+    histogram_pass(key_at, n_local, shift, bits, pshift, prefix, h);
+  };
+  return cluster_threshold_by<NT>(pass, hist, k, C, sh, ts);
 }
 
 // Ordered compaction of this CTA's selected keys (ascending index i in [0, n)):

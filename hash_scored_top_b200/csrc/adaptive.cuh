@@ -264,6 +264,8 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
   // ---- the adaptive k
   const int n_all = p.N;
   int k_mass = 0;
+  bool reached = false;          // the search ended on one key value v, with n_above keys above it
+  uint32_t v = 0u, n_above = 0u;
   unsigned long long target = 0ull;
   int sc = 0;
   if (S > 0.0) {
@@ -274,7 +276,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
     unsigned long long need = target;
     uint32_t prefix = 0, cnt_total = 0;
     int pshift = 32;
-    bool reached = true;
+    reached = true;
     uint32_t* mlo = mass_words;
 #pragma unroll 1
     for (int lvl = 0; lvl < SEL_LEVELS; ++lvl) {
@@ -313,26 +315,40 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
     if (reached) {
       const unsigned long long ft = fixed_mass(prefix, sc);   // every key of the final bin equals prefix
       k_mass = (int)cnt_total + (int)((need + ft - 1ull) / ft);
+      v = prefix;
+      n_above = cnt_total;
     } else {
       k_mass = n_all;
     }
-    cluster_sync();                                // every CTA has read every CTA's level-1 and level-2 bins
-    for (int i = tid; i < hist_words(1) + hist_words(2); i += blockDim.x) h1[i] = 0u;
-    __syncthreads();
   }
   const int k = max(p.k_min, min(k_mass, min(p.k_max, n_all)));
 
-  // ---- the exact top-k with that k (level-0 counts from the load, published
-  // by the barrier after the sums; the other levels are zero), then the
-  // thread-contiguous compaction, staged in the mass bins, which no CTA reads
-  // any more
+  // ---- the exact top-k with that k: from the mass search's last bin when k
+  // was not clamped, else by the count search (level-0 counts from the load,
+  // published by the barrier after the sums; the other levels zeroed). Then
+  // the thread-contiguous compaction, staged in the mass bins (its barrier
+  // comes before the first staged write, and after every CTA's last read of
+  // them)
   auto pass = [&](int shift, int bits, int pshift, uint32_t prefix, uint32_t* h) {
     const uint32_t mask = (1u << bits) - 1u;
     for_each_key4(keys, n_local, [&](uint32_t key) {
       if (pshift >= 32 || (key >> pshift) == prefix) atomicAdd(&h[(key >> shift) & mask], 1u);
     });
   };
-  const SelThreshold th = cluster_threshold_by<FUSED_THREADS / 2>(pass, hist, (uint32_t)k, C, sh);
+  SelThreshold th;
+  if (reached && k == k_mass) {
+    // the k-th largest key is v itself: keys above v, and the first
+    // k - n_above keys equal to v (1 <= k - n_above <= keys equal to v)
+    th.t = v;
+    th.take_eq = (uint32_t)k - n_above;
+  } else {
+    if (target > 0ull) {
+      cluster_sync();                              // every CTA has read every CTA's level-1 and level-2 bins
+      for (int i = tid; i < hist_words(1) + hist_words(2); i += blockDim.x) h1[i] = 0u;
+      __syncthreads();
+    }
+    th = cluster_threshold_by<FUSED_THREADS / 2>(pass, hist, (uint32_t)k, C, sh);
+  }
   int* out = p.idx + (size_t)unit * p.k_max;
   const uint32_t keys_s = (uint32_t)__cvta_generic_to_shared(keys);
   auto key_addr = [&](int i) -> uint32_t { return keys_s + 4u * (uint32_t)i; };

@@ -306,7 +306,13 @@ int launch_tables(const void* Q, sk_dtype q, const void* R, int B, int Hq, int H
                       : launch_tables_d<64, float>(tp, pairs, G, s);
 }
 
-constexpr int kScoreBlocksPerCta = 256;
+// Chunks of the unfused score kernel: one wave of CTAs (one per SM) over all
+// pairs when the pairs fit, else one CTA per pair.
+dim3 score_grid(int pairs, int nblk, int* blocks_per_cta) {
+  const int chunks = std::max(1, std::min(kNumSMs / std::max(1, pairs), nblk));
+  *blocks_per_cta = (nblk + chunks - 1) / chunks;
+  return dim3(pairs, (nblk + *blocks_per_cta - 1) / *blocks_per_cta);
+}
 
 template <int LP, bool NORM = true>
 int launch_score_t(const ScoreParams& sp, dim3 grid, cudaStream_t s) {
@@ -351,9 +357,8 @@ int launch_hamming_score(const float* T, const void* codes, int pairs, int Ncap,
   sp.scores = scores;
   sp.Ncap = Ncap;
   sp.N = N;
-  sp.blocks_per_cta = kScoreBlocksPerCta;
-  const int nblk = (N + 31) / 32;
-  return launch_score_t<16, false>(sp, dim3(pairs, (nblk + kScoreBlocksPerCta - 1) / kScoreBlocksPerCta), s);
+  const dim3 grid = score_grid(pairs, (N + 31) / 32, &sp.blocks_per_cta);
+  return launch_score_t<16, false>(sp, grid, s);
 }
 
 int launch_score(const float* T, const void* ids, const void* norms, int pairs, int Ncap, int N, int L, float* scores,
@@ -366,9 +371,7 @@ int launch_score(const float* T, const void* ids, const void* norms, int pairs, 
   sp.scores = scores;
   sp.Ncap = Ncap;
   sp.N = N;
-  sp.blocks_per_cta = kScoreBlocksPerCta;
-  const int nblk = (N + 31) / 32;
-  const dim3 grid(pairs, (nblk + kScoreBlocksPerCta - 1) / kScoreBlocksPerCta);
+  const dim3 grid = score_grid(pairs, (N + 31) / 32, &sp.blocks_per_cta);
   switch (ids_bytes_per_key(L)) {
     case 16: return launch_score_t<16>(sp, grid, s);
     case 32: return launch_score_t<32>(sp, grid, s);

@@ -500,7 +500,8 @@ struct ScoreParams {
 };
 
 // grid = (pairs, chunks); the pair's table image is copied to 64 KB-aligned
-// shared memory, then each lane scores one key. NORM = false: hard-hash
+// shared memory, then each lane scores one key of a 32-key block, with the
+// warp's next blocks already requested. NORM = false: hard-hash
 // scores (ids holds the 128-bit codes, the image the 16 byte-tables, no norm).
 template <int LP, bool NORM = true>
 __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_score_kernel(const ScoreParams p) {
@@ -523,14 +524,38 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_score_kernel(const Sc
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const size_t pair_keys = (size_t)(pair / p.pair_div) * p.Ncap;
   const int nblk = (p.N + 31) / 32;
-  const int blk0 = blockIdx.y * p.blocks_per_cta;
+  const int blk0 = min(nblk, (int)blockIdx.y * p.blocks_per_cta);
   const int blk1 = min(nblk, blk0 + p.blocks_per_cta);
-  for (int blk = blk0 + warp; blk < blk1; blk += nw) {
-    const int key = blk * 32 + lane;
-    KeyIds<LP> k;
-    load_key_ids<LP, NORM>(k, p.ids + (pair_keys + key) * LP, p.norms + pair_keys + key);
-    const float s = score_key<LP, NORM>(k, tbl + 4u * lane, tbl + TABLE_BYTES + 4u * lane);
-    if (key < p.N) p.scores[(size_t)pair * p.Ncap + key] = s;
+  // this warp's blocks blk0 + warp + i * nw (i < nb), the next PF of them in
+  // flight while one is scored
+  constexpr int PF = score_pf<LP>();
+  const int nb = max(0, (blk1 - blk0 - warp + nw - 1) / nw);
+  const uint8_t* ids_pair = p.ids + pair_keys * LP;
+  const __half* norms_pair = NORM ? p.norms + pair_keys : nullptr;
+  float* out = p.scores + (size_t)pair * p.Ncap;
+  KeyIds<LP> buf[PF];
+#pragma unroll
+  for (int u = 0; u < PF; ++u) {
+    if (u < nb) {
+      const int key = (blk0 + warp + u * nw) * 32 + lane;
+      load_key_ids<LP, NORM>(buf[u], ids_pair + (size_t)key * LP, norms_pair + key);
+    }
+  }
+  for (int it = 0; it < nb; it += PF) {
+#pragma unroll
+    for (int u = 0; u < PF; ++u) {
+      const int i = it + u;
+      if (i < nb) {
+        const KeyIds<LP> cur = buf[u];
+        if (i + PF < nb) {
+          const int key = (blk0 + warp + (i + PF) * nw) * 32 + lane;
+          load_key_ids<LP, NORM>(buf[u], ids_pair + (size_t)key * LP, norms_pair + key);
+        }
+        const float sc = score_key<LP, NORM>(cur, tbl + 4u * lane, tbl + TABLE_BYTES + 4u * lane);
+        const int key = (blk0 + warp + i * nw) * 32 + lane;
+        if (key < p.N) out[key] = sc;
+      }
+    }
   }
 }
 

@@ -243,13 +243,51 @@ int launch_cluster(Kern kern, int grid, int C, size_t smem, cudaStream_t s, cons
 }
 
 template <int D, typename QT, bool HATA>
-int launch_select_t(const FusedParams& p, int pairs, bool pdl, cudaStream_t s) {
-  const int grid = pairs * p.C;
+int launch_select_t(const FusedParams& p0, int pairs, bool pdl, cudaStream_t s) {
+  const int grid = pairs * p0.C;
+  FusedParams p = p0;
+  auto go = [&](auto kern) {
+    if (grid > kNumSMs) {
+      // CTAs per wave: clusters that fit at once (occupancy API, cached per
+      // kernel and cluster size) times the cluster size
+      static std::mutex mu;
+      static std::vector<std::pair<std::pair<const void*, int>, int>> cache;
+      const void* fn = reinterpret_cast<const void*>(kern);
+      int n = -1;
+      {
+        std::lock_guard<std::mutex> lock(mu);
+        for (const auto& e : cache)
+          if (e.first.first == fn && e.first.second == p.C) n = e.second;
+      }
+      if (n < 0) {
+        n = 0;
+        if (set_kernel_smem(kern, SMEM_DYN_MAX, p.C > 8) == cudaSuccess) {
+          cudaLaunchConfig_t cfg = {};
+          cfg.gridDim = dim3(grid, 1, 1);
+          cfg.blockDim = dim3(FUSED_THREADS, 1, 1);
+          cfg.dynamicSmemBytes = SMEM_DYN_MAX;
+          cudaLaunchAttribute attr[1];
+          attr[0].id = cudaLaunchAttributeClusterDimension;
+          attr[0].val.clusterDim.x = (unsigned)p.C;
+          attr[0].val.clusterDim.y = 1;
+          attr[0].val.clusterDim.z = 1;
+          cfg.attrs = attr;
+          cfg.numAttrs = 1;
+          if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) n = 0;
+        }
+        cudaGetLastError();
+        std::lock_guard<std::mutex> lock(mu);
+        cache.push_back({{fn, p.C}, n});
+      }
+      p.next_stride = n * p.C < grid ? n * p.C : 0;
+    }
+    return launch_cluster(kern, grid, p.C, SMEM_DYN_MAX, s, p, pdl);
+  };
   switch (ids_bytes_per_key(p.L)) {
-    case 16: return launch_cluster(socket_select_kernel<D, 16, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p, pdl);
-    case 32: return launch_cluster(socket_select_kernel<D, 32, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p, pdl);
-    case 48: return launch_cluster(socket_select_kernel<D, 48, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p, pdl);
-    default: return launch_cluster(socket_select_kernel<D, 64, QT, HATA>, grid, p.C, SMEM_DYN_MAX, s, p, pdl);
+    case 16: return go(socket_select_kernel<D, 16, QT, HATA>);
+    case 32: return go(socket_select_kernel<D, 32, QT, HATA>);
+    case 48: return go(socket_select_kernel<D, 48, QT, HATA>);
+    default: return go(socket_select_kernel<D, 64, QT, HATA>);
   }
 }
 

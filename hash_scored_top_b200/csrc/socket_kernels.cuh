@@ -28,6 +28,7 @@ constexpr int FUSED_WARPS = FUSED_THREADS / 32;
 template <int LP>
 __host__ __device__ constexpr int score_pf() { return 2; }
 constexpr uint32_t SCORE_L2_PREFETCH = 96u * 1024u;   // bytes of each CTA's key slice prefetched into L2
+constexpr uint32_t NEXT_L2_PREFETCH = 512u * 1024u;   // bytes of ID rows prefetched for the next wave's CTA
 constexpr int ATTEND_THREADS = 256;              // the attention kernel
 constexpr int ATTEND_WARPS = ATTEND_THREADS / 32;
 constexpr int ATTEND_BUFS = 2;                    // bf16: K/V slots per computing warp
@@ -66,6 +67,10 @@ struct FusedParams {
   // table kernel beforehand (bucket_table_kernel / hamming_table_kernel);
   // every CTA copies its unit's image instead of building tables
   const float* tables = nullptr;
+  // CTAs of one wave when the grid runs in several (0: one wave): once it has
+  // scored its slice, CTA b asks for CTA b + next_stride's slice in L2, so the
+  // next wave's reads overlap this wave's selection
+  int next_stride = 0;
 };
 
 constexpr int PHASES = 24;
@@ -387,6 +392,24 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_select_kernel(const F
   score_blocks<LP, !HATA>(buf, ids_pair, norms_pair, p.N, blk0, nb, fs.tbl0 + 4u * lane, fs.tbl1 + 4u * lane, keys,
                           hist[0], sh);
   stamp(p.phase_ts, 11);
+  if (p.next_stride > 0 && warp == 1) {
+    // the slice of the CTA one wave later (same rank arithmetic as above)
+    const int nx = (int)blockIdx.x + p.next_stride;
+    if (nx < (int)gridDim.x) {
+      const int nb0 = min(nblk_pair, (nx % C) * p.blocks_per_cta);
+      const int nb1 = min(nblk_pair, nb0 + p.blocks_per_cta);
+      if (nb1 > nb0) {
+        constexpr uint32_t kChunk = 32768u;
+        const size_t npk = (size_t)((nx / C) / p.pair_div) * p.Ncap + (size_t)nb0 * 32;
+        const uint32_t keys_n = min((uint32_t)(nb1 - nb0) * 32u, NEXT_L2_PREFETCH / LP) & ~31u;   // 16-byte sizes
+        const char* src = reinterpret_cast<const char*>(p.ids + npk * LP);
+        const uint32_t bytes = keys_n * LP;
+        for (uint32_t off = (uint32_t)lane * kChunk; off < bytes; off += 32u * kChunk)
+          prefetch_l2_bulk(src + off, min(kChunk, bytes - off));
+        if (!HATA && lane == 31) prefetch_l2_bulk(p.norms + npk, keys_n * 2u);
+      }
+    }
+  }
   // keys past the slice, up to its last 128-key chunk, read as 0
   if (warp == 0) {
     const int tail_end = (n_local + 127) & ~127;

@@ -233,3 +233,26 @@ def test_decode_heads_over_several_waves(api):
                 err = pa.row_rel_err(O[b, h * w.G + g:h * w.G + g + 1].cpu().numpy(), o_ref[g:g + 1])
                 assert err < pa.out_tol(w), (err, b, h, g)
     assert compared >= 12
+
+
+@pytest.mark.parametrize("name,per_head,mass,k_min,k_max", [
+    ("llama8b_100k", False, 0.3, 1, None),       # 4-CTA clusters, k from the mass search
+    ("llama8b_100k", True, 0.6, 1, None),
+    ("llama8b_100k", False, 1e-6, 17, 900),      # clamped: the count search across 4 CTAs
+    ("llama8b_100k", True, 1.0, 5, 333),
+    ("ties_60k", False, 0.4, 1, None),           # many exactly equal scores across 2 CTAs
+    ("ties_60k", True, 0.05, 1, None),
+])
+def test_decode_adaptive_multi_cta(api, name, per_head, mass, k_min, k_max):
+    """Units of more keys than one CTA holds (the adaptive top-k then runs in
+    clusters of 2 or 4 CTAs: cluster-wide mass sums and resolves, tie quotas and
+    output offsets across CTAs); N is not a multiple of 4, so the last CTA's
+    slice is ragged. In the tie-heavy shape (2 tables of 2 hyperplanes: 16
+    bucket combinations times the f16 norms) about 89% of the keys share
+    their score with another key (19.5K distinct scores over 60K keys)."""
+    w = {"llama8b_100k": wl.shrink(wl.LLAMA_8B, B=1, Hkv=2, Hq=8, N=100003, k=100003 // 33),
+         "ties_60k": wl.shrink(wl.LLAMA_8B, B=1, Hkv=2, Hq=4, N=60001, k=60001 // 33, needles=0, L=2, P=2,
+                               tau=0.7)}[name]
+    inp = wl.make_inputs(w, DEV)
+    ids, nrm, ids_nat, norms = _cache(w, inp)
+    _adaptive_and_compare(api, w, inp, ids, nrm, ids_nat, norms, mass, k_min, k_max if k_max else w.N, per_head)

@@ -39,122 +39,131 @@ struct AdaptParams {
 
 struct AdaptShared {
   double part[SEL_MAX_C];            // every CTA's float64 score sum
-  unsigned long long scan_tmp[32];   // block-scan scratch
+  unsigned long long scan_tmp[32];   // per-warp float64 score sums
   unsigned long long mass_above;     // broadcast of the level's result
   uint32_t bin, cnt_above, found, pad;
 };
 
 constexpr int kAdaptHistWords = hist_words(0) + hist_words(1) + hist_words(2);
-// counts (one word per bin) and masses (two words per bin) of the three levels
+// per level, three words (mass low and high, count) per group of 32 bins
+constexpr int kAdaptGroupWords = 3 * (kAdaptHistWords / 32);
+// counts (one word per bin), masses (two words per bin) and group sums of the three levels
 constexpr uint32_t kAdaptFixedBytes = (uint32_t)(((sizeof(SelShared) + 15) & ~15) + 4 * kAdaptHistWords +
-                                                 8 * kAdaptHistWords + ((sizeof(AdaptShared) + 15) & ~15));
+                                                 8 * kAdaptHistWords + 4 * kAdaptGroupWords +
+                                                 ((sizeof(AdaptShared) + 15) & ~15));
+static_assert((4 * kAdaptGroupWords) % 16 == 0, "the keys after the group sums stay 16-byte aligned");
 
-// Block-wide exclusive scan of one unsigned 64-bit value per thread.
-__device__ __forceinline__ unsigned long long block_exclusive_scan_u64(unsigned long long v, AdaptShared* as) {
+// This CTA's mass and count of every group of 32 bins of one level (all
+// warps; the level's atomics are complete): glo, ghi, gc [ngroups].
+__device__ __forceinline__ void group_sums(const uint32_t* mlo, const uint32_t* mhi, const uint32_t* hc, int ngroups,
+                                           uint32_t* glo, uint32_t* ghi, uint32_t* gc) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  unsigned long long x = v;
+  for (int g = warp; g < ngroups; g += nw) {
+    const int b = g * 32 + lane;
+    unsigned long long m = ((unsigned long long)mhi[b] << 32) | mlo[b];
 #pragma unroll
-  for (int o = 1; o < 32; o <<= 1) {
-    const unsigned long long y = __shfl_up_sync(FULL, x, o);
-    if (lane >= o) x += y;
-  }
-  if (lane == 31) as->scan_tmp[warp] = x;
-  __syncthreads();
-  if (warp == 0) {
-    unsigned long long t = lane < nw ? as->scan_tmp[lane] : 0ull;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const unsigned long long y = __shfl_up_sync(FULL, t, o);
-      if (lane >= o) t += y;
+    for (int o = 16; o > 0; o >>= 1) m += __shfl_xor_sync(FULL, m, o);
+    const uint32_t c = __reduce_add_sync(FULL, hc[b]);
+    if (lane == 0) {
+      glo[g] = (uint32_t)m;
+      ghi[g] = (uint32_t)(m >> 32);
+      gc[g] = c;
     }
-    if (lane < nw) as->scan_tmp[lane] = t;
   }
-  __syncthreads();
-  const unsigned long long before = warp > 0 ? as->scan_tmp[warp - 1] : 0ull;
-  __syncthreads();
-  return before + x - v;
 }
 
-// One level of the mass search over nbins bins (descending bin order across
-// the threads, BPT bins each): the cluster-wide mass and count of every bin,
-// then the bin where the running mass from the top first reaches `need`.
-// mlo, mhi: the level's low and high mass words; hc: its key counts.
-template <int BPT>
-__device__ void resolve_mass_level(const uint32_t* mlo, const uint32_t* mhi, const uint32_t* hc, int nbins,
-                                   unsigned long long need, int C, SelShared* sh, AdaptShared* as) {
+// Exclusive scan over the lanes of a warp (lane 0 first) of a mass and a count.
+__device__ __forceinline__ void warp_exclusive_scan2(unsigned long long m, uint32_t c, unsigned long long& m_before,
+                                                     uint32_t& c_before) {
+  const int lane = threadIdx.x & 31;
+  unsigned long long im = m;
+  uint32_t ic = c;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned long long ym = __shfl_up_sync(FULL, im, o);
+    const uint32_t yc = __shfl_up_sync(FULL, ic, o);
+    if (lane >= o) {
+      im += ym;
+      ic += yc;
+    }
+  }
+  m_before = im - m;
+  c_before = ic - c;
+}
+
+// One level of the mass search (warp 0 only): the cluster-wide mass and count
+// of every group of 32 bins (descending), the group where the running mass
+// from the top first reaches `need`, then that group's 32 bins. Reads of
+// other CTAs' shared memory: three words per group and per bin of that group,
+// from every CTA. Writes found, bin, mass_above (mass in bins above it) and
+// cnt_above to `as`. ngroups <= 64.
+__device__ void resolve_mass_grouped(const uint32_t* mlo, const uint32_t* mhi, const uint32_t* hc,
+                                     const uint32_t* glo, const uint32_t* ghi, const uint32_t* gc, int ngroups,
+                                     unsigned long long need, int C, AdaptShared* as) {
   cg::cluster_group cluster = cg::this_cluster();
-  const int tid = threadIdx.x;
-  const int base = nbins - (tid + 1) * BPT;
-  const bool mine = base >= 0;
-  if (tid == 0) {
-    as->found = 0u;
-    as->bin = 0u;
-    as->cnt_above = 0u;
-    as->mass_above = 0ull;
-  }
-  unsigned long long m[BPT];
-  uint32_t c[BPT];
-#pragma unroll
-  for (int j = 0; j < BPT; ++j) {
-    m[j] = 0ull;
-    c[j] = 0u;
-  }
-  if (mine) {
-    for (int r = 0; r < C; ++r) {
-      const uint32_t* pl = cluster.map_shared_rank(mlo, r) + base;
-      const uint32_t* ph = cluster.map_shared_rank(mhi, r) + base;
-      const uint32_t* pc = cluster.map_shared_rank(hc, r) + base;
-      if constexpr (BPT % 4 == 0) {
-        // 16-byte reads: a read of another CTA's shared memory costs about
-        // the same whatever its width
-#pragma unroll
-        for (int j = 0; j < BPT; j += 4) {
-          const uint4 l = *reinterpret_cast<const uint4*>(pl + j);
-          const uint4 h = *reinterpret_cast<const uint4*>(ph + j);
-          const uint4 n = *reinterpret_cast<const uint4*>(pc + j);
-          m[j] += ((unsigned long long)h.x << 32) | l.x;
-          m[j + 1] += ((unsigned long long)h.y << 32) | l.y;
-          m[j + 2] += ((unsigned long long)h.z << 32) | l.z;
-          m[j + 3] += ((unsigned long long)h.w << 32) | l.w;
-          c[j] += n.x;
-          c[j + 1] += n.y;
-          c[j + 2] += n.z;
-          c[j + 3] += n.w;
-        }
-      } else {
-#pragma unroll
-        for (int j = 0; j < BPT; ++j) {
-          m[j] += ((unsigned long long)ph[j] << 32) | pl[j];
-          c[j] += pc[j];
-        }
-      }
+  const int lane = threadIdx.x & 31;
+  // lane l: groups ngroups - 1 - 2l and ngroups - 2 - 2l
+  const int ga = ngroups - 1 - 2 * lane, gb = ga - 1;
+  unsigned long long ma = 0ull, mb = 0ull;
+  uint32_t ca = 0u, cb = 0u;
+  for (int r = 0; r < C; ++r) {
+    const uint32_t* pl = cluster.map_shared_rank(glo, r);
+    const uint32_t* ph = cluster.map_shared_rank(ghi, r);
+    const uint32_t* pc = cluster.map_shared_rank(gc, r);
+    if (ga >= 0) {
+      ma += ((unsigned long long)ph[ga] << 32) | pl[ga];
+      ca += pc[ga];
+    }
+    if (gb >= 0) {
+      mb += ((unsigned long long)ph[gb] << 32) | pl[gb];
+      cb += pc[gb];
     }
   }
-  unsigned long long lm = 0ull;
-  uint32_t lc = 0u;
-#pragma unroll
-  for (int j = 0; j < BPT; ++j) {
-    lm += m[j];
-    lc += c[j];
+  unsigned long long m_before;
+  uint32_t c_before;
+  warp_exclusive_scan2(ma + mb, ca + cb, m_before, c_before);
+  int grp = -1;
+  unsigned long long g_mass = 0ull;
+  uint32_t g_cnt = 0u;
+  if (m_before < need && need <= m_before + ma) {
+    grp = ga;
+    g_mass = m_before;
+    g_cnt = c_before;
+  } else if (m_before + ma < need && need <= m_before + ma + mb) {
+    grp = gb;
+    g_mass = m_before + ma;
+    g_cnt = c_before + ca;
   }
-  const unsigned long long mb = block_exclusive_scan_u64(lm, as);
-  const uint32_t cb = block_exclusive_scan(lc, sh);
-  if (mine && mb < need && need <= mb + lm) {
-    unsigned long long run = mb;
-    uint32_t crun = cb;
-#pragma unroll
-    for (int j = BPT - 1; j >= 0; --j) {
-      if (run < need && need <= run + m[j]) {
-        as->bin = (uint32_t)(base + j);
-        as->mass_above = run;
-        as->cnt_above = crun;
-        as->found = 1u;
-      }
-      run += m[j];
-      crun += c[j];
-    }
+  const unsigned hit = __ballot_sync(FULL, grp >= 0);
+  if (hit == 0u) {                      // the whole unit's mass stays below the target
+    if (lane == 0) as->found = 0u;
+    return;
   }
-  __syncthreads();
+  const int src = __ffs(hit) - 1;
+  grp = __shfl_sync(FULL, grp, src);
+  g_mass = __shfl_sync(FULL, g_mass, src);
+  g_cnt = __shfl_sync(FULL, g_cnt, src);
+  // the group's bins, lane l: bin 32 grp + 31 - l
+  const int bin = grp * 32 + 31 - lane;
+  unsigned long long m = 0ull;
+  uint32_t c = 0u;
+  for (int r = 0; r < C; ++r) {
+    m += ((unsigned long long)cluster.map_shared_rank(mhi, r)[bin] << 32) | cluster.map_shared_rank(mlo, r)[bin];
+    c += cluster.map_shared_rank(hc, r)[bin];
+  }
+  warp_exclusive_scan2(m, c, m_before, c_before);
+  const unsigned long long before = g_mass + m_before;
+  const unsigned hit2 = __ballot_sync(FULL, before < need && need <= before + m);
+  if (hit2 == 0u) {                     // cannot happen: the group's mass covers the rest of need
+    if (lane == 0) as->found = 0u;
+    return;
+  }
+  if (lane == __ffs(hit2) - 1) {
+    as->found = 1u;
+    as->bin = (uint32_t)bin;
+    as->mass_above = before;
+    as->cnt_above = g_cnt + c_before;
+  }
 }
 
 // floor(x * 2^sc) for the bit pattern `key` of a finite float x >= 0, from
@@ -202,7 +211,9 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
   uint32_t* h2 = h1 + hist_words(1);
   // masses, level by level: low words of the level's bins, then high words
   uint32_t* mass_words = h0 + kAdaptHistWords;
-  a += 12 * kAdaptHistWords;
+  // group sums, level by level: low words, high words, counts
+  uint32_t* group_words = mass_words + 2 * kAdaptHistWords;
+  a += 12 * kAdaptHistWords + 4 * kAdaptGroupWords;
   AdaptShared* as = reinterpret_cast<AdaptShared*>(a);
   a += (sizeof(AdaptShared) + 15) & ~15;
   uint32_t* keys = reinterpret_cast<uint32_t*>(a);
@@ -278,6 +289,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
     int pshift = 32;
     reached = true;
     uint32_t* mlo = mass_words;
+    uint32_t* gw = group_words;
 #pragma unroll 1
     for (int lvl = 0; lvl < SEL_LEVELS; ++lvl) {
       const int bits = sel_bits(lvl), shift = sel_shift(lvl);
@@ -296,8 +308,12 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
         }
       });
       __syncthreads();
+      const int ng = (1 << bits) / 32;
+      group_sums(mlo, mhi, hc, ng, gw, gw + ng, gw + 2 * ng);
+      __syncthreads();
       cluster_sync();
-      resolve_mass_level<4>(mlo, mhi, hc, 1 << bits, need, C, sh, as);
+      if (warp == 0) resolve_mass_grouped(mlo, mhi, hc, gw, gw + ng, gw + 2 * ng, ng, need, C, as);
+      __syncthreads();
       const bool found = as->found != 0u;
       const uint32_t bn = as->bin, ca = as->cnt_above;
       const unsigned long long ma = as->mass_above;
@@ -311,6 +327,7 @@ __global__ void __launch_bounds__(FUSED_THREADS, 1) socket_adaptive_topk_kernel(
       prefix = (prefix << bits) | bn;
       pshift = shift;
       mlo = mhi + (1 << bits);
+      gw += 3 * ng;
     }
     if (reached) {
       const unsigned long long ft = fixed_mass(prefix, sc);   // every key of the final bin equals prefix

@@ -34,6 +34,8 @@ SIGNATURES = {
                            _p]),
     "socket_decode_append": (_i, [_p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _f, _p, _p, _p,
                                   _z, _p]),
+    "socket_decode_step_host": (_i, [_p, _p, _p, _p, _p, _p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i,
+                                     _f, _p, _p, _p, _z, _p]),
     "socket_select": (_i, [_p, _i, _p, _p, _p, _i, _i, _i, _i, _i, _i, _i, _i, _f, _i, _p, _p, _z, _p]),
     "hata_hash_keys": (_i, [_p, _i, _p, _i, _i, _i, _i, _i, _i, _p, _p]),
     "hata_decode": (_i, [_p, _p, _p, _i, _p, _p, _i, _i, _i, _i, _i, _i, _i, _f, _p, _p, _p, _z, _p]),

@@ -362,6 +362,40 @@ def socket_decode_append(Q, K, V, R, ids, norms, N: int, L: int, P: int, tau: fl
     _check(rc, "socket_decode_append")
 
 
+def _host_ptr(t, name):
+    if t.is_cuda or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous host tensor (pinned for asynchronous copies)")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def socket_decode_step_host(Q_host, K_new_host, V_new_host, Q, K, V, R, ids, norms, N: int, L: int, P: int,
+                            tau: float, k: int, scale: float, O, O_host, ws=None):
+    """One decode step from host buffers: Q_host [B, Hq, d] and the new token's rows K_new_host, V_new_host
+    [B, Hkv, d] (pinned, K's dtype) are copied in (the rows to position N - 1 of K and V), the step runs as
+    socket_decode_append, and O [B, Hq, d] float32 is copied to O_host (pinned). All on the current stream:
+    O_host holds the result once the stream has synchronised."""
+    B, Hq, d = Q.shape
+    _, Hkv, Ncap, _ = K.shape
+    _want(Q, K.dtype, (B, Hq, d), "Q")
+    _want(V, K.dtype, K.shape, "V")
+    _want(R, torch.bfloat16, (L * P, d), "R")
+    _want(ids, torch.uint8, (B, Hkv, Ncap, ids_bytes_per_key(L)), "ids")
+    _want(norms, torch.float16, (B, Hkv, Ncap), "norms")
+    _want(O, torch.float32, (B, Hq, d), "O")
+    _want(Q_host, K.dtype, (B, Hq, d), "Q_host")
+    _want(K_new_host, K.dtype, (B, Hkv, d), "K_new_host")
+    _want(V_new_host, K.dtype, (B, Hkv, d), "V_new_host")
+    _want(O_host, torch.float32, (B, Hq, d), "O_host")
+    if ws is None:                # a caller's workspace is passed as it is: the library checks its size
+        ws = _workspace(workspace_bytes(OP_DECODE, B, Hq, Hkv, Ncap, N, d, L, P, k), Q.device, ws)
+    rc = _lib.lib.socket_decode_step_host(_host_ptr(Q_host, "Q_host"), _host_ptr(K_new_host, "K_new_host"),
+                                          _host_ptr(V_new_host, "V_new_host"), _ptr(Q), _ptr(K), _ptr(V),
+                                          _dtype_code(K), _ptr(R), _ptr(ids), _ptr(norms), B, Hq, Hkv, Ncap, N, d, L,
+                                          P, ctypes.c_float(tau), k, ctypes.c_float(scale), _ptr(O),
+                                          _host_ptr(O_host, "O_host"), _ptr(ws), _ws_bytes(ws), _stream())
+    _check(rc, "socket_decode_step_host")
+
+
 def socket_select(Q, R, ids, norms, N: int, L: int, P: int, tau: float, k: int, idx, ws=None):
     """SOCKET steps 2-4 without the attention: idx [B, Hkv, k] int32 ascending."""
     B, Hq, d = Q.shape

@@ -18,6 +18,7 @@
 #include "estimator.cuh"
 #include "adaptive.cuh"
 #include "hash_tc.cuh"
+#include "step_io.cuh"
 
 using namespace hst;
 
@@ -764,7 +765,7 @@ int encode_rows_map(CUtensorMap* map, const void* base, long rows, int d, int bo
 constexpr int kAppendMaxKeys = 16;
 
 int hash_launch(const void* K, const void* V, sk_dtype kv, const void* R, int B, int Hkv, int Ncap, int n_begin,
-                int n_count, int d, int L, int P, void* ids, void* norms, cudaStream_t s) {
+                int n_count, int d, int L, int P, void* ids, void* norms, cudaStream_t s, bool pdl = false) {
   HashParams hp;
   hp.K = K;
   hp.V = V;
@@ -814,8 +815,19 @@ int hash_launch(const void* K, const void* V, sk_dtype kv, const void* R, int B,
   if (n_count <= kAppendMaxKeys) {      // decode-time append: a few keys per pair
     const dim3 grid(hp.pairs, n_count);
     const int threads = (LP + 31) / 32 * 32;
-    if (kv == SK_BF16) hash_keys_append_kernel<__nv_bfloat16><<<grid, threads, 0, s>>>(hp);
-    else hash_keys_append_kernel<float><<<grid, threads, 0, s>>>(hp);
+    // pdl: the programmatic dependent of the kernel that wrote the step's inputs
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(threads);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const cudaError_t e = kv == SK_BF16 ? cudaLaunchKernelEx(&cfg, hash_keys_append_kernel<__nv_bfloat16>, hp)
+                                        : cudaLaunchKernelEx(&cfg, hash_keys_append_kernel<float>, hp);
+    if (e != cudaSuccess) return fail(SK_ERR_CUDA, "append launch: %s", cudaGetErrorString(e));
     return check_launch("hash_keys_append_kernel");
   }
   const size_t smem = (((size_t)d * LP * 2 + 15) & ~(size_t)15) + (size_t)32 * d * 4 + (size_t)LP * 4;
@@ -1213,9 +1225,27 @@ int socket_decode(const void* Q, const void* K, const void* V, sk_dtype kv, cons
                      false, true, as_stream(stream));
 }
 
-int socket_decode_append(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, void* ids,
-                         void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k,
-                         float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, void* stream) {
+}  // extern "C" (reopened below)
+
+namespace {
+// The device's address of page-locked host memory that it can read and write
+// directly (16-byte aligned), or null (pageable memory, or anything else):
+// the step then uses DMA copies, which accept any host memory.
+void* mapped_host(const void* ptr) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, ptr) != cudaSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  if (a.type != cudaMemoryTypeHost || a.devicePointer == nullptr) return nullptr;
+  if ((reinterpret_cast<uintptr_t>(a.devicePointer) & 15) != 0) return nullptr;
+  return a.devicePointer;
+}
+
+// The argument checks of socket_decode_append (no launch).
+int socket_decode_append_check(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R,
+                               const void* ids, const void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d,
+                               int L, int P, float tau, int k, const float* O, const void* ws, size_t ws_bytes) {
   SK_NONNULL(Q);
   SK_NONNULL(K);
   SK_NONNULL(V);
@@ -1244,10 +1274,128 @@ int socket_decode_append(const void* Q, const void* K, const void* V, sk_dtype k
     if (ws == nullptr || ws_bytes < need)
       return fail(SK_ERR_WORKSPACE, "workspace: need %zu bytes, got %zu", need, ws == nullptr ? (size_t)0 : ws_bytes);
   }
-  const cudaStream_t s = as_stream(stream);
-  SK_TRY(hash_launch(K, V, kv, R, B, Hkv, Ncap, N - 1, 1, d, L, P, ids, norms, s));
+  return SK_OK;
+}
+}  // namespace
+
+extern "C" {
+
+}  // extern "C" (reopened below)
+
+namespace {
+// The step of socket_decode_append after its checks; pdl: the hashing kernel
+// is the programmatic dependent of a kernel that wrote the step's inputs.
+int append_and_decode(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, void* ids, void* norms,
+                      int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k, float scale,
+                      float* O, int* idx_out, void* ws, size_t ws_bytes, cudaStream_t s, bool pdl) {
+  SK_TRY(hash_launch(K, V, kv, R, B, Hkv, Ncap, N - 1, 1, d, L, P, ids, norms, s, pdl));
   return decode_impl(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, scale, O, idx_out, ws, ws_bytes,
                      false, true, s, true);
+}
+}  // namespace
+
+extern "C" {
+
+int socket_decode_append(const void* Q, const void* K, const void* V, sk_dtype kv, const void* R, void* ids,
+                         void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P, float tau, int k,
+                         float scale, float* O, int* idx_out, void* ws, size_t ws_bytes, void* stream) {
+  SK_TRY(socket_decode_append_check(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, O, ws,
+                                    ws_bytes));
+  const cudaStream_t s = as_stream(stream);
+  return append_and_decode(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, scale, O, idx_out, ws,
+                           ws_bytes, s, false);
+}
+
+int socket_decode_step_host(const void* Q_host, const void* K_new_host, const void* V_new_host, void* Q, void* K,
+                            void* V, sk_dtype kv, const void* R, void* ids, void* norms, int B, int Hq, int Hkv,
+                            int Ncap, int N, int d, int L, int P, float tau, int k, float scale, float* O,
+                            float* O_host, void* ws, size_t ws_bytes, void* stream) {
+  SK_NONNULL(Q_host);
+  SK_NONNULL(K_new_host);
+  SK_NONNULL(V_new_host);
+  SK_NONNULL(O_host);
+  SK_NONNULL(Q);
+  SK_NONNULL(K);
+  SK_NONNULL(V);
+  SK_NONNULL(O);
+  SK_TRY(check_dtype(kv));
+  SK_TRY(check_heads(B, Hq, Hkv, d));
+  SK_TRY(check_cache(Ncap, N));
+  // everything the step checks, before the first copy: a failure moves and launches nothing
+  SK_TRY(socket_decode_append_check(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, O, ws, ws_bytes));
+  const cudaStream_t s = as_stream(stream);
+  const size_t es = kv == SK_BF16 ? 2 : 4;
+  const size_t row = (size_t)d * es;                 // a multiple of 16 bytes (d % 32 == 0)
+  char* krow = reinterpret_cast<char*>(K) + (size_t)(N - 1) * row;
+  char* vrow = reinterpret_cast<char*>(V) + (size_t)(N - 1) * row;
+  const void* qd = mapped_host(Q_host);
+  const void* kd = mapped_host(K_new_host);
+  const void* vd = mapped_host(V_new_host);
+  void* od = mapped_host(O_host);
+  cudaError_t e = cudaSuccess;
+  if (qd && kd && vd) {
+    // one kernel reads the three inputs from host memory: the query, and the
+    // new token's rows into row N - 1 of every pair (Ncap rows apart)
+    StepCopyParams cp = {};
+    cp.jobs = 3;
+    cp.src[0] = static_cast<const char*>(qd);
+    cp.dst[0] = static_cast<char*>(Q);
+    cp.rows[0] = B * Hq;
+    cp.src[1] = static_cast<const char*>(kd);
+    cp.dst[1] = krow;
+    cp.rows[1] = B * Hkv;
+    cp.src[2] = static_cast<const char*>(vd);
+    cp.dst[2] = vrow;
+    cp.rows[2] = B * Hkv;
+    for (int j = 0; j < 3; ++j) {
+      cp.row16[j] = (int)(row / 16);
+      cp.src_pitch[j] = row;
+      cp.dst_pitch[j] = j == 0 ? row : (size_t)Ncap * row;
+    }
+    const long long words = (long long)(B * Hq) * (long long)(row / 16);
+    const int blocks = (int)std::min<long long>(kNumSMs, (words + STEP_COPY_THREADS - 1) / STEP_COPY_THREADS);
+    step_copy_kernel<<<blocks, STEP_COPY_THREADS, 0, s>>>(cp);
+    SK_TRY(check_launch("step_copy_kernel"));
+  } else {
+    e = cudaMemcpyAsync(Q, Q_host, (size_t)B * Hq * row, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(krow, (size_t)Ncap * row, K_new_host, row, row, (size_t)B * Hkv, cudaMemcpyHostToDevice, s);
+    if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(vrow, (size_t)Ncap * row, V_new_host, row, row, (size_t)B * Hkv, cudaMemcpyHostToDevice, s);
+    if (e != cudaSuccess) return fail(SK_ERR_CUDA, "step input copy: %s", cudaGetErrorString(e));
+  }
+  // with the copy kernel, the hashing kernel is its programmatic dependent
+  SK_TRY(append_and_decode(Q, K, V, kv, R, ids, norms, B, Hq, Hkv, Ncap, N, d, L, P, tau, k, scale, O, nullptr, ws,
+                           ws_bytes, s, qd && kd && vd));
+  const size_t obytes = (size_t)B * Hq * d * sizeof(float);
+  if (od) {
+    StepCopyParams cp = {};
+    cp.jobs = 1;
+    cp.src[0] = reinterpret_cast<const char*>(O);
+    cp.dst[0] = static_cast<char*>(od);
+    cp.rows[0] = 1;
+    cp.row16[0] = (int)(obytes / 16);
+    cp.src_pitch[0] = obytes;
+    cp.dst_pitch[0] = obytes;
+    // the programmatic dependent of the attention kernel: launched ahead, it
+    // reads O once that kernel has completed
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)std::min<size_t>(kNumSMs, (obytes / 16 + STEP_COPY_THREADS - 1) / STEP_COPY_THREADS));
+    cfg.blockDim = dim3(STEP_COPY_THREADS);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, step_copy_kernel, cp);
+    if (e != cudaSuccess) return fail(SK_ERR_CUDA, "step output copy launch: %s", cudaGetErrorString(e));
+    SK_TRY(check_launch("step_copy_kernel"));
+  } else {
+    e = cudaMemcpyAsync(O_host, O, obytes, cudaMemcpyDeviceToHost, s);
+    if (e != cudaSuccess) return fail(SK_ERR_CUDA, "step output copy: %s", cudaGetErrorString(e));
+  }
+  return SK_OK;
 }
 
 int socket_select(const void* Q, sk_dtype q, const void* R, const void* ids, const void* norms, int B, int Hq, int Hkv,

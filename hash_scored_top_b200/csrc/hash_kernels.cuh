@@ -114,6 +114,10 @@ template <typename KVT>
 __global__ void __launch_bounds__(512) hash_keys_append_kernel(const HashParams p) {
   __shared__ float ks[128];
   __shared__ uint32_t bits[16];       // 512 projection signs
+  // launched as the programmatic dependent of the kernel that copies this
+  // step's query and key/value rows in, wait for it first (a no-op for an
+  // ordinary launch): the selection started below reads the query at once
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // a selection kernel launched after this one as its programmatic dependent
   // may start now: it waits (griddepcontrol.wait) before reading any bucket
   // ID or norm, and reads nothing else this kernel writes

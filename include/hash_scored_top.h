@@ -210,6 +210,27 @@ int socket_decode_append(const void* Q, const void* K, const void* V, sk_dtype k
                          size_t ws_bytes, void* stream);
 
 /*
+ * One decode step from host buffers (the serving loop's step: the token's
+ * query and key/value rows arrive from the host, its output goes back).
+ * On `stream`, in order: copies Q_host [B][Hq][d] into Q (device), the new
+ * token's rows K_new_host and V_new_host [B][Hkv][d] into row N - 1 of
+ * every pair of K and V (one strided copy each), runs socket_decode_append
+ * over the N keys (SOCKET page, 中核メカニズム：ソフト LSH, steps 1-4: the
+ * appended key's hashing, then the selection and the sparse attention), and
+ * copies O [B][Hq][d] float32 into O_host. Host buffers in kv's dtype (Q in
+ * it too); they should be page-locked (cudaHostAlloc / pinned), so that the
+ * copies are asynchronous: O_host holds the result once the stream has
+ * synchronised. Every argument is checked before the first copy, so an
+ * error moves and launches nothing. Requires what socket_decode_append
+ * requires. ws: sk_workspace_bytes(SK_OP_DECODE, ...) bytes.
+ */
+int socket_decode_step_host(const void* Q_host, const void* K_new_host, const void* V_new_host,
+                            void* Q, void* K, void* V, sk_dtype kv, const void* R, void* ids,
+                            void* norms, int B, int Hq, int Hkv, int Ncap, int N, int d, int L, int P,
+                            float tau, int k, float scale, float* O, float* O_host, void* ws,
+                            size_t ws_bytes, void* stream);
+
+/*
  * Selection only, SOCKET steps 2-4 without the attention: the index list of
  * socket_decode (bucket tables, scores, exact top-k with ties to the lower
  * index), written ascending to idx [B][Hkv][k], for callers that run their

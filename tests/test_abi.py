@@ -30,7 +30,7 @@ def lib():
 def test_header_lists_the_path_entry_points():
     names = _declared_functions()
     for want in ("socket_hash_keys", "socket_score", "socket_topk", "socket_sparse_attend", "socket_decode",
-                 "socket_decode_append", "socket_select",
+                 "socket_decode_append", "socket_decode_step_host", "socket_select",
                  "hata_hash_keys", "hata_decode", "dense_decode", "sk_workspace_bytes", "sk_check_status",
                  "sk_last_error", "sk_version"):
         assert want in names
@@ -128,6 +128,14 @@ def test_host_validation_rejects_without_launching(lib):
     # unknown dtype
     rc, msg = _rc_and_msg(lib, L.dense_decode, p, p, p, 7, 1, 4, 1, 64, 64, 128, 0.1, p, p, 1 << 20, null)
     assert rc == 1 and "dtype" in msg
+    # decode step from host buffers: a missing host buffer, then a missing
+    # workspace, both reported before any copy or launch
+    rc, msg = _rc_and_msg(lib, L.socket_decode_step_host, null, p, p, p, p, p, 1, p, p, p, 1, 4, 1, 64, 64, 128, 8, 4,
+                          0.5, 8, 0.1, p, p, p, 1 << 20, null)
+    assert rc == 1 and "Q_host" in msg
+    rc, msg = _rc_and_msg(lib, L.socket_decode_step_host, p, p, p, p, p, p, 1, p, p, p, 1, 4, 1, 64, 64, 128, 8, 4, 0.5,
+                          8, 0.1, p, p, null, 0, null)
+    assert rc == 5 and "workspace" in msg
 
 
 def test_host_validation_of_the_later_entry_points(lib):

@@ -306,6 +306,43 @@ def test_decode_append_equals_hash_then_decode(api, name):
     assert torch.equal(idx1, idx2) and torch.equal(O1, O2)
 
 
+@pytest.mark.parametrize("name,pinned", [("llama8b_needles", True), ("tiny_f32", True), ("llama8b_needles", False)])
+def test_decode_step_from_host_buffers(api, name, pinned):
+    """socket_decode_step_host copies the query and the new token's K/V rows in
+    from host memory (the rows into position N - 1 of every pair), runs
+    socket_decode_append and copies O out: the cache, the hashed rows and O
+    equal those of the device-resident step bit for bit. Pinned buffers are
+    read and written by a copy kernel; pageable ones by DMA copies."""
+    w = _w(name)
+    inp = wl.make_inputs(w, DEV)
+    Ncap = inp["K"].shape[2]
+    ids = api.empty_ids(w.B, w.Hkv, Ncap, w.L, DEV)
+    nrm = api.empty_norms(w.B, w.Hkv, Ncap, DEV)
+    api.socket_hash_keys(inp["K"], inp["V"], inp["R"], w.L, w.P, ids, nrm, 0, w.N - 1)   # the cache before the step
+    ids2, nrm2 = ids.clone(), nrm.clone()
+    # reference: the rows already in the device cache, the device-resident step
+    O1 = torch.empty(w.B, w.Hq, w.d, device=DEV)
+    api.socket_decode_append(inp["Q"], inp["K"], inp["V"], inp["R"], ids, nrm, w.N, w.L, w.P, w.tau, w.k, w.scale, O1)
+    # the host-buffer step: the cache's row N - 1 and the query start as garbage
+    pin = (lambda t: t.pin_memory()) if pinned else (lambda t: t)
+    q_host = pin(inp["Q"].cpu())
+    k_host = pin(inp["K"][:, :, w.N - 1].contiguous().cpu())
+    v_host = pin(inp["V"][:, :, w.N - 1].contiguous().cpu())
+    K2, V2 = inp["K"].clone(), inp["V"].clone()
+    K2[:, :, w.N - 1] = 7.0
+    V2[:, :, w.N - 1] = -3.0
+    Q2 = torch.full_like(inp["Q"], 5.0)
+    O2 = torch.empty_like(O1)
+    o_host = pin(torch.full((w.B, w.Hq, w.d), float("nan")))
+    api.socket_decode_step_host(q_host, k_host, v_host, Q2, K2, V2, inp["R"], ids2, nrm2, w.N, w.L, w.P, w.tau, w.k,
+                                w.scale, O2, o_host)
+    torch.cuda.synchronize()
+    api.check_status()
+    assert torch.equal(K2, inp["K"]) and torch.equal(V2, inp["V"]) and torch.equal(Q2, inp["Q"])
+    assert torch.equal(ids, ids2) and torch.equal(nrm, nrm2)
+    assert torch.equal(O2, O1) and torch.equal(o_host, O1.cpu())
+
+
 @pytest.mark.parametrize("case", ["all_equal", "all_zero", "above_range"])
 def test_fused_selection_fallback_cases(api, case):
     """Score distributions the binned selection hands to the exact radix path:

@@ -15,13 +15,16 @@
 // as well as keys; integer sums do not depend on the order of the atomics, so
 // the decision is deterministic. Truncation moves a unit's mass by at most
 // one part in 2^62 / (keys), far below the scores' own f32 rounding. Then the
-// plain count-based radix select takes the top k.
+// top k: when k was not clamped, the search's last bin is the k-th largest
+// key itself; otherwise the plain count-based radix select finds it.
 //
 // Shared-memory traffic: a bin's mass is two 32-bit words (low word, high
 // word plus the carry out of the low word), so every histogram update is a
 // native 32-bit atomic; the level-0 key counts are taken while the scores
 // are loaded and serve both the mass search and the top-k; each level of the
-// mass search has bins of its own, so one cluster barrier per level suffices.
+// mass search has bins of its own, so one cluster barrier per level suffices;
+// a level is resolved over groups of 32 bins first, so a CTA reads the other
+// CTAs' group sums and one group's bins, not every bin.
 #pragma once
 
 #include "select.cuh"

@@ -217,9 +217,13 @@ int socket_decode_append(const void* Q, const void* K, const void* V, sk_dtype k
  * every pair of K and V (one strided copy each), runs socket_decode_append
  * over the N keys (SOCKET page, 中核メカニズム：ソフト LSH, steps 1-4: the
  * appended key's hashing, then the selection and the sparse attention), and
- * copies O [B][Hq][d] float32 into O_host. Host buffers in kv's dtype (Q in
- * it too); they should be page-locked (cudaHostAlloc / pinned), so that the
- * copies are asynchronous: O_host holds the result once the stream has
+ * copies O [B][Hq][d] float32 into O_host (O holds it too). Host buffers in
+ * kv's dtype (Q in it too). Page-locked host memory that the device maps
+ * (cudaHostAlloc, pinned tensors), 16-byte aligned, is read and written by a
+ * small copy kernel chained to the step's kernels by programmatic launch;
+ * any other host memory goes through DMA copies. The buffers must hold the
+ * sizes above (the device reads and writes exactly those bytes). All of it
+ * is asynchronous on `stream`: O_host holds the result once the stream has
  * synchronised. Every argument is checked before the first copy, so an
  * error moves and launches nothing. Requires what socket_decode_append
  * requires. ws: sk_workspace_bytes(SK_OP_DECODE, ...) bytes.

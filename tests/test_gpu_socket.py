@@ -35,6 +35,8 @@ def _w(name):
         "qwen_l48_g8": wl.shrink(wl.QWEN3_30B, B=1, Hkv=2, Hq=16, N=10000, k=10000 // 50),
         "d64_g1": wl.shrink(wl.LLAMA_1B, B=2, Hkv=1, Hq=1, N=3000, k=100, L=20, P=6, tau=0.4),
         "g2_small_n": wl.shrink(wl.LLAMA_8B, B=1, Hkv=3, Hq=6, N=70, k=9, needles=0, L=5, P=3, tau=0.7),
+        # 160 pairs: more than one wave of score CTAs, one CTA per pair
+        "many_pairs": wl.shrink(wl.LLAMA_8B, B=10, Hkv=16, Hq=16, N=777, k=25, needles=0, L=8, P=4, tau=0.5),
     }[name]
 
 
@@ -135,7 +137,7 @@ def test_hash_keys_append_touches_only_the_range(api):
 
 # ---------------------------------------------------------------- steps 2-3: scores
 
-@pytest.mark.parametrize("name", ["tiny_f32", "llama1b_ragged", "qwen_l48_g8", "d64_g1", "g2_small_n"])
+@pytest.mark.parametrize("name", ["tiny_f32", "llama1b_ragged", "qwen_l48_g8", "d64_g1", "g2_small_n", "many_pairs"])
 def test_scores_match_oracle(api, name):
     w = _w(name)
     inp = wl.make_inputs(w, DEV)

@@ -679,7 +679,7 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
   const int pair = blockIdx.x, split = blockIdx.y;
   const int G = p.Hq / p.Hkv;
   const int b = pair / p.Hkv, kvh = pair % p.Hkv;
-  const int i0 = split * p.keys_per_split;
+  int i0 = split * p.keys_per_split;
   const size_t pair_keys = (size_t)(pair / p.pair_div) * p.Ncap;
   const KVT* Qg = reinterpret_cast<const KVT*>(p.Q) + (size_t)(b * p.Hq + kvh * G) * D;
   const uint32_t base = smem_u32(dyn);
@@ -707,7 +707,13 @@ __global__ void __launch_bounds__(ATTEND_THREADS) socket_attend_kernel(const Att
   // this unit's list length: n, or its count (clamped to [0, n]) when the
   // lists have per-unit lengths
   const int n_unit = p.counts ? min(max(__ldcg(p.counts + pair), 0), p.n) : p.n;
-  const int cnt = max(0, min(n_unit - i0, p.keys_per_split));
+  int cnt = max(0, min(n_unit - i0, p.keys_per_split));
+  if (p.counts) {
+    // per-unit lengths (planned for the longest): the unit's own keys split
+    // evenly over its splits, so that every split has work
+    i0 = (int)((long long)split * n_unit / p.splits);
+    cnt = (int)((long long)(split + 1) * n_unit / p.splits) - i0;
+  }
   const bool paged = p.page_table != nullptr;
   const size_t key0 = paged ? 0 : pair_keys;            // a paged pool is addressed by physical row
   const KVT* Kp = reinterpret_cast<const KVT*>(p.K) + key0 * D;
